@@ -1,0 +1,14 @@
+"""fp64 CPU oracle for sliding-window / global causal GQA attention with a
+per-head attention-sink logit.
+
+TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference leg may import this package. The product
+library never imports it, and it imports nothing from the product package.
+"""
+from .oracle import (  # noqa: F401
+    decode,
+    kv_commit,
+    prefill,
+    prefill_rows,
+    default_threads,
+)

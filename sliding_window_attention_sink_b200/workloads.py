@@ -1,0 +1,145 @@
+"""Seeded synthetic inputs shaped like the workloads the MiMo pages describe.
+
+This module only draws random numbers and packs them; it holds none of the
+attention arithmetic. Both the CUDA path and the CPU oracle are fed from here,
+so they see identical bytes. Every tensor is made on the CPU with a
+``torch.Generator`` seeded per case; floating inputs are drawn in fp32 and
+rounded to bf16 (round to nearest even); the sink stays fp32.
+
+Shapes (the pages give none of these; they are the workload definitions used
+throughout this package):
+
+* prefill: q [total, Hq, D], k/v [total, Hkv, D] bf16, packed varlen with
+  cu_seqlens [num_seqs + 1] int32 (first entry 0), sink [Hq] fp32.
+* decode: q [B, n_q, Hq, D], k_new/v_new [B, n_q, Hkv, D], ring k/v
+  [B, W, Hkv, D] bf16, pos [B] int32, sink [Hq] fp32.
+"""
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import torch
+
+
+@dataclass
+class PrefillCase:
+    name: str
+    seqlens: List[int]
+    Hq: int
+    Hkv: int
+    D: int
+    window: int            # > 0: sliding window incl. self; <= 0: full causal
+    sigma: float           # q, k, v ~ N(0, 1) * sigma
+    sink: Optional[str]    # "uniform2" (U(-2,2)), "normal" (N(0,1)) or None
+    seed: int
+    varlen_draw: Optional[tuple] = None  # (num_seqs, lo, hi) drawn from seed
+
+
+@dataclass
+class DecodeCase:
+    name: str
+    B: int
+    n_q: int
+    Hq: int
+    Hkv: int
+    D: int
+    W: int
+    sigma: float
+    sink: Optional[str]
+    seed: int
+    pos_lo: int = 128
+    pos_hi: int = 262144   # inclusive
+
+
+# The five workloads: a tiny parity case, one SWA layer, one global layer, a
+# packed varlen SWA batch and a decode / draft-verification batch.
+WORKLOADS = {
+    "tiny_swa_prefill": PrefillCase(
+        "tiny_swa_prefill T=512 Hq=4 Hkv=1 D=64 W=128", [512], 4, 1, 64, 128,
+        1.0, "uniform2", 0),
+    "swa_prefill_32k": PrefillCase(
+        "swa_prefill T=32768 Hq=64 Hkv=8 D=128 W=128", [32768], 64, 8, 128,
+        128, 0.5, "normal", 2),
+    "global_prefill_8k": PrefillCase(
+        "global_prefill T=8192 Hq=64 Hkv=8 D=128 full-causal", [8192], 64, 8,
+        128, 0, 0.5, "normal", 3),
+    "varlen_swa_prefill": PrefillCase(
+        "varlen_swa_prefill 16 seqs L~U[1024,16384] Hq=64 Hkv=8 D=128 W=128",
+        [], 64, 8, 128, 128, 0.5, "normal", 4, varlen_draw=(16, 1024, 16384)),
+    "swa_decode_mtp": DecodeCase(
+        "swa_decode B=256 n_q=4 ring=128 Hq=64 Hkv=8 D=128", 256, 4, 64, 8,
+        128, 128, 0.5, "normal", 5),
+}
+
+
+def _bf16(x: torch.Tensor) -> torch.Tensor:
+    return x.to(torch.bfloat16)
+
+
+def _sink(kind, Hq, g):
+    if kind is None:
+        return None
+    if kind == "uniform2":
+        return torch.rand((Hq,), generator=g, dtype=torch.float32) * 4.0 - 2.0
+    if kind == "normal":
+        return torch.randn((Hq,), generator=g, dtype=torch.float32)
+    raise ValueError(kind)
+
+
+def make_prefill(case: PrefillCase):
+    """Returns a dict of CPU tensors: q, k, v, cu_seqlens, sink, plus sizes."""
+    g = torch.Generator().manual_seed(case.seed)
+    seqlens = list(case.seqlens)
+    if case.varlen_draw is not None:
+        n, lo, hi = case.varlen_draw
+        seqlens = torch.randint(lo, hi + 1, (n,), generator=g).tolist()
+    cu = torch.zeros(len(seqlens) + 1, dtype=torch.int32)
+    if seqlens:
+        cu[1:] = torch.cumsum(torch.tensor(seqlens, dtype=torch.int64), 0).to(torch.int32)
+    total = int(cu[-1])
+    q = _bf16(torch.randn((total, case.Hq, case.D), generator=g) * case.sigma)
+    k = _bf16(torch.randn((total, case.Hkv, case.D), generator=g) * case.sigma)
+    v = _bf16(torch.randn((total, case.Hkv, case.D), generator=g) * case.sigma)
+    sink = _sink(case.sink, case.Hq, g)
+    return dict(q=q, k=k, v=v, cu_seqlens=cu, sink=sink, seqlens=seqlens,
+                total=total, Hq=case.Hq, Hkv=case.Hkv, D=case.D,
+                window=case.window, max_seqlen=max(seqlens) if seqlens else 0)
+
+
+def make_decode(case: DecodeCase):
+    """Returns a dict of CPU tensors for one decode / verification step."""
+    g = torch.Generator().manual_seed(case.seed)
+    pos = torch.randint(case.pos_lo, case.pos_hi + 1, (case.B,), generator=g,
+                        dtype=torch.int64).to(torch.int32)
+    s = case.sigma
+    q = _bf16(torch.randn((case.B, case.n_q, case.Hq, case.D), generator=g) * s)
+    k_new = _bf16(torch.randn((case.B, case.n_q, case.Hkv, case.D), generator=g) * s)
+    v_new = _bf16(torch.randn((case.B, case.n_q, case.Hkv, case.D), generator=g) * s)
+    k_ring = _bf16(torch.randn((case.B, case.W, case.Hkv, case.D), generator=g) * s)
+    v_ring = _bf16(torch.randn((case.B, case.W, case.Hkv, case.D), generator=g) * s)
+    sink = _sink(case.sink, case.Hq, g)
+    return dict(q=q, k_new=k_new, v_new=v_new, k_ring=k_ring, v_ring=v_ring,
+                pos=pos, sink=sink, B=case.B, n_q=case.n_q, Hq=case.Hq,
+                Hkv=case.Hkv, D=case.D, W=case.W)
+
+
+def prefill_case(seqlens, Hq, Hkv, D, window, sigma=0.5, sink="normal", seed=0):
+    """An ad-hoc prefill case (tests use it for edge shapes)."""
+    return make_prefill(PrefillCase("adhoc", list(seqlens), Hq, Hkv, D, window,
+                                    sigma, sink, seed))
+
+
+def decode_case(B, n_q, Hq, Hkv, D, W, sigma=0.5, sink="normal", seed=0,
+                pos_lo=128, pos_hi=262144):
+    return make_decode(DecodeCase("adhoc", B, n_q, Hq, Hkv, D, W, sigma, sink,
+                                  seed, pos_lo, pos_hi))
+
+
+def shard_units(num_units: int, world_size: int, rank: int):
+    """Contiguous block split of independent units (sequences, decode rows)
+    over ranks: rank r gets [lo, hi). Sizes differ by at most one."""
+    if world_size <= 0 or not (0 <= rank < world_size):
+        raise ValueError("bad rank / world size")
+    base, extra = divmod(num_units, world_size)
+    lo = rank * base + min(rank, extra)
+    hi = lo + base + (1 if rank < extra else 0)
+    return lo, hi
