@@ -1,0 +1,513 @@
+"""Benchmark of the sliding-window / global attention with a per-head sink on
+B200, through the C ABI of libswasink.so.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+One JSON line on rank 0. A step is one call of the hot path over the
+workload's whole batch (default: one SWA layer, T=32768, Hq=64, Hkv=8, D=128,
+W=128). `value` is whole-job throughput from CUDA events with the inputs
+resident in HBM; `e2e` adds the host->device copy of the inputs from pinned
+memory and the device->host copy of the outputs, per step. With N > 1 (one
+process per GPU under torch.distributed.run) every rank runs its own replica
+of the workload on its own seeded inputs (independent sequences: no
+collective on the data path), timing is the max over ranks, and `value`
+counts the work of all ranks (weak scaling).
+
+`--impl reference` times the fp64 CPU oracle instead, on bounded samples of
+the same workload (rank 0 only; the other ranks exit at once).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SWA+sink attention TFLOP/s (prefill), GB/s (decode); % of 1×B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- work model --
+def prefill_work(seqlens, Hq, Hkv, D, window):
+    """Algorithmic FLOPs and bytes of one prefill call: FLOPs = 4*D*Hq*pairs
+    (QK^T and PV over the visible (query, key) pairs; softmax not counted);
+    bytes = read q, k, v, sink, cu_seqlens once + write o, lse once."""
+    pairs = 0
+    for L in seqlens:
+        if window > 0 and window < L:
+            pairs += window * (window + 1) // 2 + (L - window) * window
+        else:
+            pairs += L * (L + 1) // 2
+    total = sum(seqlens)
+    flops = 4 * D * Hq * pairs
+    nbytes = (total * Hq * D * 2 * 2          # q read, o write
+              + total * Hkv * D * 2 * 2      # k, v read
+              + Hq * total * 4               # lse write
+              + Hq * 4 + (len(seqlens) + 1) * 4)
+    return flops, nbytes
+
+
+def decode_work(pos, n_q, Hq, Hkv, D, W):
+    """FLOPs over visible pairs; bytes = ring K/V + new K/V + q + pos + sink
+    read once, o + lse written once."""
+    pairs = 0
+    for P in pos:
+        for t in range(n_q):
+            pairs += min(P, W - 1 - t) + (t + 1)   # ring keys + new keys 0..t
+    B = len(pos)
+    flops = 4 * D * Hq * pairs
+    nbytes = (B * W * Hkv * D * 2 * 2 + B * n_q * Hkv * D * 2 * 2
+              + B * n_q * Hq * D * 2 * 2 + B * n_q * Hq * 4 + B * 4 + Hq * 4)
+    return flops, nbytes
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sliding_window_attention_sink_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path)).get(workload)
+    except Exception:
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# -------------------------------------------------------------------- clocks --
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of this process's GPU during the timed region."""
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workloads --
+class PrefillRunner:
+    def __init__(self, case, rank, torch, B, wl):
+        self.torch, self.B = torch, B
+        case = wl.PrefillCase(**{**case.__dict__, "seed": case.seed + 1000 * rank})
+        c = wl.make_prefill(case)
+        self.c = c
+        self.flops, self.bytes = prefill_work(c["seqlens"], c["Hq"], c["Hkv"], c["D"],
+                                              c["window"])
+        dev = torch.device("cuda")
+        self.q, self.k, self.v = c["q"].to(dev), c["k"].to(dev), c["v"].to(dev)
+        self.cu = c["cu_seqlens"].to(dev)
+        self.sink = c["sink"].to(dev) if c["sink"] is not None else None
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((c["Hq"], c["total"]), dtype=torch.float32, device=dev)
+        # pinned host copies for the end-to-end leg
+        self.h_in = [c["q"].pin_memory(), c["k"].pin_memory(), c["v"].pin_memory(),
+                     c["cu_seqlens"].pin_memory()]
+        self.d_in = [self.q, self.k, self.v, self.cu]
+        if c["sink"] is not None:
+            self.h_in.append(c["sink"].pin_memory())
+            self.d_in.append(self.sink)
+        self.h_out = [torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory(),
+                      torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()]
+        self.d_out = [self.o, self.lse]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+        self.units = c["total"]
+
+    def call(self, stream):
+        c = self.c
+        rc = self.B.swa_sink_attn_fwd(self.q, self.k, self.v, self.cu, len(c["seqlens"]),
+                                      c["max_seqlen"], c["total"], c["Hq"], c["Hkv"], c["D"],
+                                      c["window"], self.sink, 0.0, self.o, self.lse, stream)
+        if rc != 0:
+            raise RuntimeError("swa_sink_attn_fwd: %s" % self.B.status_string(rc))
+
+    def describe(self):
+        c = self.c
+        return {"Hq": c["Hq"], "Hkv": c["Hkv"], "head_dim": c["D"], "window": c["window"],
+                "num_seqs": len(c["seqlens"]), "tokens": c["total"]}
+
+
+class DecodeRunner:
+    """The decode batch reads ~170 MB, close to the 126 MB L2, so the timed
+    steps rotate over three independent input sets (> 500 MB together)."""
+    NSETS = 3
+
+    def __init__(self, case, rank, torch, B, wl):
+        self.torch, self.B = torch, B
+        case = wl.DecodeCase(**{**case.__dict__, "seed": case.seed + 1000 * rank})
+        d = wl.make_decode(case)
+        self.d = d
+        self.flops, self.bytes = decode_work(d["pos"].tolist(), d["n_q"], d["Hq"], d["Hkv"],
+                                             d["D"], d["W"])
+        dev = torch.device("cuda")
+        names = ["q", "k_new", "v_new", "k_ring", "v_ring", "pos", "sink"]
+        self.g = {n: d[n].to(dev) for n in names}
+        self.sets = [self.g] + [{n: (t.clone() if n != "pos" else t) for n, t in self.g.items()}
+                                for _ in range(self.NSETS - 1)]
+        self.turn = 0
+        self.o = torch.empty_like(self.g["q"])
+        self.lse = torch.empty((d["B"], d["n_q"], d["Hq"]), dtype=torch.float32, device=dev)
+        self.h_in = [d[n].pin_memory() for n in names]
+        self.d_in = [self.g[n] for n in names]
+        self.h_out = [torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory(),
+                      torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()]
+        self.d_out = [self.o, self.lse]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+        self.units = d["B"]
+
+    def call(self, stream):
+        d, g = self.d, self.sets[self.turn]
+        self.turn = (self.turn + 1) % self.NSETS
+        rc = self.B.swa_sink_attn_decode(g["q"], g["k_new"], g["v_new"], g["k_ring"],
+                                         g["v_ring"], g["pos"], d["B"], d["n_q"], d["Hq"],
+                                         d["Hkv"], d["D"], d["W"], g["sink"], 0.0, self.o,
+                                         self.lse, stream)
+        if rc != 0:
+            raise RuntimeError("swa_sink_attn_decode: %s" % self.B.status_string(rc))
+
+    def describe(self):
+        d = self.d
+        return {"batch": d["B"], "n_q": d["n_q"], "Hq": d["Hq"], "Hkv": d["Hkv"],
+                "head_dim": d["D"], "ring": d["W"]}
+
+
+# ------------------------------------------------------------ oracle timing --
+_INPUTS = {}
+
+
+def _cached_inputs(workload, wl):
+    if workload not in _INPUTS:
+        case = wl.WORKLOADS[workload]
+        _INPUTS[workload] = (wl.make_prefill(case) if isinstance(case, wl.PrefillCase)
+                             else wl.make_decode(case))
+    return _INPUTS[workload]
+
+
+def oracle_sample(workload, wl, seconds, threads, seed=0):
+    """Time the fp64 oracle on a bounded sample of the workload. Returns
+    (flops_done, bytes_equiv, elapsed_s, description)."""
+    import numpy as np
+    import oracle
+    case = wl.WORKLOADS[workload]
+    rng = np.random.default_rng(seed)
+    if isinstance(case, wl.PrefillCase):
+        c = _cached_inputs(workload, wl)
+        F, Bt = prefill_work(c["seqlens"], c["Hq"], c["Hkv"], c["D"], c["window"])
+        total_rows = c["total"] * c["Hq"]
+
+        def run(n):
+            rt = rng.integers(0, c["total"], n)
+            rh = rng.integers(0, c["Hq"], n).astype(np.int32)
+            t0 = time.perf_counter()
+            oracle.prefill_rows(c["q"], c["k"], c["v"], c["cu_seqlens"], c["Hq"], c["Hkv"],
+                                c["D"], c["window"], rt, rh, sink=c["sink"], nthreads=threads)
+            return time.perf_counter() - t0
+        unit = "random (token, head) rows"
+    else:
+        d = _cached_inputs(workload, wl)
+        F, Bt = decode_work(d["pos"].tolist(), d["n_q"], d["Hq"], d["Hkv"], d["D"], d["W"])
+        total_rows = d["B"]
+
+        def run(n):
+            idx = np.sort(rng.choice(d["B"], size=min(n, d["B"]), replace=False))
+            sub = {k: (d[k][idx] if k in ("q", "k_new", "v_new", "k_ring", "v_ring", "pos")
+                       else d[k]) for k in d}
+            t0 = time.perf_counter()
+            oracle.decode(sub["q"], sub["k_new"], sub["v_new"], sub["k_ring"], sub["v_ring"],
+                          sub["pos"], len(idx), d["n_q"], d["Hq"], d["Hkv"], d["D"], d["W"],
+                          sink=d["sink"], nthreads=threads)
+            return time.perf_counter() - t0
+        unit = "sequences"
+    # calibrate on a small sample, then size the timed sample to `seconds`
+    n0 = max(1, min(total_rows, 2000 if unit != "sequences" else 4))
+    t_cal = run(n0)
+    n = int(min(total_rows, max(n0, n0 * seconds / max(t_cal, 1e-3))))
+    elapsed = run(n)
+    frac = n / total_rows
+    return F * frac, Bt * frac, elapsed, "%d of %d %s of %s, %d threads" % (
+        n, total_rows, unit, workload, threads)
+
+
+def run_reference(args, wl):
+    """The reference arm: the fp64 CPU oracle as it stands, on bounded samples."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    threads = oracle.default_threads()
+    case = wl.WORKLOADS[args.workload]
+    is_prefill = isinstance(case, wl.PrefillCase)
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(args.workload, wl, per_step / 4, threads)
+    flops = nb = el = 0.0
+    desc = ""
+    for s in range(args.steps):
+        f, b, e, desc = oracle_sample(args.workload, wl, per_step, threads, seed=s + 1)
+        flops += f
+        nb += b
+        el += e
+    value = flops / el / 1e12 if is_prefill else nb / el / 1e9
+    unit = "TFLOP/s" if is_prefill else "GB/s"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": case.name, "impl_note": "fp64 CPU oracle, bounded samples"},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------- main --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="swa_prefill_32k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    from sliding_window_attention_sink_b200 import workloads as wl
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from sliding_window_attention_sink_b200 import binding as B
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    B.load()
+
+    case = wl.WORKLOADS[args.workload]
+    is_prefill = isinstance(case, wl.PrefillCase)
+    runner = (PrefillRunner if is_prefill else DecodeRunner)(case, rank, torch, B, wl)
+    stream = torch.cuda.Stream()
+    sptr = stream.cuda_stream
+
+    # CPU baseline (rank 0, N = 1), before the GPU timing so it does not overlap
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        threads = oracle.default_threads()
+        f, b, e, desc = oracle_sample(args.workload, wl, args.cpu_seconds, threads)
+        cpu = {"value": (f / e / 1e12) if is_prefill else (b / e / 1e9),
+               "unit": "TFLOP/s" if is_prefill else "GB/s", "cores": threads,
+               "kind": "oracle", "sample": desc + ", %.1f s" % e}
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # warm-up
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            runner.call(sptr)
+    barrier()
+
+    # timed region: K steps, one launch each, events around every launch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        barrier()
+        with torch.cuda.stream(stream):
+            t_start.record(stream)
+            for s in range(args.steps):
+                ev[s][0].record(stream)
+                runner.call(sptr)
+                ev[s][1].record(stream)
+            t_end.record(stream)
+        barrier()
+        time.sleep(0.3)
+    total_ms = t_start.elapsed_time(t_end)
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    kern_avg = sum(kern_ms) / len(kern_ms)
+
+    # end to end: pinned host inputs -> device, the call, outputs -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        e_steps = max(3, min(args.steps, 10))
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                if hasattr(runner, "turn"):
+                    runner.turn = 0
+                for h, dd in zip(runner.h_in, runner.d_in):
+                    dd.copy_(h, non_blocking=True)
+                runner.call(sptr)
+                for h, dd in zip(runner.h_out, runner.d_out):
+                    h.copy_(dd, non_blocking=True)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            for _ in range(e_steps):
+                if hasattr(runner, "turn"):
+                    runner.turn = 0   # the copies below refill input set 0
+                for h, dd in zip(runner.h_in, runner.d_in):
+                    dd.copy_(h, non_blocking=True)
+                runner.call(sptr)
+                for h, dd in zip(runner.h_out, runner.d_out):
+                    h.copy_(dd, non_blocking=True)
+            b.record(stream)
+        barrier()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e_step = e_ms / e_steps
+        e_val = (runner.flops * world / (e_step * 1e-3) / 1e12) if is_prefill else (
+            runner.bytes * world / (e_step * 1e-3) / 1e9)
+        e2e = {"value": e_val, "unit": "TFLOP/s" if is_prefill else "GB/s",
+               "ms_per_step": e_step, "h2d_bytes_per_step": runner.h2d * world,
+               "d2h_bytes_per_step": runner.d2h * world}
+
+    flag = B.swa_sink_device_error()
+    peaks, src = load_peaks()
+    if is_prefill:
+        value = runner.flops * world / (ms_per_step * 1e-3) / 1e12
+        unit = "TFLOP/s"
+    else:
+        value = runner.bytes * world / (ms_per_step * 1e-3) / 1e9
+        unit = "GB/s"
+    # roofline of the (only) kernel in the step: the slower of tensor and HBM time
+    t_tensor = runner.flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = runner.bytes / (peaks["hbm_gbs"] * 1e9)
+    if t_hbm >= t_tensor:
+        achieved = runner.bytes / (kern_avg * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        achieved = runner.flops / (kern_avg * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
+    roof["peak_source"] = src
+    roof["algorithmic_bytes"] = runner.bytes
+    roof["algorithmic_flops"] = runner.flops
+    roof["kernel_ms"] = kern_avg
+    roof["traffic"] = recorded_traffic(args.workload)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": dict({"workload": case.name,
+                            "parallelism": "replicas" if world == 1 else "dp%d" % world,
+                            "l2": ("inputs larger than L2 (%.0f MB per step)" %
+                                   (runner.bytes / 1e6))},
+                           **runner.describe()),
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps, "clocks": clk.summary(), "device_error_flags": flag,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

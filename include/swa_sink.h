@@ -1,0 +1,163 @@
+/*
+ * swa_sink.h -- C ABI of libswasink.so: causal GQA attention over a sliding
+ * window (or the full prefix) with a per-head learnable attention-sink logit,
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operation (one query row i of query head h; kv head g = h / (Hq/Hkv)):
+ *
+ *   a_j  = scale * (q_i . k_j)            over the visible keys j
+ *   m    = max(s_h, max_j a_j)
+ *   den  = exp(s_h - m) + sum_j exp(a_j - m)
+ *   o_i  = sum_j exp(a_j - m) / den * v_j  (the sink carries no value)
+ *   lse  = m + ln(den)                     (natural log, sink included)
+ *
+ * Source: "MiMo-V2-Flash Technical Report" summary (mlpod.com), section 2.2.2
+ * "Learnable Attention Sink Bias" (a learnable term in the softmax denominator
+ * that lets a row attend to a virtual sink; a max term for stability; the
+ * page's equations are stripped, the above is the plain reading of its prose),
+ * and section 2.2.1 / TL;DR (window of 128 tokens; SWA and global layers
+ * interleaved 5:1). The MiMo-V2 blog review (kokolerk.github.io), section 2.2,
+ * states the same sink term. Visible keys for query i: i-W+1 <= j <= i within
+ * its own sequence (W keys including itself; the pages do not say whether the
+ * query counts, this is the reading taken); W <= 0 means the full causal prefix
+ * (the global-attention layers).
+ *
+ * Conventions for every call
+ * --------------------------
+ * - All array pointers are DEVICE pointers owned by the caller; the library
+ *   allocates no memory and keeps no per-call state. bf16 arrays must be
+ *   16-byte aligned (TMA and 16-byte vector loads); int32/fp32 arrays 4-byte.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Every call is asynchronous on that stream; the caller synchronises.
+ * - Argument errors are returned as a negative status BEFORE anything is
+ *   launched; nothing is written then. A failed launch returns SWA_ERR_CUDA.
+ * - The kernels never trap or assert. Each device-side wait has a time limit
+ *   (about 2 s); if one expires, or a device-resident argument is out of range
+ *   (a negative pos, an n_accept outside [0, n_q]), the kernel records a flag
+ *   readable with swa_sink_device_error() and returns.
+ * - Thread-safe: no global mutable host state except a per-device cache of
+ *   the driver entry point, filled once under a lock.
+ */
+#ifndef SWA_SINK_H
+#define SWA_SINK_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SWA_API __attribute__((visibility("default")))
+#else
+#define SWA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SWA_OK = 0,
+    SWA_ERR_NULL = -1,        /* a required pointer is NULL                  */
+    SWA_ERR_SHAPE = -2,       /* a size is negative or inconsistent          */
+    SWA_ERR_UNSUPPORTED = -3, /* valid but not supported (e.g. head_dim 96)  */
+    SWA_ERR_ALIGN = -4,       /* a pointer is not aligned as required        */
+    SWA_ERR_CUDA = -5         /* a CUDA runtime/driver call failed           */
+} swa_status_t;
+
+/*
+ * Packed varlen prefill (self-attention, queries and keys share cu_seqlens).
+ *
+ * Source: section 2.2 of the report summary above (Hybrid SWA: sliding-window
+ * layers with W = 128 and global layers), section 2.2.2 (the sink).
+ *
+ *   q           bf16 [total_tokens, Hq, D], row-major (token, head, dim)
+ *   k, v        bf16 [total_tokens, Hkv, D]
+ *   cu_seqlens  int32 [num_seqs + 1], device; cu_seqlens[0] = 0,
+ *               non-decreasing, cu_seqlens[num_seqs] = total_tokens.
+ *               Zero-length sequences are allowed. The host does not read it.
+ *   max_seqlen  an upper bound on any sequence length (>= 0); used only to
+ *               check sizes.
+ *   Hq, Hkv     query / kv heads; Hkv divides Hq; Hq/Hkv <= 128.
+ *               Query head h reads kv head h / (Hq/Hkv).
+ *   D           head dim: 64 or 128.
+ *   window      > 0: key j visible to query i iff i-window+1 <= j <= i;
+ *               <= 0: full causal prefix.
+ *   sink        fp32 [Hq] device, or NULL for no sink (s_h = -inf).
+ *   softmax_scale  <= 0 selects 1/sqrt(D). The sink is not scaled.
+ *   o           bf16 [total_tokens, Hq, D] output (round to nearest even).
+ *   lse         fp32 [Hq, total_tokens] output in natural-log units, or NULL.
+ *
+ * Returns SWA_OK or a negative swa_status_t.
+ */
+SWA_API int swa_sink_attn_fwd(const void *q, const void *k, const void *v,
+                      const int32_t *cu_seqlens, int num_seqs, int max_seqlen,
+                      int total_tokens, int Hq, int Hkv, int D, int window,
+                      const float *sink, float softmax_scale, void *o,
+                      float *lse, void *stream);
+
+/*
+ * Decode / draft verification over a W-slot KV ring per sequence.
+ *
+ * Source: section 2.3 "Lightweight MTP" of the report summary above (draft
+ * tokens from the MTP layers are verified by the main model in parallel,
+ * raising arithmetic intensity without more KV-cache I/O), section 2.2.1
+ * (SWA keeps a constant window of W tokens), and the Q&A of the ICML 2026
+ * talk write-up (hzrcw.cc): positions keep increasing while the window slides.
+ *
+ * Sequence b has n_q new tokens at absolute positions pos[b] .. pos[b]+n_q-1
+ * (1 real token + n_q-1 drafts). The ring holds the committed tokens at
+ * positions pos[b]-W .. pos[b]-1, the token at position p in slot p mod W;
+ * slots whose position would be negative are ignored. Query t sees the ring
+ * tokens at positions >= pos[b]+t-W+1 and the new tokens 0..t (causal among
+ * themselves). The ring is read-only here (see swa_sink_kv_commit).
+ *
+ *   q             bf16 [B, n_q, Hq, D]
+ *   k_new, v_new  bf16 [B, n_q, Hkv, D]   keys/values of the new tokens
+ *   k_ring,v_ring bf16 [B, W, Hkv, D]
+ *   pos           int32 [B] device, >= 0 (a negative entry is treated as 0
+ *                 and flagged)
+ *   n_q           1..8;  W: 1..256;  D: 64 or 128;  n_q*(Hq/Hkv) <= 32.
+ *   sink, softmax_scale  as for swa_sink_attn_fwd.
+ *   o             bf16 [B, n_q, Hq, D]
+ *   lse           fp32 [B, n_q, Hq] (natural log), or NULL.
+ */
+SWA_API int swa_sink_attn_decode(const void *q, const void *k_new, const void *v_new,
+                         const void *k_ring, const void *v_ring,
+                         const int32_t *pos, int B, int n_q, int Hq, int Hkv,
+                         int D, int W, const float *sink, float softmax_scale,
+                         void *o, float *lse, void *stream);
+
+/*
+ * Commit accepted tokens into the ring after verification: for
+ * u < n_accept[b], new token u (absolute position pos[b]+u) is copied into
+ * slot (pos[b]+u) mod W of k_ring / v_ring. pos is not modified; the caller
+ * advances it by n_accept. An n_accept[b] outside [0, n_q] is clamped and
+ * flagged. Source: section 2.3 of the report summary above (only verified
+ * draft tokens become part of the sequence).
+ *
+ *   k_ring, v_ring bf16 [B, W, Hkv, D] (updated in place)
+ *   k_new, v_new   bf16 [B, n_q, Hkv, D]
+ *   pos, n_accept  int32 [B] device
+ */
+SWA_API int swa_sink_kv_commit(void *k_ring, void *v_ring, const void *k_new,
+                       const void *v_new, const int32_t *pos,
+                       const int32_t *n_accept, int B, int n_q, int Hkv, int D,
+                       int W, void *stream);
+
+/* Human-readable text for a swa_status_t (static storage). */
+SWA_API const char *swa_sink_status_string(int status);
+
+/*
+ * Device-side error flags recorded by kernels on the CURRENT device since the
+ * last clear: bit 0 = a wait timed out, bit 1 = a device-resident argument
+ * was out of range. Synchronises the device. *flags receives the bits; if
+ * clear != 0 they are reset. Returns SWA_OK or SWA_ERR_CUDA.
+ */
+SWA_API int swa_sink_device_error(unsigned int *flags, int clear);
+
+/* Library ABI version (major * 100 + minor). */
+SWA_API int swa_sink_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_SINK_H */

@@ -1,0 +1,408 @@
+// decode_sm100.cuh -- decode / draft verification over a W-slot KV ring, and
+// the commit of accepted tokens into the ring.
+//
+// Operation: the same sink attention as the prefill ("MiMo-V2-Flash Technical
+// Report" summary, mlpod.com, section 2.2.2), for n_q new tokens per sequence:
+// one real token plus the drafts of the MTP layers, verified in parallel
+// (section 2.3 "Lightweight MTP": verification raises arithmetic intensity
+// without adding KV-cache I/O). New token t at absolute position P + t sees
+// the committed tokens at positions >= P + t - W + 1 (slot p mod W of the
+// ring) and the new tokens 0..t.
+//
+// Design (sm_100a): one CTA of 4 warps per (sequence, kv head); split-free.
+// * All G query heads of the kv head and all n_q tokens are one set of
+//   R = n_q * G query rows (32 for n_q = 4, G = 8), so each ring byte is read
+//   from HBM exactly once for all of them.
+// * The ring slice (W rows of D bf16, 2 KB apart in HBM) and the new rows go
+//   to shared memory with 16-byte cp.async; keys first, values in a second
+//   group that lands while the scores are computed.
+// * The contraction has ~25 flop per HBM byte, above what CUDA-core FMAs hide,
+//   so S = Q K^T and O = P V use the tensor cores through mma.sync m16n8k16
+//   (bf16, f32 accumulate); the tiles (32 rows) are too small for tcgen05.
+// * Softmax: the 4 warps split the keys for S; row maxima and sums are
+//   reduced inside the quad that shares a row (warp shuffles), then across
+//   warps through shared memory. The max is seeded with the sink logit and
+//   the denominator gets the sink term exp(s - m). P goes to shared memory as
+//   bf16; the 4 warps then split the head dim for O = P V.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx_sm100.cuh"
+
+namespace swa {
+
+struct DecodeParams {
+  const __nv_bfloat16 *q, *k_new, *v_new, *k_ring, *v_ring;
+  const int32_t* pos;
+  int B, n_q, Hq, Hkv, G, W;
+  int R;    // query rows per CTA = n_q * G (<= 32)
+  int KP;   // keys padded to a multiple of 16: roundup16(W + n_q)
+  const float* sink;
+  float scale_log2;
+  __nv_bfloat16* o;
+  float* lse;
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void st_shared_zero16(uint32_t dst) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                        uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                          uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                          uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Shared memory: K and V [KP][D+8], Q [32][D+8], P [32][KP+8] (bf16),
+// then per-warp row maxima and two row sums [4][32] and per-row l [32] (fp32).
+__host__ __device__ constexpr int decode_row_stride(int D) { return D + 8; }
+__host__ __device__ inline size_t decode_smem_bytes(int D, int KP) {
+  const int ld = decode_row_stride(D);
+  return static_cast<size_t>(2 * KP * ld + 32 * ld + 32 * (KP + 8)) * 2 +
+         (4 * 32 * 3 + 32) * sizeof(float);
+}
+
+template <int D, int MT>
+__global__ void __launch_bounds__(128)
+    decode_sm100_kernel(const DecodeParams p) {
+  constexpr int LD = D + 8;        // bf16 elements per smem row (conflict-free ldmatrix)
+  constexpr int CPR = D / 8;       // 16-byte chunks per row
+  constexpr int RP = MT * 16;      // padded query rows
+  constexpr int NTW = 9;           // max n8 key tiles per warp (KP <= 272)
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int KP = p.KP;
+  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smem_raw);
+  __nv_bfloat16* Vs = Ks + KP * LD;
+  __nv_bfloat16* Qs = Vs + KP * LD;
+  __nv_bfloat16* Ps = Qs + 32 * LD;
+  const int LDP = KP + 8;
+  float* red_max = reinterpret_cast<float*>(Ps + 32 * LDP);  // [4][32]
+  float* red_sum = red_max + 4 * 32;                          // [4][32]
+  float* red_sum_x = red_sum + 4 * 32;                        // [4][32]
+  float* row_l = red_sum_x + 4 * 32;                          // [32]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.x / p.Hkv;
+  const int g = blockIdx.x - b * p.Hkv;
+  int P = __ldg(p.pos + b);
+  if (P < 0) {
+    if (tid == 0) flag_error(2u);
+    P = 0;
+  }
+  const int W = p.W, n_q = p.n_q, G = p.G;
+
+  // ---- loads: group 0 = Q and K rows, group 1 = V rows ---------------------
+  const uint32_t sQ = smem_u32(Qs), sK = smem_u32(Ks), sV = smem_u32(Vs);
+  for (int idx = tid; idx < RP * CPR; idx += 128) {
+    const int r = idx / CPR, c = idx - r * CPR;
+    const uint32_t dst = sQ + (r * LD + c * 8) * 2;
+    if (r < p.R) {
+      const int t = r / G, hh = r - t * G;
+      cp_async16(dst, p.q + ((static_cast<size_t>(b) * n_q + t) * p.Hq + g * G + hh) * D + c * 8);
+    } else {
+      st_shared_zero16(dst);
+    }
+  }
+  for (int idx = tid; idx < KP * CPR; idx += 128) {
+    const int key = idx / CPR, c = idx - key * CPR;
+    const uint32_t dst = sK + (key * LD + c * 8) * 2;
+    if (key < W)
+      cp_async16(dst, p.k_ring + ((static_cast<size_t>(b) * W + key) * p.Hkv + g) * D + c * 8);
+    else if (key < W + n_q)
+      cp_async16(dst, p.k_new + ((static_cast<size_t>(b) * n_q + key - W) * p.Hkv + g) * D + c * 8);
+    else
+      st_shared_zero16(dst);
+  }
+  cp_async_commit();
+  for (int idx = tid; idx < KP * CPR; idx += 128) {
+    const int key = idx / CPR, c = idx - key * CPR;
+    const uint32_t dst = sV + (key * LD + c * 8) * 2;
+    if (key < W)
+      cp_async16(dst, p.v_ring + ((static_cast<size_t>(b) * W + key) * p.Hkv + g) * D + c * 8);
+    else if (key < W + n_q)
+      cp_async16(dst, p.v_new + ((static_cast<size_t>(b) * n_q + key - W) * p.Hkv + g) * D + c * 8);
+    else
+      st_shared_zero16(dst);
+  }
+  cp_async_commit();
+  cp_async_wait<1>();
+  __syncthreads();
+
+  // ---- S = Q K^T: warp w takes key tiles w, w+4, w+8, ... ------------------
+  const int NT = KP / 8;
+  float s[MT][NTW][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int j = 0; j < NTW; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[mt][j][e] = 0.f;
+
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint32_t a[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int row = mt * 16 + (lane & 15);
+      const int col = kk * 16 + (lane >> 4) * 8;
+      ldsm_x4(sQ + (row * LD + col) * 2, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
+    }
+#pragma unroll
+    for (int j = 0; j < NTW; ++j) {
+      const int nt = warp + 4 * j;
+      if (nt < NT) {
+        uint32_t b0, b1;
+        const int key = nt * 8 + (lane & 7);
+        const int col = kk * 16 + ((lane >> 3) & 1) * 8;
+        ldsm_x2(sK + (key * LD + col) * 2, b0, b1);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+          mma_16816(s[mt][j], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
+      }
+    }
+  }
+
+  // ---- mask, scale to log2 units, per-warp row max -------------------------
+  const int Pmod = P % W;
+  float mloc[MT][2];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    mloc[mt][0] = -INFINITY;
+    mloc[mt][1] = -INFINITY;
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+    for (int j = 0; j < NTW; ++j) {
+      const int nt = warp + 4 * j;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = mt * 16 + (lane >> 2) + ((e >> 1) << 3);
+        const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
+        bool vis = false;
+        if (nt < NT && row < p.R) {
+          const int t = row / G;
+          if (col < W) {
+            int rel = col - Pmod;
+            if (rel < 0) rel += W;
+            const int pos_key = P - W + rel;  // absolute position held by slot col
+            vis = pos_key >= 0 && pos_key >= P + t - W + 1;
+          } else if (col < W + n_q) {
+            vis = (col - W) <= t;
+          }
+        }
+        const float x = vis ? s[mt][j][e] * p.scale_log2 : -INFINITY;
+        s[mt][j][e] = x;
+        mloc[mt][e >> 1] = fmaxf(mloc[mt][e >> 1], x);
+      }
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      float v = mloc[mt][hf];
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+      if ((lane & 3) == 0) red_max[warp * 32 + mt * 16 + (lane >> 2) + hf * 8] = v;
+    }
+  __syncthreads();
+
+  // ---- row max over warps and the sink; P = exp2(x - m) -> smem; row sums --
+  float mrow[MT][2];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int row = mt * 16 + (lane >> 2) + hf * 8;
+      float m = -INFINITY;
+      if (row < p.R && p.sink != nullptr) m = __ldg(p.sink + g * G + row % G) * kLog2e;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) m = fmaxf(m, red_max[w * 32 + row]);
+      mrow[mt][hf] = (m == -INFINITY) ? 0.f : m;
+    }
+  // lloc sums P as rounded to bf16 (normalises O consistently with the PV
+  // product); lexact sums it in fp32 (for the LSE).
+  float lloc[MT][2], lexact[MT][2];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    lloc[mt][0] = lloc[mt][1] = 0.f;
+    lexact[mt][0] = lexact[mt][1] = 0.f;
+  }
+  const uint32_t sP = smem_u32(Ps);
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+    for (int j = 0; j < NTW; ++j) {
+      const int nt = warp + 4 * j;
+      if (nt < NT) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int row = mt * 16 + (lane >> 2) + hf * 8;
+          const int col = nt * 8 + 2 * (lane & 3);
+          const float p0 = ex2(s[mt][j][2 * hf] - mrow[mt][hf]);
+          const float p1 = ex2(s[mt][j][2 * hf + 1] - mrow[mt][hf]);
+          const uint32_t pk = pack_bf16x2(p0, p1);
+          lloc[mt][hf] += bf16lo_to_f32(pk) + bf16hi_to_f32(pk);
+          lexact[mt][hf] += p0 + p1;
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sP + (row * LDP + col) * 2), "r"(pk)
+                       : "memory");
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      float v = lloc[mt][hf], x = lexact[mt][hf];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
+      if ((lane & 3) == 0) {
+        red_sum[warp * 32 + mt * 16 + (lane >> 2) + hf * 8] = v;
+        red_sum_x[warp * 32 + mt * 16 + (lane >> 2) + hf * 8] = x;
+      }
+    }
+  cp_async_wait<0>();
+  __syncthreads();
+  if (tid < RP) {
+    const int row = tid;
+    float m = -INFINITY;
+    if (row < p.R && p.sink != nullptr) m = __ldg(p.sink + g * G + row % G) * kLog2e;
+    for (int w = 0; w < 4; ++w) m = fmaxf(m, red_max[w * 32 + row]);
+    const float mb = (m == -INFINITY) ? 0.f : m;
+    float l = 0.f, lx = 0.f;
+    for (int w = 0; w < 4; ++w) {
+      l += red_sum[w * 32 + row];
+      lx += red_sum_x[w * 32 + row];
+    }
+    if (row < p.R && p.sink != nullptr) {
+      const float ts = ex2(__ldg(p.sink + g * G + row % G) * kLog2e - mb);
+      l += ts;
+      lx += ts;
+    }
+    row_l[row] = l;
+    if (row < p.R && p.lse != nullptr) {
+      const int t = row / G, hh = row - t * G;
+      p.lse[(static_cast<size_t>(b) * n_q + t) * p.Hq + g * G + hh] = (mb + log2f(lx)) * kLn2;
+    }
+  }
+  __syncthreads();
+
+  // ---- O = P V: warp w takes head-dim columns [w*D/4, (w+1)*D/4) -----------
+  constexpr int DW = D / 4;       // columns per warp
+  constexpr int NTO = DW / 8;     // n8 tiles per warp (4 for D=128, 2 for D=64)
+  float acc[MT][NTO][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int j = 0; j < NTO; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][j][e] = 0.f;
+  for (int kk = 0; kk < KP / 16; ++kk) {
+    uint32_t a[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int row = mt * 16 + (lane & 15);
+      const int col = kk * 16 + (lane >> 4) * 8;
+      ldsm_x4(sP + (row * LDP + col) * 2, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
+    }
+#pragma unroll
+    for (int j = 0; j < NTO; j += 2) {
+      // two n8 tiles of V^T: keys kk*16..+15, dims warp*DW + j*8 .. +15
+      uint32_t b0, b1, b2, b3;
+      const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int col = warp * DW + j * 8 + (lane >> 4) * 8;
+      ldsm_x4_t(sV + (key * LD + col) * 2, b0, b1, b2, b3);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        mma_16816(acc[mt][j], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
+        mma_16816(acc[mt][j + 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b2, b3);
+      }
+    }
+  }
+
+  // ---- O / l -> bf16 ----------------------------------------------------------
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int row = mt * 16 + (lane >> 2) + hf * 8;
+      if (row < p.R) {
+        const int t = row / G, hh = row - t * G;
+        const float inv_l = 1.f / row_l[row];
+        __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * n_q + t) * p.Hq + g * G + hh) * D;
+#pragma unroll
+        for (int j = 0; j < NTO; ++j) {
+          const int col = warp * DW + j * 8 + 2 * (lane & 3);
+          *reinterpret_cast<uint32_t*>(orow + col) =
+              pack_bf16x2(acc[mt][j][2 * hf] * inv_l, acc[mt][j][2 * hf + 1] * inv_l);
+        }
+      }
+    }
+}
+
+// Copy accepted new tokens into their ring slots: block = (sequence, token).
+__global__ void __launch_bounds__(128)
+    kv_commit_kernel(__nv_bfloat16* k_ring, __nv_bfloat16* v_ring,
+                     const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                     const int32_t* pos, const int32_t* n_accept, int n_q, int Hkv, int D,
+                     int W) {
+  const int b = blockIdx.x / n_q;
+  const int u = blockIdx.x - b * n_q;
+  int na = __ldg(n_accept + b);
+  const int P = __ldg(pos + b);
+  if (na < 0 || na > n_q || P < 0) {
+    if (u == 0 && threadIdx.x == 0) flag_error(2u);
+    if (P < 0) return;
+    na = min(max(na, 0), n_q);
+  }
+  if (u >= na) return;
+  const int64_t slot = (static_cast<int64_t>(P) + u) % W;
+  const int n16 = Hkv * D / 8;  // 16-byte chunks per token (all kv heads)
+  const uint4* ks = reinterpret_cast<const uint4*>(k_new + (static_cast<size_t>(b) * n_q + u) * Hkv * D);
+  const uint4* vs = reinterpret_cast<const uint4*>(v_new + (static_cast<size_t>(b) * n_q + u) * Hkv * D);
+  uint4* kd = reinterpret_cast<uint4*>(k_ring + (static_cast<size_t>(b) * W + slot) * Hkv * D);
+  uint4* vd = reinterpret_cast<uint4*>(v_ring + (static_cast<size_t>(b) * W + slot) * Hkv * D);
+  for (int idx = threadIdx.x; idx < n16; idx += blockDim.x) {
+    kd[idx] = ks[idx];
+    vd[idx] = vs[idx];
+  }
+}
+
+}  // namespace swa

@@ -1,0 +1,279 @@
+// swa_sink.cu -- the C ABI of libswasink.so (declared in include/swa_sink.h):
+// argument validation, TMA tensor-map encoding and kernel launches for the
+// sliding-window / global attention with a per-head sink on sm_100a.
+//
+// The operation and its sources are described in include/swa_sink.h. Every
+// argument error is returned before any launch; the library allocates no
+// device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "../../include/swa_sink.h"
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// ---- driver entry point for cuTensorMapEncodeTiled (no -lcuda needed) -------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int cuda_fail(const char* what, int err);
+
+// 3-D bf16 tensor [outer][mid][inner] (inner contiguous), 128-byte swizzle.
+int encode_3d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t mid,
+              uint64_t outer, uint32_t box_inner, uint32_t box_mid, uint32_t box_outer) {
+  auto fn = get_encode_fn();
+  if (!fn) return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", 0);
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+  cuuint32_t box[3] = {box_inner, box_mid, box_outer};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SWA_OK : cuda_fail("cuTensorMapEncodeTiled", static_cast<int>(r));
+}
+
+// With SWA_SINK_DEBUG set in the environment, failing CUDA calls are named
+// on stderr (the status code alone says only SWA_ERR_CUDA).
+int cuda_fail(const char* what, int err) {
+  static const bool debug = std::getenv("SWA_SINK_DEBUG") != nullptr;
+  if (debug) std::fprintf(stderr, "swa_sink: %s failed (%d)\n", what, err);
+  return SWA_ERR_CUDA;
+}
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` (once per size
+// increase, per device). The limit plus the kernel's static shared memory
+// must stay within the device's opt-in maximum.
+std::mutex g_attr_mu;
+template <typename K>
+int ensure_smem_attr(K kernel, size_t bytes, size_t (&done)[kMaxDevices]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail("cudaGetDevice", e);
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (done[dev] < bytes) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bytes));
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+    done[dev] = bytes;
+  }
+  return SWA_OK;
+}
+
+size_t g_attr_prefill64[kMaxDevices], g_attr_prefill128[kMaxDevices];
+size_t g_attr_dec[2][2][kMaxDevices];
+
+int next_pow2(int x) {
+  int p = 32;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+template <int D>
+int launch_prefill(const void* q, const void* k, const void* v, const int32_t* cu, int num_seqs,
+                   int total, int Hq, int Hkv, int window, const float* sink, float scale,
+                   void* o, float* lse, cudaStream_t st) {
+  const int G = Hq / Hkv;
+  const int TM = 128 / G;
+  int BN;
+  if (window > 0 && window + TM - 1 <= 256)
+    BN = round_up(window + TM - 1, 16);
+  else
+    BN = 128;
+  swa::PrefillParams p;
+  p.cu_seqlens = cu;
+  p.num_seqs = num_seqs;
+  p.total = total;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.TM = TM;
+  p.window = window;
+  p.BN = BN;
+  p.n_tok_tiles = (total + TM - 1) / TM;
+  p.reverse = window > 0 ? 0 : 1;
+  p.sink = sink;
+  p.scale_log2 = scale * swa::kLog2e;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.q_box_bytes = 128u * TM * G;
+  p.o_col = static_cast<uint32_t>(round_up(BN, 32));
+  p.tmem_cols = static_cast<uint32_t>(next_pow2(static_cast<int>(p.o_col) + D));
+  if (p.tmem_cols > 512) return SWA_ERR_UNSUPPORTED;
+
+  CUtensorMap tq, tk, tv;
+  if (encode_3d(&tq, q, D, Hq, total, 64, G, TM) != SWA_OK) return SWA_ERR_CUDA;
+  if (encode_3d(&tk, k, D, Hkv, total, 64, 1, BN) != SWA_OK) return SWA_ERR_CUDA;
+  if (encode_3d(&tv, v, D, Hkv, total, 64, 1, BN) != SWA_OK) return SWA_ERR_CUDA;
+
+  const size_t smem = 1024 + (D / 64) * 16384 + 2 * (D / 64) * static_cast<size_t>(BN) * 128 +
+                      static_cast<size_t>((BN + 63) / 64) * 16384;
+  auto kern = swa::prefill_sm100_kernel<D>;
+  if (ensure_smem_attr(kern, smem, D == 64 ? g_attr_prefill64 : g_attr_prefill128) != SWA_OK)
+    return SWA_ERR_CUDA;
+  const long long grid = static_cast<long long>(p.n_tok_tiles) * Hkv;
+  if (grid > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  kern<<<static_cast<unsigned>(grid), 128, smem, st>>>(tq, tk, tv, p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SWA_OK : cuda_fail("prefill launch", e);
+}
+
+template <int D, int MT>
+int launch_decode(const swa::DecodeParams& p, cudaStream_t st) {
+  const size_t smem = swa::decode_smem_bytes(D, p.KP);
+  auto kern = swa::decode_sm100_kernel<D, MT>;
+  if (ensure_smem_attr(kern, smem, g_attr_dec[D == 128][MT - 1]) != SWA_OK) return SWA_ERR_CUDA;
+  kern<<<static_cast<unsigned>(p.B) * p.Hkv, 128, smem, st>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SWA_OK : cuda_fail("decode launch", e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int swa_sink_version(void) { return 100; }
+
+const char* swa_sink_status_string(int status) {
+  switch (status) {
+    case SWA_OK: return "ok";
+    case SWA_ERR_NULL: return "a required pointer is NULL";
+    case SWA_ERR_SHAPE: return "a size is negative or inconsistent";
+    case SWA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SWA_ERR_ALIGN: return "a pointer is misaligned";
+    case SWA_ERR_CUDA: return "a CUDA call failed";
+    default: return "unknown status";
+  }
+}
+
+int swa_sink_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                      int num_seqs, int max_seqlen, int total_tokens, int Hq, int Hkv, int D,
+                      int window, const float* sink, float softmax_scale, void* o, float* lse,
+                      void* stream) {
+  if (num_seqs < 0 || max_seqlen < 0 || total_tokens < 0 || Hq <= 0 || Hkv <= 0)
+    return SWA_ERR_SHAPE;
+  if (Hq % Hkv != 0) return SWA_ERR_SHAPE;
+  if (total_tokens > 0 && num_seqs == 0) return SWA_ERR_SHAPE;
+  if (max_seqlen > total_tokens) return SWA_ERR_SHAPE;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 128) return SWA_ERR_UNSUPPORTED;
+  if (total_tokens == 0) return SWA_OK;
+  if (!q || !k || !v || !o || !cu_seqlens) return SWA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SWA_ERR_ALIGN;
+  if (!aligned4(cu_seqlens) || (sink && !aligned4(sink)) || (lse && !aligned4(lse)))
+    return SWA_ERR_ALIGN;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64)
+    return launch_prefill<64>(q, k, v, cu_seqlens, num_seqs, total_tokens, Hq, Hkv, window, sink,
+                              softmax_scale, o, lse, st);
+  return launch_prefill<128>(q, k, v, cu_seqlens, num_seqs, total_tokens, Hq, Hkv, window, sink,
+                             softmax_scale, o, lse, st);
+}
+
+int swa_sink_attn_decode(const void* q, const void* k_new, const void* v_new, const void* k_ring,
+                         const void* v_ring, const int32_t* pos, int B, int n_q, int Hq, int Hkv,
+                         int D, int W, const float* sink, float softmax_scale, void* o,
+                         float* lse, void* stream) {
+  if (B < 0 || n_q <= 0 || Hq <= 0 || Hkv <= 0 || W <= 0) return SWA_ERR_SHAPE;
+  if (Hq % Hkv != 0) return SWA_ERR_SHAPE;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (n_q > 8 || W > 256 || n_q * (Hq / Hkv) > 32) return SWA_ERR_UNSUPPORTED;
+  if (B == 0) return SWA_OK;
+  if (!q || !k_new || !v_new || !k_ring || !v_ring || !pos || !o) return SWA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_ring) ||
+      !aligned16(v_ring) || !aligned16(o))
+    return SWA_ERR_ALIGN;
+  if (!aligned4(pos) || (sink && !aligned4(sink)) || (lse && !aligned4(lse))) return SWA_ERR_ALIGN;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
+  swa::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.k_ring = static_cast<const __nv_bfloat16*>(k_ring);
+  p.v_ring = static_cast<const __nv_bfloat16*>(v_ring);
+  p.pos = pos;
+  p.B = B;
+  p.n_q = n_q;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.W = W;
+  p.R = n_q * p.G;
+  p.KP = round_up(W + n_q, 16);
+  p.sink = sink;
+  p.scale_log2 = softmax_scale * swa::kLog2e;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  if (static_cast<long long>(B) * Hkv > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool two = p.R > 16;
+  if (D == 64) return two ? launch_decode<64, 2>(p, st) : launch_decode<64, 1>(p, st);
+  return two ? launch_decode<128, 2>(p, st) : launch_decode<128, 1>(p, st);
+}
+
+int swa_sink_kv_commit(void* k_ring, void* v_ring, const void* k_new, const void* v_new,
+                       const int32_t* pos, const int32_t* n_accept, int B, int n_q, int Hkv,
+                       int D, int W, void* stream) {
+  if (B < 0 || n_q <= 0 || Hkv <= 0 || W <= 0) return SWA_ERR_SHAPE;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (B == 0) return SWA_OK;
+  if (!k_ring || !v_ring || !k_new || !v_new || !pos || !n_accept) return SWA_ERR_NULL;
+  if (!aligned16(k_ring) || !aligned16(v_ring) || !aligned16(k_new) || !aligned16(v_new))
+    return SWA_ERR_ALIGN;
+  if (!aligned4(pos) || !aligned4(n_accept)) return SWA_ERR_ALIGN;
+  const long long grid = static_cast<long long>(B) * n_q;
+  if (grid > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  swa::kv_commit_kernel<<<static_cast<unsigned>(grid), 128, 0, st>>>(
+      static_cast<__nv_bfloat16*>(k_ring), static_cast<__nv_bfloat16*>(v_ring),
+      static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), pos,
+      n_accept, n_q, Hkv, D, W);
+  return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int swa_sink_device_error(unsigned int* flags, int clear) {
+  if (!flags) return SWA_ERR_NULL;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SWA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, swa::g_device_error, sizeof v) != cudaSuccess) return SWA_ERR_CUDA;
+  *flags = v;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(swa::g_device_error, &zero, sizeof zero) != cudaSuccess)
+      return SWA_ERR_CUDA;
+  }
+  return SWA_OK;
+}
+
+}  // extern "C"

@@ -143,3 +143,18 @@ def shard_units(num_units: int, world_size: int, rank: int):
     lo = rank * base + min(rank, extra)
     hi = lo + base + (1 if rank < extra else 0)
     return lo, hi
+
+
+def slice_sequences(c, lo, hi):
+    """The packed sub-batch of sequences [lo, hi) of a prefill input dict:
+    contiguous token slices of q, k, v and a rebased cu_seqlens."""
+    cu = c["cu_seqlens"]
+    a, b = int(cu[lo]), int(cu[hi])
+    sub = dict(c)
+    sub["q"], sub["k"], sub["v"] = c["q"][a:b], c["k"][a:b], c["v"][a:b]
+    sub["cu_seqlens"] = (cu[lo:hi + 1] - a).to(torch.int32)
+    sub["seqlens"] = list(c["seqlens"][lo:hi])
+    sub["total"] = b - a
+    sub["max_seqlen"] = max(sub["seqlens"]) if sub["seqlens"] else 0
+    sub["token_range"] = (a, b)
+    return sub

@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI: the library loads and exports every symbol
+include/swa_sink.h declares, and argument errors are returned before any
+launch (these calls never reach the GPU, so they run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sliding_window_attention_sink_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "swa_sink.h")
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"SWA_API\s+[\w\s\*]*?\b(swa_sink_\w+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.load()
+    names = declared_symbols()
+    assert len(names) >= 6
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings():
+    assert B.swa_sink_version() == 100
+    assert B.status_string(0) == "ok"
+    for code in (-1, -2, -3, -4, -5):
+        assert B.status_string(code) != "unknown status"
+
+
+FAKE = 0x10000  # a 16-byte aligned address that is never dereferenced
+
+
+def fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, cu_seqlens=FAKE, num_seqs=1, max_seqlen=8,
+             total_tokens=8, Hq=8, Hkv=2, D=128, window=128, sink=None,
+             softmax_scale=0.0, o=FAKE, lse=None, stream=0)
+    a.update(kw)
+    return B.swa_sink_attn_fwd(**a)
+
+
+def test_fwd_argument_errors():
+    assert fwd(Hq=8, Hkv=3) == -2
+    assert fwd(total_tokens=-1) == -2
+    assert fwd(num_seqs=-1) == -2
+    assert fwd(num_seqs=0) == -2
+    assert fwd(max_seqlen=9) == -2
+    assert fwd(D=96) == -3
+    assert fwd(Hq=256, Hkv=1) == -3
+    assert fwd(q=None) == -1
+    assert fwd(cu_seqlens=None) == -1
+    assert fwd(o=FAKE + 2) == -4
+    assert fwd(k=FAKE + 8) == -4
+    assert fwd(lse=FAKE + 2) == -4
+    assert fwd(total_tokens=0, max_seqlen=0) == 0   # nothing to do, nothing launched
+
+
+def dec(**kw):
+    a = dict(q=FAKE, k_new=FAKE, v_new=FAKE, k_ring=FAKE, v_ring=FAKE, pos=FAKE, B=4,
+             n_q=4, Hq=64, Hkv=8, D=128, W=128, sink=None, softmax_scale=0.0, o=FAKE,
+             lse=None, stream=0)
+    a.update(kw)
+    return B.swa_sink_attn_decode(**a)
+
+
+def test_decode_argument_errors():
+    assert dec(n_q=0) == -2
+    assert dec(W=0) == -2
+    assert dec(Hkv=7) == -2
+    assert dec(n_q=9) == -3
+    assert dec(W=257) == -3
+    assert dec(Hq=128, Hkv=8, n_q=3) == -3   # 48 query rows per kv head
+    assert dec(D=80) == -3
+    assert dec(pos=None) == -1
+    assert dec(k_ring=FAKE + 4) == -4
+    assert dec(B=0) == 0
+
+
+def test_commit_argument_errors():
+    a = dict(k_ring=FAKE, v_ring=FAKE, k_new=FAKE, v_new=FAKE, pos=FAKE, n_accept=FAKE,
+             B=2, n_q=4, Hkv=8, D=128, W=128, stream=0)
+    assert B.swa_sink_kv_commit(**dict(a, n_q=0)) == -2
+    assert B.swa_sink_kv_commit(**dict(a, D=32)) == -3
+    assert B.swa_sink_kv_commit(**dict(a, n_accept=None)) == -1
+    assert B.swa_sink_kv_commit(**dict(a, v_new=FAKE + 1)) == -4
+    assert B.swa_sink_kv_commit(**dict(a, B=0)) == 0
+
+
+def test_header_is_plain_c():
+    """The header compiles as C99 with no CUDA or torch headers."""
+    import subprocess
+    import tempfile
+    with tempfile.TemporaryDirectory() as td:
+        src = os.path.join(td, "t.c")
+        open(src, "w").write('#include "swa_sink.h"\nint main(void){return swa_sink_version()>0?0:1;}\n')
+        r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only",
+                            "-I", os.path.join(ROOT, "include"), src],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr

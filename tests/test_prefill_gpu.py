@@ -1,0 +1,127 @@
+"""GPU parity of swa_sink_attn_fwd (through the C ABI) against the fp64 oracle
+on the same seeded inputs: small shapes compared element by element, the full
+workloads on sampled rows, plus edge cases (ragged tails, empty and length-1
+sequences, tiles straddling sequences, no sink, extreme sinks, W = 1, G = 1
+and G = 16, chunked windows and global layers)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sliding_window_attention_sink_b200 import binding as B
+from sliding_window_attention_sink_b200 import workloads as wl
+
+from _parity import check, to_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(c, window=None, sink="case", poison=True):
+    d = to_cuda(c)
+    w = c["window"] if window is None else window
+    s = d["sink"] if sink == "case" else sink
+    o = torch.full_like(d["q"], float("nan")) if poison else None
+    o, lse = B.attn_fwd(d["q"], d["k"], d["v"], d["cu_seqlens"], w, sink=s, out=o,
+                        max_seqlen=c["max_seqlen"])
+    torch.cuda.synchronize()
+    assert B.swa_sink_device_error() == 0
+    return o, lse
+
+
+SMALL = [  # (name, seqlens, Hq, Hkv, D, W, sink)
+    ("tiny_cfg", [512], 4, 1, 64, 128, "uniform2"),
+    ("swa_ragged", [300], 64, 8, 128, 128, "normal"),
+    ("varlen_edges", [100, 0, 257, 1, 33], 16, 2, 128, 128, "normal"),
+    ("global_chunks", [700], 16, 2, 128, 0, "normal"),
+    ("global_varlen", [129, 300, 5], 8, 1, 64, 0, "uniform2"),
+    ("wide_window", [600], 8, 1, 64, 300, "normal"),
+    ("g1", [300], 2, 2, 64, 128, "normal"),
+    ("g16", [200], 32, 2, 128, 64, "normal"),
+    ("g2_w8", [90], 4, 2, 128, 8, "normal"),
+    ("no_sink", [257], 8, 1, 128, 128, None),
+    ("w1", [70], 8, 1, 64, 1, "normal"),
+    ("short_seqs", [1, 2, 3, 17], 8, 1, 128, 128, "normal"),
+]
+
+
+@pytest.mark.parametrize("name,seqlens,Hq,Hkv,D,W,sink", SMALL, ids=[s[0] for s in SMALL])
+def test_prefill_matches_oracle(name, seqlens, Hq, Hkv, D, W, sink):
+    seed = 0 if name == "tiny_cfg" else 7
+    sigma = 1.0 if name == "tiny_cfg" else 0.5
+    c = wl.prefill_case(seqlens, Hq, Hkv, D, W, sigma=sigma, sink=sink, seed=seed)
+    o, lse = run_gpu(c)
+    ro, rl, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], Hq, Hkv, D, W,
+                               sink=c["sink"])
+    check(o, lse, ro, rl, name)
+
+
+@pytest.mark.parametrize("sval", [30.0, -30.0, 0.0])
+def test_prefill_extreme_sinks(sval):
+    c = wl.prefill_case([200], 8, 1, 128, 128, sigma=0.5, sink=None, seed=3)
+    sink = torch.full((8,), sval)
+    c["sink"] = sink
+    o, lse = run_gpu(c)
+    ro, rl, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], 8, 1, 128, 128,
+                               sink=sink)
+    check(o, lse, ro, rl, "sink=%g" % sval)
+
+
+def test_prefill_window_ge_len_equals_global():
+    c = wl.prefill_case([333], 16, 2, 128, 0, sigma=0.5, sink="normal", seed=4)
+    o0, l0 = run_gpu(c, window=0)
+    o1, l1 = run_gpu(c, window=4096)
+    ro, rl, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], 16, 2, 128, 0,
+                               sink=c["sink"])
+    check(o0, l0, ro, rl, "W=0")
+    check(o1, l1, ro, rl, "W=4096")
+
+
+def test_prefill_lse_optional_and_scale():
+    c = wl.prefill_case([150], 8, 2, 64, 32, sigma=0.5, sink="normal", seed=5)
+    d = to_cuda(c)
+    o, lse = B.attn_fwd(d["q"], d["k"], d["v"], d["cu_seqlens"], 32, sink=d["sink"],
+                        softmax_scale=0.3, want_lse=False)
+    torch.cuda.synchronize()
+    assert lse is None
+    ro, rl, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], 8, 2, 64, 32,
+                               sink=c["sink"], scale=float(np.float32(0.3)))
+    check(o, None, ro, rl, "scale=0.3")
+
+
+def sample_rows(c, n, seed):
+    rng = np.random.default_rng(seed)
+    total, Hq = c["total"], c["Hq"]
+    cu = c["cu_seqlens"].tolist()
+    toks = set(rng.integers(0, total, n).tolist())
+    for s in range(len(cu) - 1):   # sequence starts and ends, window edges
+        for t in (cu[s], cu[s] + 1, cu[s] + 127, cu[s] + 128, cu[s + 1] - 1):
+            if cu[s] <= t < cu[s + 1]:
+                toks.add(t)
+    toks = sorted(toks)
+    heads = rng.integers(0, Hq, len(toks))
+    return np.array(toks, np.int64), heads.astype(np.int32)
+
+
+@pytest.mark.parametrize("wname", ["swa_prefill_32k", "global_prefill_8k",
+                                   "varlen_swa_prefill"])
+def test_prefill_full_workloads_sampled(wname):
+    """The benchmark's launch configuration at full size; sampled rows
+    (all heads of each sampled token's kv group are checked) vs the oracle."""
+    case = wl.WORKLOADS[wname]
+    c = wl.make_prefill(case)
+    o, lse = run_gpu(c)
+    rt, rh = sample_rows(c, 384, 1)
+    G = c["Hq"] // c["Hkv"]
+    # widen each sampled (token, head) to its whole query group
+    rt = np.repeat(rt, G)
+    rh = (np.repeat(rh // G, G) * G + np.tile(np.arange(G), len(rh))).astype(np.int32)
+    ro, rl, _ = oracle.prefill_rows(c["q"], c["k"], c["v"], c["cu_seqlens"], c["Hq"],
+                                    c["Hkv"], c["D"], c["window"], rt, rh, sink=c["sink"])
+    og = o[torch.from_numpy(rt).cuda(), torch.from_numpy(rh.astype(np.int64)).cuda()]
+    lg = lse[torch.from_numpy(rh.astype(np.int64)).cuda(), torch.from_numpy(rt).cuda()]
+    check(og, lg, ro, rl, wname)
+    # every row written (the output was poisoned with NaN)
+    assert torch.isfinite(o).all().item()
+    assert torch.isfinite(lse).all().item()
