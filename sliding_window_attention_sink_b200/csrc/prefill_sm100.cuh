@@ -66,12 +66,16 @@ __device__ __forceinline__ int seq_of_token(const int32_t* cu, int num_seqs, int
   return lo;
 }
 
-// First key visible to token t (its own sequence start, or t - W + 1).
-__device__ __forceinline__ int first_visible_key(const PrefillParams& p, int t) {
-  const int s = seq_of_token(p.cu_seqlens, p.num_seqs, t);
-  int lo = __ldg(p.cu_seqlens + s);
-  if (p.window > 0) lo = max(lo, t - p.window + 1);
+// First key visible to token t: its own sequence start, or t - W + 1.
+__device__ __forceinline__ int first_key(const int32_t* cu, int num_seqs, int window, int t) {
+  const int s = seq_of_token(cu, num_seqs, t);
+  int lo = __ldg(cu + s);
+  if (window > 0) lo = max(lo, t - window + 1);
   return lo;
+}
+
+__device__ __forceinline__ int first_visible_key(const PrefillParams& p, int t) {
+  return first_key(p.cu_seqlens, p.num_seqs, p.window, t);
 }
 
 template <int D>

@@ -13,11 +13,13 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/swa_sink.h"
 #include "decode_sm100.cuh"
 #include "prefill_sm100.cuh"
+#include "prefill_swa_ring_sm100.cuh"
 
 namespace {
 
@@ -96,6 +98,80 @@ int next_pow2(int x) {
 }
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+size_t g_attr_ring64[kMaxDevices], g_attr_ring128[kMaxDevices];
+
+// Dynamic shared memory available next to the ring kernel's static barriers.
+constexpr size_t kRingSmemLimit = 232448 - 2048;
+
+// Sliding-window prefill on the persistent ring pipeline when the window's
+// keys for one tile fit one MMA (BN <= 256) and the S/P double buffer plus O
+// fit TMEM. Returns SWA_ERR_UNSUPPORTED (nothing launched) otherwise.
+template <int D>
+int launch_prefill_ring(const void* q, const void* k, const void* v, const int32_t* cu,
+                        int num_seqs, int total, int Hq, int Hkv, int window, const float* sink,
+                        float scale, void* o, float* lse, cudaStream_t st) {
+  const int G = Hq / Hkv;
+  if (window <= 0 || !(G == 2 || G == 4 || G == 8)) return SWA_ERR_UNSUPPORTED;
+  const int TM = 128 / G;
+  const int KB = (window - 1 + TM - 1) / TM;
+  const int NWIN = KB + 1;
+  const int BN = NWIN * TM;
+  const int scol = round_up(BN, 32);
+  if (BN > 256 || 2 * scol + D > 512) return SWA_ERR_UNSUPPORTED;
+  int NQ = 3, NB = std::min(swa::kRingMaxBlocks, NWIN + 3);
+  while (swa::ring_smem_bytes(D, TM, NB, NQ) > kRingSmemLimit) {
+    if (NB > NWIN + 1) --NB;
+    else if (NQ > 2) --NQ;
+    else return SWA_ERR_UNSUPPORTED;
+  }
+  if (NB <= NWIN) return SWA_ERR_UNSUPPORTED;
+  swa::RingParams p;
+  p.cu_seqlens = cu;
+  p.num_seqs = num_seqs;
+  p.total = total;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.TM = TM;
+  p.window = window;
+  p.KB = KB;
+  p.NWIN = NWIN;
+  p.NB = NB;
+  p.NQ = NQ;
+  p.n_tok_tiles = (total + TM - 1) / TM;
+  p.n_tiles = p.n_tok_tiles * Hkv;
+  p.sink = sink;
+  p.scale_log2 = scale * swa::kLog2e;
+  p.lse = lse;
+  p.q_box_bytes = 128u * TM * G;
+  p.s_stride = static_cast<uint32_t>(scol);
+  p.o_col = static_cast<uint32_t>(2 * scol);
+
+  CUtensorMap tq, tk, tv, to;
+  if (encode_3d(&tq, q, D, Hq, total, 64, G, TM) != SWA_OK) return SWA_ERR_CUDA;
+  if (encode_3d(&tk, k, D, Hkv, total, 64, 1, TM) != SWA_OK) return SWA_ERR_CUDA;
+  if (encode_3d(&tv, v, D, Hkv, total, 64, 1, TM) != SWA_OK) return SWA_ERR_CUDA;
+  if (encode_3d(&to, o, D, Hq, total, 64, G, TM) != SWA_OK) return SWA_ERR_CUDA;
+
+  const size_t smem = swa::ring_smem_bytes(D, TM, NB, NQ);
+  auto kern = swa::prefill_swa_ring_kernel<D>;
+  if (ensure_smem_attr(kern, smem, D == 64 ? g_attr_ring64 : g_attr_ring128) != SWA_OK)
+    return SWA_ERR_CUDA;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)", 0);
+  const int grid = std::min(nsm, p.n_tiles);
+  kern<<<grid, 320, smem, st>>>(tq, tk, tv, to, p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SWA_OK : cuda_fail("ring prefill launch", e);
+}
 
 template <int D>
 int launch_prefill(const void* q, const void* k, const void* v, const int32_t* cu, int num_seqs,
@@ -193,6 +269,16 @@ int swa_sink_attn_fwd(const void* q, const void* k, const void* v, const int32_t
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
     softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // sliding windows: the persistent ring pipeline when the shape allows it
+  if (window > 0) {
+    const int rc = D == 64 ? launch_prefill_ring<64>(q, k, v, cu_seqlens, num_seqs,
+                                                     total_tokens, Hq, Hkv, window, sink,
+                                                     softmax_scale, o, lse, st)
+                           : launch_prefill_ring<128>(q, k, v, cu_seqlens, num_seqs,
+                                                      total_tokens, Hq, Hkv, window, sink,
+                                                      softmax_scale, o, lse, st);
+    if (rc != SWA_ERR_UNSUPPORTED) return rc;
+  }
   if (D == 64)
     return launch_prefill<64>(q, k, v, cu_seqlens, num_seqs, total_tokens, Hq, Hkv, window, sink,
                               softmax_scale, o, lse, st);
