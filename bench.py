@@ -349,6 +349,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="prefill workloads: replace the sequence lengths by one "
+                         "sequence of this length (small cases for profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -375,6 +378,11 @@ def main():
 
     case = wl.WORKLOADS[args.workload]
     is_prefill = isinstance(case, wl.PrefillCase)
+    if args.seqlen > 0 and is_prefill:
+        import dataclasses
+        case = dataclasses.replace(case, seqlens=[args.seqlen], varlen_draw=None,
+                                   name="%s (T=%d)" % (case.name, args.seqlen))
+        args.no_cpu_baseline = True
     runner = (PrefillRunner if is_prefill else DecodeRunner)(case, rank, torch, B, wl)
     stream = torch.cuda.Stream()
     sptr = stream.cuda_stream

@@ -4,27 +4,38 @@
 // Operation: the same as prefill_sm100.cuh ("MiMo-V2-Flash Technical Report"
 // summary, mlpod.com, section 2.2.2: the sink joins the softmax max and
 // denominator; section 2.2.1: window of 128 tokens), for sliding windows whose
-// whole key range for a tile fits one MMA (BN <= 256).
+// whole key range for a tile fits one MMA (BN <= 192).
 //
 // Why a different kernel for SWA: with W = 128 a tile's keys are its own TM
 // tokens plus the W - 1 before them, so consecutive tiles of one kv head share
 // all but TM keys. Each CTA therefore walks a contiguous span of token tiles
-// (all 148 SMs busy, one CTA each) and keeps K and V in a ring of TM-key
-// blocks in shared memory: per tile it fetches one new block (TM keys) from
-// HBM instead of the whole window. What remains per tile is the Q tile in and
-// the O tile out -- the bytes that bound the layer -- and the pipeline below
-// keeps them streaming:
+// (all SMs busy, one CTA each) and keeps K and V in a ring of TM-key blocks in
+// shared memory: per tile it fetches one new block (TM keys) from HBM instead
+// of the whole window. What remains per tile is the Q tile in and the O tile
+// out -- the bytes that bound the layer -- and the pipeline below keeps them
+// streaming:
 //
-//   warp 0      TMA producer: Q tile (3-D box [64, G, TM], NQ stages) and new
+//   warps 0-3   warpgroup 0 and
+//   warps 4-7   warpgroup 1: both work on the same tile. Thread r of each owns
+//               TMEM lane r (tile row r); warpgroup h takes S columns
+//               [h*BN/2, (h+1)*BN/2) in one TMEM load into registers, masks
+//               them, and the two halves exchange their row maxima and sums
+//               through shared memory. The max is seeded with the sink, the
+//               sum gets the sink term; P = exp2(x - m) goes back over S as
+//               bf16 pairs (A operand of the PV MMA). Then, for the previous
+//               tile, warpgroup h moves O columns [h*D/2, (h+1)*D/2) from TMEM
+//               to a swizzled staging tile (O / l in bf16) and TMA-stores it.
+//   warp 8      TMA producer: Q tile (3-D box [64, G, TM], NQ stages) and new
 //               K/V blocks (box [64, 1, TM]) into the ring.
-//   warp 1      TMEM allocation; one thread issues tcgen05.mma:
-//               S = Q K^T into one of two TMEM S buffers (the window may wrap
-//               around the ring: then two MMAs, N1 + N2 = BN), and
-//               O = P V with P read from TMEM (TS form) and V from the ring.
-//   warps 2-5   softmax: thread r owns TMEM lane r; masked max seeded with the
-//               sink, P = exp2(x - m) written back over S as bf16 pairs; LSE.
-//   warps 6-9   epilogue: O / l -> bf16 into a swizzled staging tile -> TMA
-//               store.
+//   warp 9      TMEM allocation; issues S = Q K^T (tcgen05.mma, K-major
+//               operands) into S buffer (tile & 1); where the window wraps
+//               around the ring, two MMAs per k-step (N1 + N2 = BN).
+//   warp 10     issues O = P V (P from TMEM, V MN-major from the ring).
+//
+// S and PV have separate issuing warps because one thread issuing dependent
+// tcgen05.mma back to back was measured at 90-230 cycles per instruction on
+// B200 (more than the 64-72 cycles of tensor work of these N=128/144 shapes),
+// while two issuers together reach the tensor rate.
 //
 // Every wait is bounded (see mbar_wait); nothing here traps.
 #pragma once
@@ -39,6 +50,8 @@ namespace swa {
 
 constexpr int kRingMaxBlocks = 16;
 constexpr int kRingMaxQ = 4;
+constexpr int kRingThreads = 352;  // 11 warps
+constexpr int kRingMaxBN16 = 12;   // BN <= 192: a half row fits in registers
 
 struct RingParams {
   const int32_t* cu_seqlens;
@@ -67,20 +80,27 @@ __host__ __device__ inline size_t ring_smem_bytes(int D, int TM, int NB, int NQ)
          2 * nch * static_cast<size_t>(NB) * TM * 128;
 }
 
-template <int D>
-__global__ void __launch_bounds__(320, 1)
+// BN16 = BN / 16 is fixed at compile time so a half row of scores lives in
+// registers.
+template <int D, int BN16>
+__global__ void __launch_bounds__(kRingThreads, 1)
     prefill_swa_ring_kernel(const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v,
                             const __grid_constant__ CUtensorMap tm_o, const RingParams p) {
   constexpr int NCH = D / 64;
   constexpr uint32_t CH = 16384;  // one 128-row x 128-byte chunk
+  constexpr int BN = BN16 * 16;
+  constexpr int HALF = BN / 2;    // S columns per warpgroup (a multiple of 8)
+  constexpr int H16 = HALF / 16;  // x16 TMEM loads per half row ...
+  constexpr int H8 = (HALF % 16) / 8;  // ... plus one x8 load when HALF % 16 == 8
+  constexpr int DH = D / 2;       // O columns per warpgroup in the epilogue
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full[kRingMaxQ], q_empty[kRingMaxQ];
   __shared__ __align__(8) uint64_t kv_full[kRingMaxBlocks], kv_empty[kRingMaxBlocks];
-  __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], l_free[2];
+  __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2];
   __shared__ __align__(8) uint64_t o_full, o_empty;
-  __shared__ float l_s[2][128];
+  __shared__ float red_max[2][128], red_lr[2][128], red_lx[2][128];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -114,15 +134,14 @@ __global__ void __launch_bounds__(320, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&s_full[b]), 1);
       mbar_init(smem_u32(&s_empty[b]), 1);
-      mbar_init(smem_u32(&p_full[b]), 4);
-      mbar_init(smem_u32(&l_free[b]), 4);
+      mbar_init(smem_u32(&p_full[b]), 8);
     }
     mbar_init(smem_u32(&o_full), 1);
-    mbar_init(smem_u32(&o_empty), 4);
+    mbar_init(smem_u32(&o_empty), 8);
     abort_sh = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(&tmem_base_sh), 512);
     tmem_relinquish();
   }
@@ -144,12 +163,154 @@ __global__ void __launch_bounds__(320, 1)
     return tb == 0 ? p.NWIN : 1;  // a new kv head restarts the window
   };
 
-  if (warp == 0) {
+  if (warp < 8) {
+    // ============ softmax + epilogue (two warpgroups, one tile) ==============
+    const int hw = warp >> 2;              // half of the row / of O
+    const int r = 32 * (warp & 3) + lane;  // TMEM lane == tile row
+    const int tok = r / p.G, hh = r - tok * p.G;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const bool store_thread = (warp & 3) == 0 && lane == 0;  // one per warpgroup
+    float l_prev = 0.f;
+    int g_prev = 0, tb_prev = 0;
+    for (int j = 0; j <= ntile && !*abort; ++j) {
+      float l_cur = 0.f;
+      int g = 0, tb = 0;
+      if (j < ntile) {
+        // ---------------------------- softmax of tile j ---------------------
+        tile_of(j, g, tb);
+        const int b = j & 1;
+        const int i = tb * p.TM + tok;
+        const int h = g * p.G + hh;
+        const bool valid = i < p.total;
+        int row_lo = 1, row_hi = 0;  // empty unless valid
+        if (valid) {
+          row_lo = first_key(p.cu_seqlens, p.num_seqs, p.window, i);
+          row_hi = i;
+        }
+        // visible columns of this half: e with (e - cmin) in [0, span]
+        const int cmin = row_lo - (tb - p.KB) * p.TM - hw * HALF;
+        const unsigned span = static_cast<unsigned>(row_hi - row_lo);
+        const float sink2 =
+            (valid && p.sink != nullptr) ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+        if (!mbar_wait(smem_u32(&s_full[b]), (j >> 1) & 1, abort)) break;
+        __syncwarp();
+        tc_fence_after();
+        const uint32_t tS = tmem + lane_off + b * p.s_stride;
+        uint32_t v[HALF];
+#pragma unroll
+        for (int c = 0; c < H16; ++c) tmem_ld16_at(tS + hw * HALF + c * 16, &v[c * 16]);
+        if (H8) tmem_ld8_at(tS + hw * HALF + H16 * 16, &v[H16 * 16]);
+        tmem_ld_wait();
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < HALF; e += 2) {
+          if (static_cast<unsigned>(e - cmin) > span) v[e] = 0xff800000u;  // -inf
+          if (static_cast<unsigned>(e + 1 - cmin) > span) v[e + 1] = 0xff800000u;
+          mx0 = fmaxf(mx0, __uint_as_float(v[e]));
+          mx1 = fmaxf(mx1, __uint_as_float(v[e + 1]));
+        }
+        const float mx = fmaxf(mx0, mx1);
+        red_max[hw][r] = mx;
+        named_bar_sync(1, 256);
+        const float m = fmaxf(sink2, fmaxf(mx, red_max[hw ^ 1][r]) * p.scale_log2);
+        const float mb = (m == -INFINITY) ? 0.f : m;
+        // P = exp2(x - m) (masked: exp2(-inf) = 0) as bf16 pairs over S
+        // columns [hw*HALF/2, (hw+1)*HALF/2); sums of the rounded P (for O)
+        // and of fp32 P (for the LSE)
+        float lr0 = 0.f, lr1 = 0.f, lx0 = 0.f, lx1 = 0.f;
+        const uint32_t tP = tS + hw * (HALF / 2);
+#pragma unroll
+        for (int c = 0; c < HALF; c += 16) {
+          uint32_t w[8];
+          const int n = (HALF - c) >= 16 ? 16 : 8;
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            if (e < n) {
+              const float x0 = ex2(fmaf(__uint_as_float(v[c + e]), p.scale_log2, -mb));
+              const float x1 = ex2(fmaf(__uint_as_float(v[c + e + 1]), p.scale_log2, -mb));
+              w[e >> 1] = pack_bf16x2(x0, x1);
+              lr0 += bf16lo_to_f32(w[e >> 1]);
+              lr1 += bf16hi_to_f32(w[e >> 1]);
+              lx0 += x0;
+              lx1 += x1;
+            }
+          }
+          if (n == 16) tmem_st8(tP + c / 2, w);
+          else tmem_st4(tP + c / 2, w);
+        }
+        red_lr[hw][r] = lr0 + lr1;
+        red_lx[hw][r] = lx0 + lx1;
+        tmem_st_wait();
+        tc_fence_before();
+        named_bar_sync(1, 256);
+        float l_r = red_lr[0][r] + red_lr[1][r];
+        float l_x = red_lx[0][r] + red_lx[1][r];
+        if (sink2 != -INFINITY) {
+          const float ts = ex2(sink2 - mb);
+          l_r += ts;
+          l_x += ts;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&p_full[b]));
+        if (hw == 0 && valid && p.lse != nullptr)
+          p.lse[static_cast<size_t>(h) * p.total + i] = (mb + log2f(l_x)) * kLn2;
+        l_cur = l_r;
+      }
+      if (j > 0) {
+        // ------------------------ epilogue of tile j - 1 --------------------
+        const int je = j - 1;
+        if (!mbar_wait(smem_u32(&o_full), je & 1, abort)) break;
+        __syncwarp();
+        tc_fence_after();
+        const uint32_t tO = tmem + lane_off + p.o_col + hw * DH;
+        uint32_t v[DH];
+#pragma unroll
+        for (int c = 0; c < DH; c += 16) tmem_ld16_at(tO + c, &v[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&o_empty));
+        const float inv_l = l_prev > 0.f ? 1.f / l_prev : 0.f;
+        // staging: 64-column chunks, 128-byte swizzle (16-byte unit u of row
+        // r at u ^ (r & 7)); with D = 128 each warpgroup owns one chunk and
+        // stores it itself, with D = 64 the two halves share chunk 0
+        const uint32_t chunk = NCH == 2 ? static_cast<uint32_t>(hw) : 0u;
+        const uint32_t unit0 = NCH == 2 ? 0u : static_cast<uint32_t>(hw) * 4u;
+        const uint32_t bar_id = NCH == 2 ? 2u + hw : 1u;
+        const uint32_t bar_n = NCH == 2 ? 128u : 256u;
+        const bool issuer = NCH == 2 ? store_thread : tid == 0;
+        if (issuer) tma_store_wait_read<0>();
+        named_bar_sync(bar_id, bar_n);
+        const uint32_t rowaddr = sO + chunk * CH + r * 128;
+#pragma unroll
+        for (int u = 0; u < DH / 8; ++u) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(v[u * 8 + 2 * e]) * inv_l,
+                               __uint_as_float(v[u * 8 + 2 * e + 1]) * inv_l);
+          st_shared_v4(rowaddr + (((unit0 + u) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(bar_id, bar_n);
+        if (issuer) {
+          tma_store_3d(&tm_o, sO + chunk * CH, static_cast<int>(chunk) * 64, g_prev * p.G,
+                       tb_prev * p.TM);
+          tma_store_commit();
+        }
+      }
+      l_prev = l_cur;
+      g_prev = g;
+      tb_prev = tb;
+    }
+    if (store_thread || tid == 0) tma_store_wait_all<0>();
+  } else if (warp == 8) {
     // ======================= TMA producer ====================================
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_o);
       int nload = 0;
       for (int j = 0; j < ntile && !*abort; ++j) {
         int g, tb;
@@ -177,216 +338,87 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ======================= MMA issuer ======================================
-    if (lane == 0) {
-      const int BN = p.NWIN * p.TM;
-      const uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      int nload = 0;          // blocks loaded up to and including the current tile
-      int win_first_prev = 0;
-      // O = P V for tile j: P from TMEM (over S buffer j & 1), V from the ring
-      auto issue_pv = [&](int j, int win_first) -> bool {
-        const int b = j & 1;
-        if (!mbar_wait(smem_u32(&p_full[b]), (j >> 1) & 1, abort)) return false;
-        if (!mbar_wait(smem_u32(&o_empty), (j & 1) ^ 1, abort)) return false;
-        tc_fence_after();
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const int wb = (kk * 16) / p.TM;       // block within the window
-          const int off = kk * 16 - wb * p.TM;   // first key inside the block
-          const int slot = (win_first + wb) % p.NB;
-          // V as the MN-major B operand: 64-dim blocks ring_ch apart (LBO),
-          // 8-key groups 1024 bytes apart (SBO)
-          const uint64_t bd = smem_desc_sw128(sV + slot * blk_bytes + off * 128, ring_ch, 1024);
-          mma_bf16_ts(tmem + p.o_col, tmem + b * p.s_stride + kk * 8, bd, idesc_pv,
-                      kk > 0 ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&o_full));
-        mma_commit(smem_u32(&s_empty[b]));
-        return true;
-      };
-      for (int j = 0; j < ntile && !*abort; ++j) {
-        const int b = j & 1, st = j % p.NQ;
-        const int nnew = new_blocks(j);
-        const int first_new = nload;
-        nload += nnew;
-        const int win_first = nload - p.NWIN;
-        // A tile that starts a new kv head replaces the whole window: finish
-        // the previous tile and release its blocks before waiting for the new
-        // ones (the producer needs the slots).
-        const bool restart = j > 0 && nnew == p.NWIN;
-        if (restart) {
-          if (!issue_pv(j - 1, win_first_prev)) break;
-          for (int s = win_first_prev; s < first_new; ++s)
-            mma_commit(smem_u32(&kv_empty[s % p.NB]));
-        }
-        if (!mbar_wait(smem_u32(&s_empty[b]), ((j >> 1) & 1) ^ 1, abort)) break;
-        if (!mbar_wait(smem_u32(&q_full[st]), (j / p.NQ) & 1, abort)) break;
-        bool ok = true;
-        for (int s = first_new; s < nload && ok; ++s)
-          ok = mbar_wait(smem_u32(&kv_full[s % p.NB]), (s / p.NB) & 1, abort);
-        if (!ok) break;
-        tc_fence_after();
-        // S = Q K^T over the window; two MMAs where it wraps around the ring
+  } else if (warp == 9) {
+    // ======================= S = Q K^T issuer ================================
+    int nload = 0;
+    for (int j = 0; j < ntile && !*abort; ++j) {
+      const int b = j & 1, st = j % p.NQ;
+      const int first_new = nload;
+      nload += new_blocks(j);
+      const int win_first = nload - p.NWIN;
+      if (!mbar_wait(smem_u32(&s_empty[b]), ((j >> 1) & 1) ^ 1, abort)) break;
+      if (!mbar_wait(smem_u32(&q_full[st]), (j / p.NQ) & 1, abort)) break;
+      bool ok = true;
+      for (int s = first_new; s < nload && ok; ++s)
+        ok = mbar_wait(smem_u32(&kv_full[s % p.NB]), (s / p.NB) & 1, abort);
+      if (!ok) break;
+      __syncwarp();
+      tc_fence_after();
+      if (elect_one()) {
+        // the window's blocks are consecutive ring slots; two MMAs per k-step
+        // where they wrap
         const int slot0 = win_first % p.NB;
-        const int n1 = min(p.NWIN, p.NB - slot0);  // blocks before the wrap
+        const int n1 = min(p.NWIN, p.NB - slot0);
         const int n2 = p.NWIN - n1;
         const uint32_t idesc1 = idesc_bf16_f32(128, n1 * p.TM, false, false);
         const uint32_t idesc2 = idesc_bf16_f32(128, n2 > 0 ? n2 * p.TM : 16, false, false);
+        const uint32_t dS = tmem + b * p.s_stride;
+        const uint32_t aQ = sQ + st * NCH * CH;
+        const uint32_t bK1 = sK + slot0 * blk_bytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ch = kk >> 2, koff = (kk & 3) * 32;
-          const uint64_t ad = smem_desc_sw128(sQ + (st * NCH + ch) * CH + koff, 16, 1024);
-          const uint64_t bd1 =
-              smem_desc_sw128(sK + ch * ring_ch + slot0 * blk_bytes + koff, 16, 1024);
-          mma_bf16_ss(tmem + b * p.s_stride, ad, bd1, idesc1, kk > 0 ? 1u : 0u);
-          if (n2 > 0) {
-            const uint64_t bd2 = smem_desc_sw128(sK + ch * ring_ch + koff, 16, 1024);
-            mma_bf16_ss(tmem + b * p.s_stride + n1 * p.TM, ad, bd2, idesc2, kk > 0 ? 1u : 0u);
-          }
+          const uint32_t off = (kk >> 2) * CH + (kk & 3) * 32;
+          const uint32_t offk = (kk >> 2) * ring_ch + (kk & 3) * 32;
+          const uint64_t ad = smem_desc_sw128(aQ + off, 16, 1024);
+          mma_bf16_ss(dS, ad, smem_desc_sw128(bK1 + offk, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
+          if (n2 > 0)
+            mma_bf16_ss(dS + n1 * p.TM, ad, smem_desc_sw128(sK + offk, 16, 1024), idesc2,
+                        kk > 0 ? 1u : 0u);
         }
         mma_commit(smem_u32(&s_full[b]));
         mma_commit(smem_u32(&q_empty[st]));
-        // PV of the previous tile, then release the blocks the window left
-        if (j > 0 && !restart) {
-          if (!issue_pv(j - 1, win_first_prev)) break;
-          for (int s = win_first_prev; s < win_first; ++s)
-            mma_commit(smem_u32(&kv_empty[s % p.NB]));
-        }
-        win_first_prev = win_first;
       }
-      if (ntile > 0 && !*abort) issue_pv(ntile - 1, win_first_prev);
-    }
-    __syncwarp();
-  } else if (warp < 6) {
-    // ======================= softmax (warps 2..5) ============================
-    const int r = 32 * (warp & 3) + lane;  // TMEM lane == tile row
-    const int tok = r / p.G, hh = r - tok * p.G;
-    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const int BN = p.NWIN * p.TM;
-    for (int j = 0; j < ntile; ++j) {
-      int g, tb;
-      tile_of(j, g, tb);
-      const int b = j & 1;
-      const int i = tb * p.TM + tok;
-      const int h = g * p.G + hh;
-      const bool valid = i < p.total;
-      int row_lo = 1, row_hi = 0;  // empty unless valid
-      if (valid) {
-        row_lo = first_key(p.cu_seqlens, p.num_seqs, p.window, i);
-        row_hi = i;
-      }
-      const int kw0 = (tb - p.KB) * p.TM;  // key of S column 0
-      const int cmin = row_lo - kw0, cmax = row_hi - kw0;
-      const float sink2 = (valid && p.sink != nullptr) ? __ldg(p.sink + h) * kLog2e : -INFINITY;
-      if (!mbar_wait(smem_u32(&s_full[b]), (j >> 1) & 1, abort)) break;
       __syncwarp();
-      tc_fence_after();
-      const uint32_t tS = tmem + lane_off + b * p.s_stride;
-      // pass 1: masked row max, seeded with the sink
-      float mx = -INFINITY;
-      for (int cb = 0; cb < BN; cb += 16) {
-        uint32_t v[16];
-        tmem_ld16(tS + cb, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int col = cb + e;
-          if (col >= cmin && col <= cmax) mx = fmaxf(mx, __uint_as_float(v[e]));
-        }
-      }
-      const float m = fmaxf(sink2, mx * p.scale_log2);
-      const float mb = (m == -INFINITY) ? 0.f : m;
-      // pass 2: P = exp2(x - m) as bf16 pairs written over S (columns
-      // [0, BN/2)); sums of the rounded P (for O) and of fp32 P (for LSE)
-      float l_r = 0.f, l_x = 0.f;
-      for (int cb = 0; cb < BN; cb += 16) {
-        uint32_t v[16];
-        tmem_ld16(tS + cb, v);
-        tmem_ld_wait();
-        uint32_t w[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const int col = cb + e;
-          const float x0 = (col >= cmin && col <= cmax)
-                               ? ex2(__uint_as_float(v[e]) * p.scale_log2 - mb) : 0.f;
-          const float x1 = (col + 1 >= cmin && col + 1 <= cmax)
-                               ? ex2(__uint_as_float(v[e + 1]) * p.scale_log2 - mb) : 0.f;
-          w[e >> 1] = pack_bf16x2(x0, x1);
-          l_r += bf16lo_to_f32(w[e >> 1]) + bf16hi_to_f32(w[e >> 1]);
-          l_x += x0 + x1;
-        }
-        tmem_st8(tS + (cb >> 1), w);
-      }
-      if (sink2 != -INFINITY) {
-        const float ts = ex2(sink2 - mb);
-        l_r += ts;
-        l_x += ts;
-      }
-      tmem_st_wait();
-      if (valid && p.lse != nullptr)
-        p.lse[static_cast<size_t>(h) * p.total + i] = (mb + log2f(l_x)) * kLn2;
-      // hand l to the epilogue once it has read this buffer's previous value
-      if (!mbar_wait(smem_u32(&l_free[b]), ((j >> 1) & 1) ^ 1, abort)) break;
-      l_s[b][r] = l_r;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&p_full[b]));
     }
   } else {
-    // ======================= epilogue (warps 6..9) ===========================
-    const int r = 32 * (warp & 3) + lane;
-    const int et = tid - 192;  // 0..127
-    const uint32_t tO = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + p.o_col;
-    for (int j = 0; j < ntile; ++j) {
-      int g, tb;
-      tile_of(j, g, tb);
+    // ======================= O = P V issuer (warp 10) ========================
+    const uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+    int nload = 0;
+    for (int j = 0; j < ntile && !*abort; ++j) {
       const int b = j & 1;
-      if (!mbar_wait(smem_u32(&o_full), j & 1, abort)) break;
-      // p_full[b] of this tile completed before PV was issued; waiting on it
-      // here orders the softmax's write of l_s[b] before the read below
+      nload += new_blocks(j);
+      const int win_first = nload - p.NWIN;
+      // first window block of the next tile: blocks before it are released
+      const int win_next = j + 1 < ntile ? nload + new_blocks(j + 1) - p.NWIN : win_first;
       if (!mbar_wait(smem_u32(&p_full[b]), (j >> 1) & 1, abort)) break;
+      if (!mbar_wait(smem_u32(&o_empty), (j & 1) ^ 1, abort)) break;
       __syncwarp();
       tc_fence_after();
-      const float l = l_s[b][r];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&l_free[b]));
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      // the staging tile is free once the previous TMA store has read it
-      if (et == 0) tma_store_wait_read<0>();
-      named_bar_sync(1, 128);
-#pragma unroll
-      for (int db = 0; db < D; db += 16) {
-        uint32_t v[16];
-        tmem_ld16(tO + db, v);
-        tmem_ld_wait();
-        uint32_t w[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2)
-          w[e >> 1] = pack_bf16x2(__uint_as_float(v[e]) * inv_l, __uint_as_float(v[e + 1]) * inv_l);
-        // 128-byte swizzle, as the TMA store expects: unit u -> u ^ (r & 7)
-        const uint32_t rowaddr = sO + (db >> 6) * CH + r * 128;
-        const uint32_t u0 = (db & 63) >> 3;
-        st_shared_v4(rowaddr + ((u0 ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
-        st_shared_v4(rowaddr + (((u0 + 1) ^ (r & 7)) << 4), w[4], w[5], w[6], w[7]);
+      if (elect_one()) {
+        int slot = win_first % p.NB;
+        uint32_t aP = tmem + b * p.s_stride;  // P: 8 columns per 16 keys
+        for (int wb = 0; wb < p.NWIN; ++wb) {
+          const uint32_t vb = sV + slot * blk_bytes;
+          for (int off = 0; off < p.TM; off += 16) {
+            // V as the MN-major B operand: 64-dim blocks ring_ch apart (LBO),
+            // 8-key groups 1024 bytes apart (SBO)
+            mma_bf16_ts(tmem + p.o_col, aP, smem_desc_sw128(vb + off * 128, ring_ch, 1024),
+                        idesc_pv, (wb | off) != 0 ? 1u : 0u);
+            aP += 8;
+          }
+          slot = slot + 1 == p.NB ? 0 : slot + 1;
+        }
+        mma_commit(smem_u32(&o_full));
+        mma_commit(smem_u32(&s_empty[b]));
+        for (int s = win_first; s < win_next; ++s) mma_commit(smem_u32(&kv_empty[s % p.NB]));
       }
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&o_empty));
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (et == 0) {
-#pragma unroll
-        for (int ch = 0; ch < NCH; ++ch)
-          tma_store_3d(&tm_o, sO + ch * CH, ch * 64, g * p.G, tb * p.TM);
-        tma_store_commit();
-      }
     }
-    if (et == 0) tma_store_wait_all<0>();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

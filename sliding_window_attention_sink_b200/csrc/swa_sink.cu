@@ -106,10 +106,21 @@ int sm_count() {
   return n;
 }
 
-size_t g_attr_ring64[kMaxDevices], g_attr_ring128[kMaxDevices];
+size_t g_attr_ring[2][swa::kRingMaxBN16 + 1][kMaxDevices];
+
+template <int D, int BN16>
+int run_ring(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+             const CUtensorMap& to, const swa::RingParams& p, size_t smem, int grid,
+             cudaStream_t st) {
+  auto kern = swa::prefill_swa_ring_kernel<D, BN16>;
+  if (ensure_smem_attr(kern, smem, g_attr_ring[D == 128][BN16]) != SWA_OK) return SWA_ERR_CUDA;
+  kern<<<grid, swa::kRingThreads, smem, st>>>(tq, tk, tv, to, p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SWA_OK : cuda_fail("ring prefill launch", e);
+}
 
 // Dynamic shared memory available next to the ring kernel's static barriers.
-constexpr size_t kRingSmemLimit = 232448 - 2048;
+constexpr size_t kRingSmemLimit = 232448 - 4096;
 
 // Sliding-window prefill on the persistent ring pipeline when the window's
 // keys for one tile fit one MMA (BN <= 256) and the S/P double buffer plus O
@@ -125,7 +136,7 @@ int launch_prefill_ring(const void* q, const void* k, const void* v, const int32
   const int NWIN = KB + 1;
   const int BN = NWIN * TM;
   const int scol = round_up(BN, 32);
-  if (BN > 256 || 2 * scol + D > 512) return SWA_ERR_UNSUPPORTED;
+  if (BN > 16 * swa::kRingMaxBN16 || 2 * scol + D > 512) return SWA_ERR_UNSUPPORTED;
   int NQ = 3, NB = std::min(swa::kRingMaxBlocks, NWIN + 3);
   while (swa::ring_smem_bytes(D, TM, NB, NQ) > kRingSmemLimit) {
     if (NB > NWIN + 1) --NB;
@@ -162,15 +173,20 @@ int launch_prefill_ring(const void* q, const void* k, const void* v, const int32
   if (encode_3d(&to, o, D, Hq, total, 64, G, TM) != SWA_OK) return SWA_ERR_CUDA;
 
   const size_t smem = swa::ring_smem_bytes(D, TM, NB, NQ);
-  auto kern = swa::prefill_swa_ring_kernel<D>;
-  if (ensure_smem_attr(kern, smem, D == 64 ? g_attr_ring64 : g_attr_ring128) != SWA_OK)
-    return SWA_ERR_CUDA;
   const int nsm = sm_count();
   if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)", 0);
   const int grid = std::min(nsm, p.n_tiles);
-  kern<<<grid, 320, smem, st>>>(tq, tk, tv, to, p);
-  const cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? SWA_OK : cuda_fail("ring prefill launch", e);
+  switch (BN / 16) {
+#define SWA_RING_CASE(N)                                                        \
+  case N:                                                                       \
+    return run_ring<D, N>(tq, tk, tv, to, p, smem, grid, st);
+    SWA_RING_CASE(1) SWA_RING_CASE(2) SWA_RING_CASE(3) SWA_RING_CASE(4) SWA_RING_CASE(5)
+    SWA_RING_CASE(6) SWA_RING_CASE(7) SWA_RING_CASE(8) SWA_RING_CASE(9) SWA_RING_CASE(10)
+    SWA_RING_CASE(11) SWA_RING_CASE(12)
+#undef SWA_RING_CASE
+    default:
+      return SWA_ERR_UNSUPPORTED;
+  }
 }
 
 template <int D>
