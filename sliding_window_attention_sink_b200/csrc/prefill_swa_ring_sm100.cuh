@@ -15,22 +15,23 @@
 // out -- the bytes that bound the layer -- and the pipeline below keeps them
 // streaming:
 //
-//   warps 0-3   warpgroup 0 and
-//   warps 4-7   warpgroup 1: both work on the same tile. Thread r of each owns
-//               TMEM lane r (tile row r); warpgroup h takes S columns
-//               [h*BN/2, (h+1)*BN/2) in one TMEM load into registers, masks
-//               them, and the two halves exchange their row maxima and sums
-//               through shared memory. The max is seeded with the sink, the
-//               sum gets the sink term; P = exp2(x - m) goes back over S as
-//               bf16 pairs (A operand of the PV MMA). Then, for the previous
-//               tile, warpgroup h moves O columns [h*D/2, (h+1)*D/2) from TMEM
-//               to a swizzled staging tile (O / l in bf16) and TMA-stores it.
-//   warp 8      TMA producer: Q tile (3-D box [64, G, TM], NQ stages) and new
+//   warps 0-3   softmax warpgroup 0 and
+//   warps 4-7   softmax warpgroup 1: both work on the same tile. Thread r of
+//               each owns TMEM lane r (tile row r); warpgroup h takes S
+//               columns [h*BN/2, (h+1)*BN/2) in one TMEM load into registers,
+//               masks them (only 16-column chunks that cross some row's window
+//               edge), and the two halves exchange their row maxima and sums
+//               through shared memory. The max is seeded with the sink, the sum
+//               gets the sink term; P = exp2(x - m) goes back over S as bf16
+//               pairs (A operand of the PV MMA).
+//   warps 8-11  epilogue: O / l -> bf16 into a swizzled staging tile -> TMA
+//               store, one 64-column chunk at a time.
+//   warp 12     TMA producer: Q tile (3-D box [64, G, TM], NQ stages) and new
 //               K/V blocks (box [64, 1, TM]) into the ring.
-//   warp 9      TMEM allocation; issues S = Q K^T (tcgen05.mma, K-major
+//   warp 13     TMEM allocation; issues S = Q K^T (tcgen05.mma, K-major
 //               operands) into S buffer (tile & 1); where the window wraps
 //               around the ring, two MMAs per k-step (N1 + N2 = BN).
-//   warp 10     issues O = P V (P from TMEM, V MN-major from the ring).
+//   warp 14     issues O = P V (P from TMEM, V MN-major from the ring).
 //
 // S and PV have separate issuing warps because one thread issuing dependent
 // tcgen05.mma back to back was measured at 90-230 cycles per instruction on
@@ -48,9 +49,26 @@
 
 namespace swa {
 
+// Pipeline timeline hooks: compiled out unless SWA_RING_TRACE is defined (a
+// profiling build then supplies swa_ring_trace: clock64 stamps of CTA 0,
+// [role][tile][event], roles 0 producer, 1 S issuer, 2 PV issuer, 3 softmax,
+// 4 epilogue).
+#ifdef SWA_RING_TRACE
+__device__ unsigned long long* swa_ring_trace;
+#define RING_TRACE(role, j, ev)                                                           \
+  do {                                                                                    \
+    if (blockIdx.x == 0 && (j) < 128)                                                     \
+      swa_ring_trace[((role) * 128 + (j)) * 8 + (ev)] = static_cast<unsigned long long>(clock64()); \
+  } while (0)
+#else
+#define RING_TRACE(role, j, ev) \
+  do {                          \
+  } while (0)
+#endif
+
 constexpr int kRingMaxBlocks = 16;
 constexpr int kRingMaxQ = 4;
-constexpr int kRingThreads = 352;  // 11 warps
+constexpr int kRingThreads = 480;  // 15 warps
 constexpr int kRingMaxBN16 = 12;   // BN <= 192: a half row fits in registers
 
 struct RingParams {
@@ -94,13 +112,12 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   constexpr int HALF = BN / 2;    // S columns per warpgroup (a multiple of 8)
   constexpr int H16 = HALF / 16;  // x16 TMEM loads per half row ...
   constexpr int H8 = (HALF % 16) / 8;  // ... plus one x8 load when HALF % 16 == 8
-  constexpr int DH = D / 2;       // O columns per warpgroup in the epilogue
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full[kRingMaxQ], q_empty[kRingMaxQ];
   __shared__ __align__(8) uint64_t kv_full[kRingMaxBlocks], kv_empty[kRingMaxBlocks];
-  __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2];
+  __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], l_free[2];
   __shared__ __align__(8) uint64_t o_full, o_empty;
-  __shared__ float red_max[2][128], red_lr[2][128], red_lx[2][128];
+  __shared__ float red_max[2][128], red_lr[2][128], red_lx[2][128], l_s[2][128];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -135,13 +152,14 @@ __global__ void __launch_bounds__(kRingThreads, 1)
       mbar_init(smem_u32(&s_full[b]), 1);
       mbar_init(smem_u32(&s_empty[b]), 1);
       mbar_init(smem_u32(&p_full[b]), 8);
+      mbar_init(smem_u32(&l_free[b]), 4);
     }
     mbar_init(smem_u32(&o_full), 1);
-    mbar_init(smem_u32(&o_empty), 8);
+    mbar_init(smem_u32(&o_empty), 4);
     abort_sh = 0;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(&tmem_base_sh), 512);
     tmem_relinquish();
   }
@@ -164,147 +182,188 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   };
 
   if (warp < 8) {
-    // ============ softmax + epilogue (two warpgroups, one tile) ==============
-    const int hw = warp >> 2;              // half of the row / of O
+    // ================== softmax (two warpgroups, one tile) ===================
+    const int hw = warp >> 2;              // half of the row
     const int r = 32 * (warp & 3) + lane;  // TMEM lane == tile row
     const int tok = r / p.G, hh = r - tok * p.G;
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const bool store_thread = (warp & 3) == 0 && lane == 0;  // one per warpgroup
-    float l_prev = 0.f;
-    int g_prev = 0, tb_prev = 0;
-    for (int j = 0; j <= ntile && !*abort; ++j) {
-      float l_cur = 0.f;
-      int g = 0, tb = 0;
-      if (j < ntile) {
-        // ---------------------------- softmax of tile j ---------------------
-        tile_of(j, g, tb);
-        const int b = j & 1;
-        const int i = tb * p.TM + tok;
-        const int h = g * p.G + hh;
-        const bool valid = i < p.total;
-        int row_lo = 1, row_hi = 0;  // empty unless valid
-        if (valid) {
-          row_lo = first_key(p.cu_seqlens, p.num_seqs, p.window, i);
-          row_hi = i;
+    const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+    for (int j = 0; j < ntile; ++j) {
+      int g, tb;
+      tile_of(j, g, tb);
+      const int b = j & 1;
+      const int t0 = tb * p.TM;
+      const int i = t0 + tok;
+      const int h = g * p.G + hh;
+      const bool valid = i < p.total;
+      int row_lo = 1, row_hi = 0;  // empty unless valid
+      if (valid) {
+        row_lo = first_key(p.cu_seqlens, p.num_seqs, p.window, i);
+        row_hi = i;
+      }
+      const int c0 = (tb - p.KB) * p.TM + hw * HALF;  // key of this half's column 0
+      // visible columns of this half: e with (e - cmin) in [0, span]
+      const int cmin = row_lo - c0;
+      const unsigned span = static_cast<unsigned>(row_hi - row_lo);
+      // columns visible to every valid row of the tile (uniform): from the
+      // last valid token's first key to the first token itself
+      const int t_last = min(t0 + p.TM, p.total) - 1;
+      const int all_lo = first_key(p.cu_seqlens, p.num_seqs, p.window, t_last) - c0;
+      const int all_hi = t0 - c0;
+      const float sink2 = (valid && p.sink != nullptr) ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+      if (tid == 0) RING_TRACE(3, j, 0);
+      if (!mbar_wait(smem_u32(&s_full[b]), (j >> 1) & 1, abort)) break;
+      __syncwarp();
+      tc_fence_after();
+      if (tid == 0) RING_TRACE(3, j, 1);
+      const uint32_t tS = tmem + lane_off + b * p.s_stride;
+      uint32_t v[HALF];
+#pragma unroll
+      for (int c = 0; c < H16; ++c) tmem_ld16_at(tS + hw * HALF + c * 16, &v[c * 16]);
+      if (H8) tmem_ld8_at(tS + hw * HALF + H16 * 16, &v[H16 * 16]);
+      tmem_ld_wait();
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < HALF; c += 16) {
+        const int n = (HALF - c) >= 16 ? 16 : 8;
+        if (!(c >= all_lo && c + n - 1 <= all_hi)) {  // some row's window edge is here
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (e < n && static_cast<unsigned>(c + e - cmin) > span) v[c + e] = 0xff800000u;
         }
-        // visible columns of this half: e with (e - cmin) in [0, span]
-        const int cmin = row_lo - (tb - p.KB) * p.TM - hw * HALF;
-        const unsigned span = static_cast<unsigned>(row_hi - row_lo);
-        const float sink2 =
-            (valid && p.sink != nullptr) ? __ldg(p.sink + h) * kLog2e : -INFINITY;
-        if (!mbar_wait(smem_u32(&s_full[b]), (j >> 1) & 1, abort)) break;
-        __syncwarp();
-        tc_fence_after();
-        const uint32_t tS = tmem + lane_off + b * p.s_stride;
-        uint32_t v[HALF];
 #pragma unroll
-        for (int c = 0; c < H16; ++c) tmem_ld16_at(tS + hw * HALF + c * 16, &v[c * 16]);
-        if (H8) tmem_ld8_at(tS + hw * HALF + H16 * 16, &v[H16 * 16]);
-        tmem_ld_wait();
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < HALF; e += 2) {
-          if (static_cast<unsigned>(e - cmin) > span) v[e] = 0xff800000u;  // -inf
-          if (static_cast<unsigned>(e + 1 - cmin) > span) v[e + 1] = 0xff800000u;
-          mx0 = fmaxf(mx0, __uint_as_float(v[e]));
-          mx1 = fmaxf(mx1, __uint_as_float(v[e + 1]));
-        }
-        const float mx = fmaxf(mx0, mx1);
-        red_max[hw][r] = mx;
-        named_bar_sync(1, 256);
-        const float m = fmaxf(sink2, fmaxf(mx, red_max[hw ^ 1][r]) * p.scale_log2);
-        const float mb = (m == -INFINITY) ? 0.f : m;
-        // P = exp2(x - m) (masked: exp2(-inf) = 0) as bf16 pairs over S
-        // columns [hw*HALF/2, (hw+1)*HALF/2); sums of the rounded P (for O)
-        // and of fp32 P (for the LSE)
-        float lr0 = 0.f, lr1 = 0.f, lx0 = 0.f, lx1 = 0.f;
-        const uint32_t tP = tS + hw * (HALF / 2);
-#pragma unroll
-        for (int c = 0; c < HALF; c += 16) {
-          uint32_t w[8];
-          const int n = (HALF - c) >= 16 ? 16 : 8;
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            if (e < n) {
-              const float x0 = ex2(fmaf(__uint_as_float(v[c + e]), p.scale_log2, -mb));
-              const float x1 = ex2(fmaf(__uint_as_float(v[c + e + 1]), p.scale_log2, -mb));
-              w[e >> 1] = pack_bf16x2(x0, x1);
-              lr0 += bf16lo_to_f32(w[e >> 1]);
-              lr1 += bf16hi_to_f32(w[e >> 1]);
-              lx0 += x0;
-              lx1 += x1;
-            }
+        for (int e = 0; e < 16; e += 4) {
+          if (e < n) {
+            mx0 = max3(mx0, __uint_as_float(v[c + e]), __uint_as_float(v[c + e + 1]));
+            mx1 = max3(mx1, __uint_as_float(v[c + e + 2]), __uint_as_float(v[c + e + 3]));
           }
-          if (n == 16) tmem_st8(tP + c / 2, w);
-          else tmem_st4(tP + c / 2, w);
         }
-        red_lr[hw][r] = lr0 + lr1;
-        red_lx[hw][r] = lx0 + lx1;
-        tmem_st_wait();
-        tc_fence_before();
-        named_bar_sync(1, 256);
+      }
+      const float mx = fmaxf(mx0, mx1);
+      red_max[hw][r] = mx;
+      if (tid == 0) RING_TRACE(3, j, 2);
+      named_bar_sync(1, 256);
+      if (tid == 0) RING_TRACE(3, j, 3);
+      const float m = fmaxf(sink2, fmaxf(mx, red_max[hw ^ 1][r]) * p.scale_log2);
+      const float mb = (m == -INFINITY) ? 0.f : m;
+      // P = exp2(x - m) (masked: exp2(-inf) = 0) as bf16 pairs over S
+      // columns [hw*HALF/2, (hw+1)*HALF/2); sums of the rounded P (for O)
+      // and of fp32 P (for the LSE)
+      uint64_t lr2 = 0, lx2 = 0;  // packed pair sums (0.0f, 0.0f)
+      const uint64_t nm2 = f2_pack(-mb, -mb);
+      const uint32_t tP = tS + hw * (HALF / 2);
+#pragma unroll
+      for (int c = 0; c < HALF; c += 16) {
+        uint32_t w[8];
+        const int n = (HALF - c) >= 16 ? 16 : 8;
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          if (e < n) {
+            float t0f, t1f;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(v[c + e]), __uint_as_float(v[c + e + 1])),
+                             sc2, nm2),
+                      t0f, t1f);
+            const float x0 = ex2(t0f), x1 = ex2(t1f);
+            w[e >> 1] = pack_bf16x2(x0, x1);
+            lr2 = f2_add(lr2, f2_pack(bf16lo_to_f32(w[e >> 1]), bf16hi_to_f32(w[e >> 1])));
+            lx2 = f2_add(lx2, f2_pack(x0, x1));
+          }
+        }
+        if (n == 16) tmem_st8(tP + c / 2, w);
+        else tmem_st4(tP + c / 2, w);
+      }
+      {
+        float a0, a1;
+        f2_unpack(lr2, a0, a1);
+        red_lr[hw][r] = a0 + a1;
+        f2_unpack(lx2, a0, a1);
+        red_lx[hw][r] = a0 + a1;
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      if (tid == 0) RING_TRACE(3, j, 4);
+      named_bar_sync(1, 256);
+      if (tid == 0) RING_TRACE(3, j, 5);
+      float l_x = 0.f;
+      if (hw == 0) {
         float l_r = red_lr[0][r] + red_lr[1][r];
-        float l_x = red_lx[0][r] + red_lx[1][r];
+        l_x = red_lx[0][r] + red_lx[1][r];
         if (sink2 != -INFINITY) {
           const float ts = ex2(sink2 - mb);
           l_r += ts;
           l_x += ts;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&p_full[b]));
-        if (hw == 0 && valid && p.lse != nullptr)
-          p.lse[static_cast<size_t>(h) * p.total + i] = (mb + log2f(l_x)) * kLn2;
-        l_cur = l_r;
+        // l for the epilogue, once it has read this buffer's previous value
+        if (!mbar_wait(smem_u32(&l_free[b]), ((j >> 1) & 1) ^ 1, abort)) break;
+        l_s[b][r] = l_r;
       }
-      if (j > 0) {
-        // ------------------------ epilogue of tile j - 1 --------------------
-        const int je = j - 1;
-        if (!mbar_wait(smem_u32(&o_full), je & 1, abort)) break;
-        __syncwarp();
-        tc_fence_after();
-        const uint32_t tO = tmem + lane_off + p.o_col + hw * DH;
-        uint32_t v[DH];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&p_full[b]));
+      if (tid == 0) RING_TRACE(3, j, 6);
+      if (hw == 0 && valid && p.lse != nullptr)
+        p.lse[static_cast<size_t>(h) * p.total + i] = (mb + lg2(l_x)) * kLn2;
+    }
+  } else if (warp < 12) {
+    // ======================= epilogue (warps 8..11) ==========================
+    const int r = 32 * (warp & 3) + lane;
+    const bool issuer = tid == 256;
+    const uint32_t tO = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + p.o_col;
+    for (int j = 0; j < ntile; ++j) {
+      int g, tb;
+      tile_of(j, g, tb);
+      const int b = j & 1;
+      if (issuer) RING_TRACE(4, j, 0);
+      if (!mbar_wait(smem_u32(&o_full), j & 1, abort)) break;
+      if (issuer) RING_TRACE(4, j, 1);
+      // p_full[b] of this tile completed before PV was issued; waiting on it
+      // here orders the softmax's write of l_s[b] before the read below
+      if (!mbar_wait(smem_u32(&p_full[b]), (j >> 1) & 1, abort)) break;
+      __syncwarp();
+      tc_fence_after();
+      const float l = l_s[b][r];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&l_free[b]));
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      // O leaves one 64-column chunk at a time: TMEM -> registers -> bf16 ->
+      // staging chunk (128-byte swizzle: 16-byte unit u of row r at u ^ (r&7))
+      // -> TMA store as its own bulk group. The staging chunk is reused once
+      // its previous store has read it. TMEM O is released after the last
+      // chunk's load.
 #pragma unroll
-        for (int c = 0; c < DH; c += 16) tmem_ld16_at(tO + c, &v[c]);
+      for (int ch = 0; ch < NCH; ++ch) {
+        uint32_t v[64];
+#pragma unroll
+        for (int c = 0; c < 64; c += 16) tmem_ld16_at(tO + ch * 64 + c, &v[c]);
         tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&o_empty));
-        const float inv_l = l_prev > 0.f ? 1.f / l_prev : 0.f;
-        // staging: 64-column chunks, 128-byte swizzle (16-byte unit u of row
-        // r at u ^ (r & 7)); with D = 128 each warpgroup owns one chunk and
-        // stores it itself, with D = 64 the two halves share chunk 0
-        const uint32_t chunk = NCH == 2 ? static_cast<uint32_t>(hw) : 0u;
-        const uint32_t unit0 = NCH == 2 ? 0u : static_cast<uint32_t>(hw) * 4u;
-        const uint32_t bar_id = NCH == 2 ? 2u + hw : 1u;
-        const uint32_t bar_n = NCH == 2 ? 128u : 256u;
-        const bool issuer = NCH == 2 ? store_thread : tid == 0;
-        if (issuer) tma_store_wait_read<0>();
-        named_bar_sync(bar_id, bar_n);
-        const uint32_t rowaddr = sO + chunk * CH + r * 128;
+        if (ch == NCH - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&o_empty));
+          if (issuer) RING_TRACE(4, j, 2);
+        }
+        if (issuer) tma_store_wait_read<NCH - 1>();
+        named_bar_sync(2, 128);
+        const uint32_t rowaddr = sO + ch * CH + r * 128;
 #pragma unroll
-        for (int u = 0; u < DH / 8; ++u) {
+        for (int u = 0; u < 8; ++u) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             w[e] = pack_bf16x2(__uint_as_float(v[u * 8 + 2 * e]) * inv_l,
                                __uint_as_float(v[u * 8 + 2 * e + 1]) * inv_l);
-          st_shared_v4(rowaddr + (((unit0 + u) ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+          st_shared_v4(rowaddr + ((u ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
-        named_bar_sync(bar_id, bar_n);
+        named_bar_sync(2, 128);
         if (issuer) {
-          tma_store_3d(&tm_o, sO + chunk * CH, static_cast<int>(chunk) * 64, g_prev * p.G,
-                       tb_prev * p.TM);
+          tma_store_3d(&tm_o, sO + ch * CH, ch * 64, g * p.G, tb * p.TM);
           tma_store_commit();
         }
       }
-      l_prev = l_cur;
-      g_prev = g;
-      tb_prev = tb;
+      if (issuer) RING_TRACE(4, j, 3);
     }
-    if (store_thread || tid == 0) tma_store_wait_all<0>();
-  } else if (warp == 8) {
+    if (issuer) tma_store_wait_all<0>();
+  } else if (warp == 12) {
     // ======================= TMA producer ====================================
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -316,7 +375,9 @@ __global__ void __launch_bounds__(kRingThreads, 1)
         int g, tb;
         tile_of(j, g, tb);
         const int st = j % p.NQ;
+        RING_TRACE(0, j, 0);
         if (!mbar_wait(smem_u32(&q_empty[st]), ((j / p.NQ) & 1) ^ 1, abort)) break;
+        RING_TRACE(0, j, 1);
         mbar_arrive_expect_tx(smem_u32(&q_full[st]), NCH * p.q_box_bytes);
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch)
@@ -338,51 +399,64 @@ __global__ void __launch_bounds__(kRingThreads, 1)
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ======================= S = Q K^T issuer ================================
+    // Descriptors are computed by the whole warp; one elected lane issues.
+    const uint64_t kmaj = smem_desc_sw128(0, 16, 1024);  // layout bits, no address
     int nload = 0;
     for (int j = 0; j < ntile && !*abort; ++j) {
       const int b = j & 1, st = j % p.NQ;
       const int first_new = nload;
       nload += new_blocks(j);
       const int win_first = nload - p.NWIN;
+      if (lane == 0) RING_TRACE(1, j, 0);
       if (!mbar_wait(smem_u32(&s_empty[b]), ((j >> 1) & 1) ^ 1, abort)) break;
+      if (lane == 0) RING_TRACE(1, j, 1);
       if (!mbar_wait(smem_u32(&q_full[st]), (j / p.NQ) & 1, abort)) break;
+      if (lane == 0) RING_TRACE(1, j, 2);
       bool ok = true;
       for (int s = first_new; s < nload && ok; ++s)
         ok = mbar_wait(smem_u32(&kv_full[s % p.NB]), (s / p.NB) & 1, abort);
       if (!ok) break;
+      if (lane == 0) RING_TRACE(1, j, 3);
       __syncwarp();
       tc_fence_after();
-      if (elect_one()) {
-        // the window's blocks are consecutive ring slots; two MMAs per k-step
-        // where they wrap
-        const int slot0 = win_first % p.NB;
-        const int n1 = min(p.NWIN, p.NB - slot0);
-        const int n2 = p.NWIN - n1;
-        const uint32_t idesc1 = idesc_bf16_f32(128, n1 * p.TM, false, false);
-        const uint32_t idesc2 = idesc_bf16_f32(128, n2 > 0 ? n2 * p.TM : 16, false, false);
-        const uint32_t dS = tmem + b * p.s_stride;
-        const uint32_t aQ = sQ + st * NCH * CH;
-        const uint32_t bK1 = sK + slot0 * blk_bytes;
+      // the window's blocks are consecutive ring slots; two MMAs per k-step
+      // where they wrap
+      const int slot0 = win_first % p.NB;
+      const int n1 = min(p.NWIN, p.NB - slot0);
+      const int n2 = p.NWIN - n1;
+      const uint32_t idesc1 = idesc_bf16_f32(128, n1 * p.TM, false, false);
+      const uint32_t idesc2 = idesc_bf16_f32(128, n2 > 0 ? n2 * p.TM : 16, false, false);
+      const uint32_t dS = tmem + b * p.s_stride;
+      const uint32_t dS2 = dS + n1 * p.TM;
+      const uint64_t aq = kmaj | ((sQ + st * NCH * CH) >> 4);
+      const uint64_t bk1 = kmaj | ((sK + slot0 * blk_bytes) >> 4);
+      const uint64_t bk2 = kmaj | (sK >> 4);
+      const bool leader = elect_one();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * CH + (kk & 3) * 32;
-          const uint32_t offk = (kk >> 2) * ring_ch + (kk & 3) * 32;
-          const uint64_t ad = smem_desc_sw128(aQ + off, 16, 1024);
-          mma_bf16_ss(dS, ad, smem_desc_sw128(bK1 + offk, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
-          if (n2 > 0)
-            mma_bf16_ss(dS + n1 * p.TM, ad, smem_desc_sw128(sK + offk, 16, 1024), idesc2,
-                        kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * CH + (kk & 3) * 32) >> 4;
+        const uint32_t offk = ((kk >> 2) * ring_ch + (kk & 3) * 32) >> 4;
+        if (leader) {
+          mma_bf16_ss(dS, aq + off, bk1 + offk, idesc1, kk > 0 ? 1u : 0u);
+          if (n2 > 0) mma_bf16_ss(dS2, aq + off, bk2 + offk, idesc2, kk > 0 ? 1u : 0u);
         }
+      }
+      if (leader) {
         mma_commit(smem_u32(&s_full[b]));
         mma_commit(smem_u32(&q_empty[st]));
+        RING_TRACE(1, j, 4);
       }
       __syncwarp();
     }
-  } else {
-    // ======================= O = P V issuer (warp 10) ========================
+  } else if (warp == 14) {
+    // ======================= O = P V issuer ==================================
     const uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+    // V as the MN-major B operand: 64-dim blocks ring_ch apart (LBO), 8-key
+    // groups 1024 bytes apart (SBO)
+    const uint64_t mnmaj = smem_desc_sw128(0, ring_ch, 1024);
+    const uint32_t ring_keys = static_cast<uint32_t>(p.NB * p.TM);
     int nload = 0;
     for (int j = 0; j < ntile && !*abort; ++j) {
       const int b = j & 1;
@@ -390,27 +464,29 @@ __global__ void __launch_bounds__(kRingThreads, 1)
       const int win_first = nload - p.NWIN;
       // first window block of the next tile: blocks before it are released
       const int win_next = j + 1 < ntile ? nload + new_blocks(j + 1) - p.NWIN : win_first;
+      if (lane == 0) RING_TRACE(2, j, 0);
       if (!mbar_wait(smem_u32(&p_full[b]), (j >> 1) & 1, abort)) break;
+      if (lane == 0) RING_TRACE(2, j, 1);
       if (!mbar_wait(smem_u32(&o_empty), (j & 1) ^ 1, abort)) break;
+      if (lane == 0) RING_TRACE(2, j, 2);
       __syncwarp();
       tc_fence_after();
-      if (elect_one()) {
-        int slot = win_first % p.NB;
-        uint32_t aP = tmem + b * p.s_stride;  // P: 8 columns per 16 keys
-        for (int wb = 0; wb < p.NWIN; ++wb) {
-          const uint32_t vb = sV + slot * blk_bytes;
-          for (int off = 0; off < p.TM; off += 16) {
-            // V as the MN-major B operand: 64-dim blocks ring_ch apart (LBO),
-            // 8-key groups 1024 bytes apart (SBO)
-            mma_bf16_ts(tmem + p.o_col, aP, smem_desc_sw128(vb + off * 128, ring_ch, 1024),
-                        idesc_pv, (wb | off) != 0 ? 1u : 0u);
-            aP += 8;
-          }
-          slot = slot + 1 == p.NB ? 0 : slot + 1;
-        }
+      // key k of the window sits in ring row (first_row + k) mod ring_keys
+      uint32_t row = static_cast<uint32_t>((win_first % p.NB) * p.TM);
+      const uint32_t aP = tmem + b * p.s_stride;  // P: 8 columns per 16 keys
+      const bool leader = elect_one();
+#pragma unroll
+      for (int kk = 0; kk < BN16; ++kk) {
+        const uint64_t bd = mnmaj | ((sV + row * 128) >> 4);
+        if (leader) mma_bf16_ts(tmem + p.o_col, aP + kk * 8, bd, idesc_pv, kk > 0 ? 1u : 0u);
+        row += 16;
+        if (row >= ring_keys) row -= ring_keys;
+      }
+      if (leader) {
         mma_commit(smem_u32(&o_full));
         mma_commit(smem_u32(&s_empty[b]));
         for (int s = win_first; s < win_next; ++s) mma_commit(smem_u32(&kv_empty[s % p.NB]));
+        RING_TRACE(2, j, 3);
       }
       __syncwarp();
     }
@@ -418,7 +494,7 @@ __global__ void __launch_bounds__(kRingThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

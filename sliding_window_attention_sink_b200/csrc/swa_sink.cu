@@ -120,7 +120,7 @@ int run_ring(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
 }
 
 // Dynamic shared memory available next to the ring kernel's static barriers.
-constexpr size_t kRingSmemLimit = 232448 - 4096;
+constexpr size_t kRingSmemLimit = 232448 - 5120;
 
 // Sliding-window prefill on the persistent ring pipeline when the window's
 // keys for one tile fit one MMA (BN <= 256) and the S/P double buffer plus O
