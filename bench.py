@@ -103,7 +103,7 @@ def recorded_traffic(workload):
 
 # -------------------------------------------------------------------- clocks --
 class ClockSampler:
-    """nvidia-smi samples (200 ms) of this process's GPU during the timed region."""
+    """nvidia-smi samples (50 ms) of this process's GPU during the timed region."""
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
@@ -117,7 +117,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + q,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -308,6 +308,8 @@ def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    if args.steps <= 0:
+        args.steps = 3
     import oracle
     threads = oracle.default_threads()
     case = wl.WORKLOADS[args.workload]
@@ -342,7 +344,8 @@ def run_reference(args, wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=0,
+                    help="timed steps (default: about one second of work, at least 20)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="swa_prefill_32k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -386,6 +389,20 @@ def main():
     runner = (PrefillRunner if is_prefill else DecodeRunner)(case, rank, torch, B, wl)
     stream = torch.cuda.Stream()
     sptr = stream.cuda_stream
+    if args.steps <= 0:
+        # about one second of timed work (enough clock samples), >= 20 steps
+        with torch.cuda.stream(stream):
+            runner.call(sptr)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            runner.call(sptr)
+            b.record(stream)
+        torch.cuda.synchronize()
+        args.steps = int(max(20, min(5000, 1000.0 / max(a.elapsed_time(b), 1e-3))))
+        if world > 1:  # every rank must time the same number of steps
+            t = torch.tensor([args.steps], device="cuda", dtype=torch.int64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            args.steps = int(t.item())
 
     # CPU baseline (rank 0, N = 1), before the GPU timing so it does not overlap
     cpu = None
