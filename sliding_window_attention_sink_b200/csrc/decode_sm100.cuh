@@ -86,22 +86,34 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Shared memory: K and V [KP][D+8], Q [32][D+8], P [32][KP+8] (bf16),
-// then per-warp row maxima and two row sums [4][32] and per-row l [32] (fp32).
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+
+constexpr int kDecodeWarps = 8;
+
+// Shared memory: K and V [KP][D+8], Q [32][D+8], P [32][KP+8] (bf16), then
+// per-warp row maxima and the two row sums [8][32] and per-row l [32] (fp32).
 __host__ __device__ constexpr int decode_row_stride(int D) { return D + 8; }
 __host__ __device__ inline size_t decode_smem_bytes(int D, int KP) {
   const int ld = decode_row_stride(D);
   return static_cast<size_t>(2 * KP * ld + 32 * ld + 32 * (KP + 8)) * 2 +
-         (4 * 32 * 3 + 32) * sizeof(float);
+         (kDecodeWarps * 32 * 3 + 32) * sizeof(float);
 }
 
 template <int D, int MT>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kDecodeWarps * 32, 2)
     decode_sm100_kernel(const DecodeParams p) {
+  constexpr int NWP = kDecodeWarps;
+  constexpr int NT_ = NWP * 32;
   constexpr int LD = D + 8;        // bf16 elements per smem row (conflict-free ldmatrix)
   constexpr int CPR = D / 8;       // 16-byte chunks per row
   constexpr int RP = MT * 16;      // padded query rows
-  constexpr int NTW = 9;           // max n8 key tiles per warp (KP <= 272)
+  constexpr int NTW = 5;           // max n8 key tiles per warp (KP <= 272)
+  constexpr int DW = D / NWP;      // PV: head-dim columns per warp (16 or 8)
+  constexpr int NTO = DW / 8;      // n8 tiles per warp in PV (2 or 1)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int KP = p.KP;
   __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smem_raw);
@@ -109,10 +121,10 @@ __global__ void __launch_bounds__(128)
   __nv_bfloat16* Qs = Vs + KP * LD;
   __nv_bfloat16* Ps = Qs + 32 * LD;
   const int LDP = KP + 8;
-  float* red_max = reinterpret_cast<float*>(Ps + 32 * LDP);  // [4][32]
-  float* red_sum = red_max + 4 * 32;                          // [4][32]
-  float* red_sum_x = red_sum + 4 * 32;                        // [4][32]
-  float* row_l = red_sum_x + 4 * 32;                          // [32]
+  float* red_max = reinterpret_cast<float*>(Ps + 32 * LDP);  // [NWP][32]
+  float* red_lr = red_max + NWP * 32;                         // [NWP][32]
+  float* red_lx = red_lr + NWP * 32;                          // [NWP][32]
+  float* row_l = red_lx + NWP * 32;                           // [32]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.x / p.Hkv;
@@ -126,7 +138,7 @@ __global__ void __launch_bounds__(128)
 
   // ---- loads: group 0 = Q and K rows, group 1 = V rows ---------------------
   const uint32_t sQ = smem_u32(Qs), sK = smem_u32(Ks), sV = smem_u32(Vs);
-  for (int idx = tid; idx < RP * CPR; idx += 128) {
+  for (int idx = tid; idx < RP * CPR; idx += NT_) {
     const int r = idx / CPR, c = idx - r * CPR;
     const uint32_t dst = sQ + (r * LD + c * 8) * 2;
     if (r < p.R) {
@@ -136,32 +148,47 @@ __global__ void __launch_bounds__(128)
       st_shared_zero16(dst);
     }
   }
-  for (int idx = tid; idx < KP * CPR; idx += 128) {
+  const __nv_bfloat16* kr = p.k_ring + (static_cast<size_t>(b) * W * p.Hkv + g) * D;
+  const __nv_bfloat16* kn = p.k_new + (static_cast<size_t>(b) * n_q * p.Hkv + g) * D;
+  const __nv_bfloat16* vr = p.v_ring + (static_cast<size_t>(b) * W * p.Hkv + g) * D;
+  const __nv_bfloat16* vn = p.v_new + (static_cast<size_t>(b) * n_q * p.Hkv + g) * D;
+  const size_t kstride = static_cast<size_t>(p.Hkv) * D;  // elements between consecutive keys
+  for (int idx = tid; idx < KP * CPR; idx += NT_) {
     const int key = idx / CPR, c = idx - key * CPR;
     const uint32_t dst = sK + (key * LD + c * 8) * 2;
-    if (key < W)
-      cp_async16(dst, p.k_ring + ((static_cast<size_t>(b) * W + key) * p.Hkv + g) * D + c * 8);
-    else if (key < W + n_q)
-      cp_async16(dst, p.k_new + ((static_cast<size_t>(b) * n_q + key - W) * p.Hkv + g) * D + c * 8);
-    else
-      st_shared_zero16(dst);
+    if (key < W) cp_async16(dst, kr + key * kstride + c * 8);
+    else if (key < W + n_q) cp_async16(dst, kn + (key - W) * kstride + c * 8);
+    else st_shared_zero16(dst);
   }
   cp_async_commit();
-  for (int idx = tid; idx < KP * CPR; idx += 128) {
+  for (int idx = tid; idx < KP * CPR; idx += NT_) {
     const int key = idx / CPR, c = idx - key * CPR;
     const uint32_t dst = sV + (key * LD + c * 8) * 2;
-    if (key < W)
-      cp_async16(dst, p.v_ring + ((static_cast<size_t>(b) * W + key) * p.Hkv + g) * D + c * 8);
-    else if (key < W + n_q)
-      cp_async16(dst, p.v_new + ((static_cast<size_t>(b) * n_q + key - W) * p.Hkv + g) * D + c * 8);
-    else
-      st_shared_zero16(dst);
+    if (key < W) cp_async16(dst, vr + key * kstride + c * 8);
+    else if (key < W + n_q) cp_async16(dst, vn + (key - W) * kstride + c * 8);
+    else st_shared_zero16(dst);
   }
   cp_async_commit();
+
+  // ---- this thread's rows (fragment rows lane/4 and lane/4 + 8 per m-tile) --
+  // ring slot s holds the token at position P - W + rel(s), rel(s) = (s - P) mod W;
+  // query t sees it iff rel >= max(t + 1, W - P); new token u iff u <= t.
+  const int Pmod = P % W;
+  int trow[MT][2], thr[MT][2];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int row = mt * 16 + (lane >> 2) + hf * 8;
+      const int t = row < p.R ? row / G : -1;  // -1: padding row, sees nothing
+      trow[mt][hf] = t;
+      thr[mt][hf] = t >= 0 ? max(t + 1, W - P) : 0x7fffffff;
+    }
+
   cp_async_wait<1>();
   __syncthreads();
 
-  // ---- S = Q K^T: warp w takes key tiles w, w+4, w+8, ... ------------------
+  // ---- S = Q K^T: warp w takes key tiles w, w+8, w+16, ... ----------------
   const int NT = KP / 8;
   float s[MT][NTW][4];
 #pragma unroll
@@ -170,7 +197,6 @@ __global__ void __launch_bounds__(128)
     for (int j = 0; j < NTW; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) s[mt][j][e] = 0.f;
-
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     uint32_t a[MT][4];
@@ -182,7 +208,7 @@ __global__ void __launch_bounds__(128)
     }
 #pragma unroll
     for (int j = 0; j < NTW; ++j) {
-      const int nt = warp + 4 * j;
+      const int nt = warp + NWP * j;
       if (nt < NT) {
         uint32_t b0, b1;
         const int key = nt * 8 + (lane & 7);
@@ -195,39 +221,31 @@ __global__ void __launch_bounds__(128)
     }
   }
 
-  // ---- mask, scale to log2 units, per-warp row max -------------------------
-  const int Pmod = P % W;
+  // ---- mask, scale to log2 units, per-warp row max --------------------------
   float mloc[MT][2];
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
-    mloc[mt][0] = -INFINITY;
-    mloc[mt][1] = -INFINITY;
-  }
+  for (int mt = 0; mt < MT; ++mt) mloc[mt][0] = mloc[mt][1] = -INFINITY;
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
+  for (int j = 0; j < NTW; ++j) {
+    const int nt = warp + NWP * j;
 #pragma unroll
-    for (int j = 0; j < NTW; ++j) {
-      const int nt = warp + 4 * j;
+    for (int e2 = 0; e2 < 2; ++e2) {
+      const int col = nt * 8 + 2 * (lane & 3) + e2;
+      // kind of key: ring (visible iff rel >= thr), new (iff u <= t) or none
+      int rel = col - Pmod;
+      if (rel < 0) rel += W;
+      const bool ring = nt < NT && col < W;
+      const bool isnew = nt < NT && col >= W && col < W + n_q;
+      const int u = col - W;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int row = mt * 16 + (lane >> 2) + ((e >> 1) << 3);
-        const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
-        bool vis = false;
-        if (nt < NT && row < p.R) {
-          const int t = row / G;
-          if (col < W) {
-            int rel = col - Pmod;
-            if (rel < 0) rel += W;
-            const int pos_key = P - W + rel;  // absolute position held by slot col
-            vis = pos_key >= 0 && pos_key >= P + t - W + 1;
-          } else if (col < W + n_q) {
-            vis = (col - W) <= t;
-          }
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const bool vis = (ring && rel >= thr[mt][hf]) || (isnew && u <= trow[mt][hf]);
+          float& x = s[mt][j][hf * 2 + e2];
+          x = vis ? x * p.scale_log2 : -INFINITY;
+          mloc[mt][hf] = fmaxf(mloc[mt][hf], x);
         }
-        const float x = vis ? s[mt][j][e] * p.scale_log2 : -INFINITY;
-        s[mt][j][e] = x;
-        mloc[mt][e >> 1] = fmaxf(mloc[mt][e >> 1], x);
-      }
     }
   }
 #pragma unroll
@@ -242,32 +260,29 @@ __global__ void __launch_bounds__(128)
   __syncthreads();
 
   // ---- row max over warps and the sink; P = exp2(x - m) -> smem; row sums --
-  float mrow[MT][2];
+  float mrow[MT][2], srow[MT][2];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const int row = mt * 16 + (lane >> 2) + hf * 8;
-      float m = -INFINITY;
-      if (row < p.R && p.sink != nullptr) m = __ldg(p.sink + g * G + row % G) * kLog2e;
+      const float sk = (trow[mt][hf] >= 0 && p.sink != nullptr)
+                           ? __ldg(p.sink + g * G + (row - trow[mt][hf] * G)) * kLog2e
+                           : -INFINITY;
+      float m = sk;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) m = fmaxf(m, red_max[w * 32 + row]);
+      for (int w = 0; w < NWP; ++w) m = fmaxf(m, red_max[w * 32 + row]);
       mrow[mt][hf] = (m == -INFINITY) ? 0.f : m;
+      srow[mt][hf] = sk;
     }
-  // lloc sums P as rounded to bf16 (normalises O consistently with the PV
-  // product); lexact sums it in fp32 (for the LSE).
-  float lloc[MT][2], lexact[MT][2];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
-    lloc[mt][0] = lloc[mt][1] = 0.f;
-    lexact[mt][0] = lexact[mt][1] = 0.f;
-  }
+  float lr[MT][2], lx[MT][2];
   const uint32_t sP = smem_u32(Ps);
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
+    lr[mt][0] = lr[mt][1] = lx[mt][0] = lx[mt][1] = 0.f;
 #pragma unroll
     for (int j = 0; j < NTW; ++j) {
-      const int nt = warp + 4 * j;
+      const int nt = warp + NWP * j;
       if (nt < NT) {
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
@@ -276,8 +291,8 @@ __global__ void __launch_bounds__(128)
           const float p0 = ex2(s[mt][j][2 * hf] - mrow[mt][hf]);
           const float p1 = ex2(s[mt][j][2 * hf + 1] - mrow[mt][hf]);
           const uint32_t pk = pack_bf16x2(p0, p1);
-          lloc[mt][hf] += bf16lo_to_f32(pk) + bf16hi_to_f32(pk);
-          lexact[mt][hf] += p0 + p1;
+          lr[mt][hf] += bf16lo_to_f32(pk) + bf16hi_to_f32(pk);
+          lx[mt][hf] += p0 + p1;
           asm volatile("st.shared.b32 [%0], %1;" ::"r"(sP + (row * LDP + col) * 2), "r"(pk)
                        : "memory");
         }
@@ -288,52 +303,52 @@ __global__ void __launch_bounds__(128)
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      float v = lloc[mt][hf], x = lexact[mt][hf];
+      float v = lr[mt][hf], x = lx[mt][hf];
       v += __shfl_xor_sync(0xffffffffu, v, 1);
       v += __shfl_xor_sync(0xffffffffu, v, 2);
       x += __shfl_xor_sync(0xffffffffu, x, 1);
       x += __shfl_xor_sync(0xffffffffu, x, 2);
       if ((lane & 3) == 0) {
-        red_sum[warp * 32 + mt * 16 + (lane >> 2) + hf * 8] = v;
-        red_sum_x[warp * 32 + mt * 16 + (lane >> 2) + hf * 8] = x;
+        red_lr[warp * 32 + mt * 16 + (lane >> 2) + hf * 8] = v;
+        red_lx[warp * 32 + mt * 16 + (lane >> 2) + hf * 8] = x;
       }
     }
   cp_async_wait<0>();
   __syncthreads();
+  // row sums over warps plus the sink term; LSE (one thread per row)
   if (tid < RP) {
     const int row = tid;
-    float m = -INFINITY;
-    if (row < p.R && p.sink != nullptr) m = __ldg(p.sink + g * G + row % G) * kLog2e;
-    for (int w = 0; w < 4; ++w) m = fmaxf(m, red_max[w * 32 + row]);
+    float m = -INFINITY, sk = -INFINITY;
+    const int t = row < p.R ? row / G : -1;
+    if (t >= 0 && p.sink != nullptr) sk = __ldg(p.sink + g * G + (row - t * G)) * kLog2e;
+    m = sk;
+    for (int w = 0; w < NWP; ++w) m = fmaxf(m, red_max[w * 32 + row]);
     const float mb = (m == -INFINITY) ? 0.f : m;
-    float l = 0.f, lx = 0.f;
-    for (int w = 0; w < 4; ++w) {
-      l += red_sum[w * 32 + row];
-      lx += red_sum_x[w * 32 + row];
+    float l = 0.f, lxs = 0.f;
+    for (int w = 0; w < NWP; ++w) {
+      l += red_lr[w * 32 + row];
+      lxs += red_lx[w * 32 + row];
     }
-    if (row < p.R && p.sink != nullptr) {
-      const float ts = ex2(__ldg(p.sink + g * G + row % G) * kLog2e - mb);
+    if (sk != -INFINITY) {
+      const float ts = ex2(sk - mb);
       l += ts;
-      lx += ts;
+      lxs += ts;
     }
     row_l[row] = l;
-    if (row < p.R && p.lse != nullptr) {
-      const int t = row / G, hh = row - t * G;
-      p.lse[(static_cast<size_t>(b) * n_q + t) * p.Hq + g * G + hh] = (mb + log2f(lx)) * kLn2;
-    }
+    if (t >= 0 && p.lse != nullptr)
+      p.lse[(static_cast<size_t>(b) * n_q + t) * p.Hq + g * G + (row - t * G)] =
+          (mb + lg2(lxs)) * kLn2;
   }
   __syncthreads();
 
-  // ---- O = P V: warp w takes head-dim columns [w*D/4, (w+1)*D/4) -----------
-  constexpr int DW = D / 4;       // columns per warp
-  constexpr int NTO = DW / 8;     // n8 tiles per warp (4 for D=128, 2 for D=64)
+  // ---- O = P V: warp w takes head-dim columns [w*DW, (w+1)*DW) --------------
   float acc[MT][NTO][4];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-    for (int j = 0; j < NTO; ++j)
+    for (int jn = 0; jn < NTO; ++jn)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[mt][j][e] = 0.f;
+      for (int e = 0; e < 4; ++e) acc[mt][jn][e] = 0.f;
   for (int kk = 0; kk < KP / 16; ++kk) {
     uint32_t a[MT][4];
 #pragma unroll
@@ -342,18 +357,22 @@ __global__ void __launch_bounds__(128)
       const int col = kk * 16 + (lane >> 4) * 8;
       ldsm_x4(sP + (row * LDP + col) * 2, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
     }
-#pragma unroll
-    for (int j = 0; j < NTO; j += 2) {
-      // two n8 tiles of V^T: keys kk*16..+15, dims warp*DW + j*8 .. +15
+    const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    if (NTO == 2) {
       uint32_t b0, b1, b2, b3;
-      const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int col = warp * DW + j * 8 + (lane >> 4) * 8;
+      const int col = warp * DW + (lane >> 4) * 8;
       ldsm_x4_t(sV + (key * LD + col) * 2, b0, b1, b2, b3);
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        mma_16816(acc[mt][j], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
-        mma_16816(acc[mt][j + 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b2, b3);
+        mma_16816(acc[mt][0], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
+        mma_16816(acc[mt][NTO - 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b2, b3);
       }
+    } else {
+      uint32_t b0, b1;
+      ldsm_x2_t(sV + (key * LD + warp * DW) * 2, b0, b1);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+        mma_16816(acc[mt][0], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
     }
   }
 
@@ -362,16 +381,17 @@ __global__ void __launch_bounds__(128)
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const int row = mt * 16 + (lane >> 2) + hf * 8;
-      if (row < p.R) {
-        const int t = row / G, hh = row - t * G;
+      const int t = trow[mt][hf];
+      if (t >= 0) {
+        const int row = mt * 16 + (lane >> 2) + hf * 8;
         const float inv_l = 1.f / row_l[row];
-        __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * n_q + t) * p.Hq + g * G + hh) * D;
+        __nv_bfloat16* orow =
+            p.o + ((static_cast<size_t>(b) * n_q + t) * p.Hq + g * G + (row - t * G)) * D;
 #pragma unroll
-        for (int j = 0; j < NTO; ++j) {
-          const int col = warp * DW + j * 8 + 2 * (lane & 3);
+        for (int jn = 0; jn < NTO; ++jn) {
+          const int col = warp * DW + jn * 8 + 2 * (lane & 3);
           *reinterpret_cast<uint32_t*>(orow + col) =
-              pack_bf16x2(acc[mt][j][2 * hf] * inv_l, acc[mt][j][2 * hf + 1] * inv_l);
+              pack_bf16x2(acc[mt][jn][2 * hf] * inv_l, acc[mt][jn][2 * hf + 1] * inv_l);
         }
       }
     }

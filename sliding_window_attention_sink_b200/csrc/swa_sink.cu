@@ -243,7 +243,7 @@ int launch_decode(const swa::DecodeParams& p, cudaStream_t st) {
   const size_t smem = swa::decode_smem_bytes(D, p.KP);
   auto kern = swa::decode_sm100_kernel<D, MT>;
   if (ensure_smem_attr(kern, smem, g_attr_dec[D == 128][MT - 1]) != SWA_OK) return SWA_ERR_CUDA;
-  kern<<<static_cast<unsigned>(p.B) * p.Hkv, 128, smem, st>>>(p);
+  kern<<<static_cast<unsigned>(p.B) * p.Hkv, swa::kDecodeWarps * 32, smem, st>>>(p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SWA_OK : cuda_fail("decode launch", e);
 }
