@@ -18,6 +18,7 @@
 
 #include "../../include/swa_sink.h"
 #include "decode_sm100.cuh"
+#include "prefill_chunked_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "prefill_swa_ring_sm100.cuh"
 
@@ -189,6 +190,53 @@ int launch_prefill_ring(const void* q, const void* k, const void* v, const int32
   }
 }
 
+size_t g_attr_chunked[2][kMaxDevices];
+
+// Global attention, and sliding windows too wide for the ring pipeline, on the
+// persistent chunked pipeline (128-key chunks) when the query heads of one kv
+// head pack a 128-row tile (G divides 128). SWA_ERR_UNSUPPORTED otherwise.
+template <int D>
+int launch_prefill_chunked(const void* q, const void* k, const void* v, const int32_t* cu,
+                           int num_seqs, int total, int Hq, int Hkv, int window,
+                           const float* sink, float scale, void* o, float* lse, cudaStream_t st) {
+  const int G = Hq / Hkv;
+  if (G < 1 || 128 % G != 0) return SWA_ERR_UNSUPPORTED;
+  const int TM = 128 / G;
+  swa::ChunkParams p;
+  p.cu_seqlens = cu;
+  p.num_seqs = num_seqs;
+  p.total = total;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.TM = TM;
+  p.window = window;
+  p.n_tok_tiles = (total + TM - 1) / TM;
+  const long long n_tiles = static_cast<long long>(p.n_tok_tiles) * Hkv;
+  if (n_tiles > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  p.n_tiles = static_cast<int>(n_tiles);
+  p.sink = sink;
+  p.scale_log2 = scale * swa::kLog2e;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.q_box_bytes = 128u * TM * G;
+
+  CUtensorMap tq, tk, tv;
+  if (encode_3d(&tq, q, D, Hq, total, 64, G, TM) != SWA_OK) return SWA_ERR_CUDA;
+  if (encode_3d(&tk, k, D, Hkv, total, 64, 1, swa::kChunkKeys) != SWA_OK) return SWA_ERR_CUDA;
+  if (encode_3d(&tv, v, D, Hkv, total, 64, 1, swa::kChunkKeys) != SWA_OK) return SWA_ERR_CUDA;
+
+  const size_t smem = swa::chunked_smem_bytes(D);
+  auto kern = swa::prefill_chunked_kernel<D>;
+  if (ensure_smem_attr(kern, smem, g_attr_chunked[D == 128]) != SWA_OK) return SWA_ERR_CUDA;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)", 0);
+  const int grid = std::min(nsm, p.n_tiles);
+  kern<<<grid, swa::kChunkThreads, smem, st>>>(tq, tk, tv, p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SWA_OK : cuda_fail("chunked prefill launch", e);
+}
+
 template <int D>
 int launch_prefill(const void* q, const void* k, const void* v, const int32_t* cu, int num_seqs,
                    int total, int Hq, int Hkv, int window, const float* sink, float scale,
@@ -293,6 +341,15 @@ int swa_sink_attn_fwd(const void* q, const void* k, const void* v, const int32_t
                            : launch_prefill_ring<128>(q, k, v, cu_seqlens, num_seqs,
                                                       total_tokens, Hq, Hkv, window, sink,
                                                       softmax_scale, o, lse, st);
+    if (rc != SWA_ERR_UNSUPPORTED) return rc;
+  }
+  {
+    const int rc = D == 64 ? launch_prefill_chunked<64>(q, k, v, cu_seqlens, num_seqs,
+                                                        total_tokens, Hq, Hkv, window, sink,
+                                                        softmax_scale, o, lse, st)
+                           : launch_prefill_chunked<128>(q, k, v, cu_seqlens, num_seqs,
+                                                         total_tokens, Hq, Hkv, window, sink,
+                                                         softmax_scale, o, lse, st);
     if (rc != SWA_ERR_UNSUPPORTED) return rc;
   }
   if (D == 64)

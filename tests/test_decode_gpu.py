@@ -42,6 +42,11 @@ CASES = [  # (B, n_q, Hq, Hkv, D, W, sink)
     (8, 4, 32, 8, 128, 128, None),
     (8, 2, 8, 1, 128, 64, "normal"),
     (8, 3, 16, 2, 64, 40, "normal"),
+    # rings too large to double-buffer at D = 128 (single-buffer path)
+    (6, 2, 16, 2, 128, 256, "normal"),
+    (6, 4, 32, 8, 128, 200, "uniform2"),
+    # more units than SMs with few rows per unit
+    (400, 1, 8, 8, 64, 128, "normal"),
 ]
 
 

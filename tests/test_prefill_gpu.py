@@ -57,15 +57,32 @@ def test_prefill_matches_oracle(name, seqlens, Hq, Hkv, D, W, sink):
     check(o, lse, ro, rl, name)
 
 
+@pytest.mark.parametrize("W", [128, 0])
 @pytest.mark.parametrize("sval", [30.0, -30.0, 0.0])
-def test_prefill_extreme_sinks(sval):
-    c = wl.prefill_case([200], 8, 1, 128, 128, sigma=0.5, sink=None, seed=3)
+def test_prefill_extreme_sinks(sval, W):
+    n = 200 if W else 450
+    c = wl.prefill_case([n], 8, 1, 128, W, sigma=0.5, sink=None, seed=3)
     sink = torch.full((8,), sval)
     c["sink"] = sink
     o, lse = run_gpu(c)
-    ro, rl, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], 8, 1, 128, 128,
+    ro, rl, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], 8, 1, 128, W,
                                sink=sink)
-    check(o, lse, ro, rl, "sink=%g" % sval)
+    check(o, lse, ro, rl, "sink=%g W=%d" % (sval, W))
+
+
+@pytest.mark.parametrize("W,seqlens", [(0, [900]), (1000, [900]), (0, [300, 700])])
+def test_prefill_growing_logits(W, seqlens):
+    # key norms grow along each sequence, so a row's running max rises by many
+    # log2 units from one 128-key chunk to the next (and falls back at a new
+    # sequence): the online-softmax rescale of O runs often
+    c = wl.prefill_case(seqlens, 8, 1, 128, W, sigma=0.5, sink="normal", seed=11)
+    n = sum(seqlens)
+    ramp = torch.cat([torch.linspace(0.2, 40.0, s) for s in seqlens])
+    c["k"] = (c["k"].float() * ramp[:, None, None]).to(torch.bfloat16)
+    o, lse = run_gpu(c)
+    ro, rl, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], 8, 1, 128, W,
+                               sink=c["sink"])
+    check(o, lse, ro, rl, "growing W=%d n=%d" % (W, n))
 
 
 def test_prefill_window_ge_len_equals_global():
