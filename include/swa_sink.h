@@ -24,9 +24,14 @@
  *
  * Conventions for every call
  * --------------------------
- * - All array pointers are DEVICE pointers owned by the caller; the library
- *   allocates no memory and keeps no per-call state. bf16 arrays must be
- *   16-byte aligned (TMA and 16-byte vector loads); int32/fp32 arrays 4-byte.
+ * - All array pointers are DEVICE pointers owned by the caller. bf16 arrays
+ *   must be 16-byte aligned (TMA and 16-byte vector loads); int32/fp32 arrays
+ *   4-byte. The library's own device memory is one 512-byte buffer per device
+ *   (64 tile-scheduler slots of two counters), allocated, zeroed and
+ *   synchronised by the first swa_sink_attn_fwd call on that device (so make
+ *   that first call outside CUDA-graph capture); each later call takes the
+ *   next slot, and its kernel leaves the slot zero again. Calls whose kernels
+ *   overlap in time must therefore be fewer than 64 apart in call order.
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   Every call is asynchronous on that stream; the caller synchronises.
  * - Argument errors are returned as a negative status BEFORE anything is
@@ -35,8 +40,9 @@
  *   (about 2 s); if one expires, or a device-resident argument is out of range
  *   (a negative pos, an n_accept outside [0, n_q]), the kernel records a flag
  *   readable with swa_sink_device_error() and returns.
- * - Thread-safe: no global mutable host state except a per-device cache of
- *   the driver entry point, filled once under a lock.
+ * - Thread-safe: the global host state (the driver entry point, per-device
+ *   kernel attributes and scheduler buffers, the slot counter) is filled
+ *   under locks or updated atomically.
  */
 #ifndef SWA_SINK_H
 #define SWA_SINK_H

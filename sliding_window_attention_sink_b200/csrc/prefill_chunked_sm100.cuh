@@ -15,20 +15,27 @@
 // heaviest under the causal mask).
 //
 // Online softmax with a lazy rescale: P = exp2(x - m_used) with a per-row
-// reference max m_used that only moves when the running max exceeds it by more
+// reference max m_used that only moves when a chunk's max exceeds it by more
 // than kRescaleLog2 (log2 units; P then stays below 2^8, well inside bf16 and
 // fp32). When it moves, the warp waits for the previous PV MMA and rescales its
-// rows of O (and of the row sums) by exp2(m_old - m_new) in TMEM. The final
+// columns of O (and its row sums) by exp2(m_old - m_new) in TMEM. The final
 // O / l and LSE = m_used + log2(l) are exact whatever m_used is.
 //
-//   warps 0-7   two softmax warpgroups, each taking 64 of the chunk's 128
-//               columns of every row (thread r owns TMEM lane r); chunk maxima
-//               and row sums exchanged through shared memory.
+//   warps 0-7   two softmax warpgroups. Each thread owns one row (TMEM lane)
+//               and reads the chunk's whole S row for the max, so both groups
+//               reach the same m_used without exchanging anything; group hw
+//               then exponentiates columns [64 hw, 64 hw + 64) and writes its
+//               half of P. The groups run unsynchronised, so one group's
+//               exponentials overlap the other's loads and maxima.
 //   warps 8-11  epilogue: after a tile's last PV, O / l -> bf16 -> global (one
-//               256-byte row per thread) and the LSE.
-//   warp 12     TMA producer: Q tile (2 stages), K / V chunks (2 stages).
-//   warp 13     TMEM allocation; issues S = Q K^T into S buffer (chunk & 1).
-//   warp 14     issues O += P V (P from TMEM over S, V MN-major).
+//               row per thread) and the LSE.
+//   warp 12     TMA producer: Q tile (2 stages), K and V chunks (2 stages
+//               each; K of chunk n goes out before V of chunk n - 1).
+//   warp 13     TMEM allocation; S = Q K^T into S buffer (chunk & 1).
+//   warp 14     O += P V (P from its own TMEM buffer, V MN-major).
+//
+// TMEM columns: S buffers [0, 128) and [128, 256), O [256, 256 + D), P buffers
+// [384, 448) and [448, 512) (bf16 pairs, 8 columns per 16 keys).
 //
 // Every wait is bounded (see mbar_wait); nothing here traps.
 #pragma once
@@ -40,6 +47,34 @@
 #include "ptx_sm100.cuh"
 
 namespace swa {
+
+// Pipeline timeline hooks: compiled out unless SWA_CHUNK_TRACE is defined (a
+// profiling build then supplies swa_chunk_trace: clock64 stamps of CTA 0,
+// [role][chunk][event], roles 0 producer, 1 S issuer, 2 PV issuer, 3 and 4 the
+// softmax groups, 5 epilogue; and swa_chunk_cta: globaltimer at each CTA's
+// start and end).
+#ifdef SWA_CHUNK_TRACE
+__device__ unsigned long long* swa_chunk_trace;
+__device__ unsigned long long* swa_chunk_cta;
+#define CHUNK_TRACE(role, j, ev)                                                          \
+  do {                                                                                    \
+    if (blockIdx.x == 0 && (j) < 256)                                                     \
+      swa_chunk_trace[((role) * 256 + (j)) * 8 + (ev)] =                                  \
+          static_cast<unsigned long long>(clock64());                                     \
+  } while (0)
+#define CHUNK_CTA(ev)                                                                     \
+  do {                                                                                    \
+    if (threadIdx.x == 0) swa_chunk_cta[blockIdx.x * 2 + (ev)] = globaltimer_ns();        \
+  } while (0)
+#else
+#define CHUNK_TRACE(role, j, ev) \
+  do {                           \
+    (void)(role);                \
+  } while (0)
+#define CHUNK_CTA(ev) \
+  do {                \
+  } while (0)
+#endif
 
 constexpr int kChunkThreads = 480;   // 15 warps
 constexpr int kChunkKeys = 128;      // keys per chunk (N of S, K of PV)
@@ -73,14 +108,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   constexpr int NCH = D / 64;
   constexpr uint32_t CH = 16384;               // one 64-dim chunk: 128 rows x 128 bytes
   constexpr int HALF = kChunkKeys / 2;         // columns per softmax warpgroup
-  constexpr uint32_t o_col = 2 * kChunkKeys;   // S buffers at columns 0 and 128, O after
+  constexpr uint32_t o_col = 2 * kChunkKeys;   // after the two S buffers
+  constexpr uint32_t p_col = 384;              // two P buffers of 64 columns
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full[2], q_empty[2], k_full[2], k_empty[2];
   __shared__ __align__(8) uint64_t v_full[2], v_empty[2];
-  __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], pv_done;
+  __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
   __shared__ __align__(8) uint64_t o_full, o_empty, l_full, l_free;
-  __shared__ float red_max[2][2][128], red_sum[2][2][128];
-  __shared__ float l_s[128], m_s[128];
+  __shared__ float red_lr[2][128], red_lx[2][128], m_s[128];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -102,13 +137,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       mbar_init(smem_u32(&v_full[s]), 1);
       mbar_init(smem_u32(&v_empty[s]), 1);
       mbar_init(smem_u32(&s_full[s]), 1);
-      mbar_init(smem_u32(&s_empty[s]), 1);
+      mbar_init(smem_u32(&s_empty[s]), 8);
       mbar_init(smem_u32(&p_full[s]), 8);
+      mbar_init(smem_u32(&p_empty[s]), 1);
     }
-    mbar_init(smem_u32(&pv_done), 1);
     mbar_init(smem_u32(&o_full), 1);
     mbar_init(smem_u32(&o_empty), 4);
-    mbar_init(smem_u32(&l_full), 4);
+    mbar_init(smem_u32(&l_full), 8);
     mbar_init(smem_u32(&l_free), 4);
     abort_sh = 0;
     fence_barrier_init();
@@ -121,6 +156,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  CHUNK_CTA(0);
 
   // the k-th tile of this CTA: heaviest (last) token tiles first
   auto tile_of = [&](int k, int& g, int& tb) {
@@ -142,13 +178,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 
   if (warp < 8) {
     // ===================== softmax (two warpgroups) ==========================
-    const int hw = warp >> 2;              // which 64 columns of the chunk
+    const int hw = warp >> 2;              // which 64 columns this group exponentiates
     const int r = 32 * (warp & 3) + lane;  // TMEM lane == tile row
     const int tok = r / p.G, hh = r - tok * p.G;
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-    int n = 0;  // chunk counter over the CTA's tiles; S / P buffer n & 1
-    for (int k = 0; k < ntile; ++k) {
+    int n = 0;  // chunk counter over the CTA's tiles; buffers n & 1
+    bool ok = true;
+    for (int k = 0; k < ntile && ok; ++k) {
       int g, tb, lo, nchunk;
       tile_of(k, g, tb);
       tile_keys(tb, lo, nchunk);
@@ -167,48 +204,58 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const int all_hi = t0;
       const float sink2 = (valid && p.sink != nullptr) ? __ldg(p.sink + h) * kLog2e : -INFINITY;
       float m_used = sink2;        // reference max of P (log2 units)
-      float l_r = 0.f, l_x = 0.f;  // this half's sums relative to m_used
-      bool stop = false;
+      float l_r = 0.f, l_x = 0.f;  // this group's sums relative to m_used
       for (int c = 0; c < nchunk; ++c, ++n) {
         const int b = n & 1;
-        const int c0 = lo + c * kChunkKeys + hw * HALF;  // key of this half's column 0
-        const bool ok = mbar_wait(smem_u32(&s_full[b]), (n >> 1) & 1, abort);
-        __syncwarp();
-        tc_fence_after();
-        const uint32_t tS = tmem + lane_off + b * kChunkKeys;
-        uint32_t v[HALF];
-#pragma unroll
-        for (int q = 0; q < HALF / 16; ++q) tmem_ld16_at(tS + hw * HALF + q * 16, &v[q * 16]);
-        tmem_ld_wait();
-        if (!(c0 >= all_lo && c0 + HALF - 1 <= all_hi)) {  // a row's edge is in this half
-          const int cmin = row_lo - c0;
-          const int cmax = row_hi - c0;
-#pragma unroll
-          for (int e = 0; e < HALF; ++e)
-            if (e < cmin || e > cmax) v[e] = 0xff800000u;  // -inf
-        }
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < HALF; e += 4) {
-          mx0 = max3(mx0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-          mx1 = max3(mx1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-        }
-        red_max[b][hw][r] = fmaxf(mx0, mx1);
-        tc_fence_before();
-        if (named_bar_any(1, 256, !ok || *abort)) {
-          stop = true;
+        const int trole = 3 + hw;
+        const bool tr = (tid & 127) == 0;
+        if (tr) CHUNK_TRACE(trole, n, 0);
+        if (!mbar_wait(smem_u32(&s_full[b]), (n >> 1) & 1, abort)) {
+          ok = false;
           break;
         }
+        __syncwarp();
         tc_fence_after();
-        const float cm = fmaxf(red_max[b][0][r], red_max[b][1][r]) * p.scale_log2;
+        if (tr) CHUNK_TRACE(trole, n, 1);
+        const uint32_t tS = tmem + lane_off + b * kChunkKeys;
+        // the other group's columns (max only), then this group's (kept)
+        uint32_t v[HALF];
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+          const int hs = pass == 0 ? (hw ^ 1) : hw;
+          const int cb = lo + c * kChunkKeys + hs * HALF;  // key of column 0 of this half
+#pragma unroll
+          for (int q = 0; q < HALF / 16; ++q) tmem_ld16_at(tS + hs * HALF + q * 16, &v[q * 16]);
+          tmem_ld_wait();
+          if (!(cb >= all_lo && cb + HALF - 1 <= all_hi)) {  // a row's edge is in this half
+            const int cmin = row_lo - cb;
+            const int cmax = row_hi - cb;
+#pragma unroll
+            for (int e = 0; e < HALF; ++e)
+              if (e < cmin || e > cmax) v[e] = 0xff800000u;  // -inf
+          }
+#pragma unroll
+          for (int e = 0; e < HALF; e += 4) {
+            mx0 = max3(mx0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+            mx1 = max3(mx1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          }
+        }
+        // S of this chunk is in registers: the buffer may take S of chunk n + 2
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&s_empty[b]));
+        if (tr) CHUNK_TRACE(trole, n, 2);
+        const float cm = fmaxf(mx0, mx1) * p.scale_log2;
         // lazy rescale: the reference moves only when the max outgrows it
         const bool grow = cm > m_used + kRescaleLog2;
         if (__any_sync(0xffffffffu, grow)) {
           const float m_new = grow ? cm : m_used;
           const float alpha = grow ? ex2(m_used - m_new) : 1.f;  // exp2(-inf) = 0
-          if (c > 0 && mbar_wait(smem_u32(&pv_done), (n - 1) & 1, abort)) {
-            // the previous chunk's PV has landed in O: rescale this half's
-            // columns of O for this warp's rows
+          // O holds the PVs of chunks before n once PV(n - 1) has completed
+          // (PV(n - 3) has, since this group wrote P(n - 1) after it)
+          if (c > 0 &&
+              mbar_wait(smem_u32(&p_empty[(n - 1) & 1]), ((n - 1) >> 1) & 1, abort)) {
             __syncwarp();
             tc_fence_after();
             const uint32_t tO = tmem + lane_off + o_col + hw * (D / 2);
@@ -227,10 +274,19 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           m_used = m_new;
         }
         const float mb = (m_used == -INFINITY) ? 0.f : m_used;
-        // P = exp2(x - m_used) as bf16 pairs over S columns [hw*HALF/2, ...)
+        if (tr) CHUNK_TRACE(trole, n, 3);
+        // P buffer b is free once PV(n - 2) has completed
+        if (!mbar_wait(smem_u32(&p_empty[b]), ((n >> 1) & 1) ^ 1, abort)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        tc_fence_after();
+        if (tr) CHUNK_TRACE(trole, n, 4);
+        // P = exp2(x - m_used) as bf16 pairs: this group's 32 columns
         uint64_t lr2 = 0, lx2 = 0;
         const uint64_t nm2 = f2_pack(-mb, -mb);
-        const uint32_t tP = tS + hw * (HALF / 2);
+        const uint32_t tP = tmem + lane_off + p_col + b * HALF + hw * (HALF / 2);
 #pragma unroll
         for (int q = 0; q < HALF; q += 16) {
           uint32_t w[8];
@@ -258,29 +314,23 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&p_full[b]));
+        if (tr) CHUNK_TRACE(trole, n, 5);
       }
-      if (stop) break;
-      // tile done: the halves' sums plus the sink term; l and the LSE (log2
-      // units) go to the epilogue
-      red_sum[0][hw][r] = l_r;
-      red_sum[1][hw][r] = l_x;
-      if (named_bar_any(1, 256, *abort != 0)) break;
-      if (hw == 0) {
-        float lr = red_sum[0][0][r] + red_sum[0][1][r];
-        float lx = red_sum[1][0][r] + red_sum[1][1][r];
-        const float mb = (m_used == -INFINITY) ? 0.f : m_used;
-        if (sink2 != -INFINITY) {
-          const float ts = ex2(sink2 - mb);
-          lr += ts;
-          lx += ts;
-        }
-        if (mbar_wait(smem_u32(&l_free), (k & 1) ^ 1, abort)) {
-          l_s[r] = lr;
-          m_s[r] = mb + lg2(lx);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&l_full));
-        }
+      if (!ok) break;
+      // tile done: this group's sums (group 0 adds the sink term) and the
+      // reference max go to the epilogue once it has read the previous tile's
+      const float mb = (m_used == -INFINITY) ? 0.f : m_used;
+      if (hw == 0 && sink2 != -INFINITY) {
+        const float ts = ex2(sink2 - mb);
+        l_r += ts;
+        l_x += ts;
       }
+      if (!mbar_wait(smem_u32(&l_free), (k & 1) ^ 1, abort)) break;
+      red_lr[hw][r] = l_r;
+      red_lx[hw][r] = l_x;
+      if (hw == 0) m_s[r] = mb;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&l_full));
     }
   } else if (warp < 12) {
     // ======================= epilogue (warps 8..11) ==========================
@@ -290,12 +340,17 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     for (int k = 0; k < ntile && !*abort; ++k) {
       int g, tb;
       tile_of(k, g, tb);
+      if (tid == 256) CHUNK_TRACE(5, k, 0);
       if (!mbar_wait(smem_u32(&o_full), k & 1, abort)) break;
+      if (tid == 256) CHUNK_TRACE(5, k, 1);
       if (!mbar_wait(smem_u32(&l_full), k & 1, abort)) break;
+      if (tid == 256) CHUNK_TRACE(5, k, 2);
       __syncwarp();
       tc_fence_after();
-      const float l = l_s[r];
-      const float lse2 = m_s[r];
+      const float l = red_lr[0][r] + red_lr[1][r];
+      const float lse2 = m_s[r] + lg2(red_lx[0][r] + red_lx[1][r]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&l_free));
       const int i = tb * p.TM + tok;
       const int h = g * p.G + hh;
       const bool valid = i < p.total;
@@ -325,14 +380,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&l_free));
       if (valid && p.lse != nullptr) p.lse[static_cast<size_t>(h) * p.total + i] = lse2 * kLn2;
+      if (tid == 256) CHUNK_TRACE(5, k, 3);
     }
   } else if (warp == 12) {
     // ======================= TMA producer ====================================
     // Order: Q of a tile before its first K; K of chunk n before V of chunk
-    // n - 1, so S can run one chunk ahead of PV.
+    // n - 1, so S can run ahead of PV.
     if (elect_one()) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -364,6 +418,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         for (int c = 0; c < nchunk; ++c, ++n) {
           const int st = n & 1;
           const int key0 = lo + c * kChunkKeys;
+          CHUNK_TRACE(0, n, 0);
           if (!mbar_wait(smem_u32(&k_empty[st]), ((n >> 1) & 1) ^ 1, abort)) {
             ok = false;
             break;
@@ -373,10 +428,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 #pragma unroll
           for (int ch = 0; ch < NCH; ++ch)
             tma_load_3d(sK + (st * NCH + ch) * CH, &tm_k, bar, ch * 64, g, key0);
+          CHUNK_TRACE(0, n, 1);
           if (pend_key >= 0 && !load_v(n - 1, pend_key, pend_g)) {
             ok = false;
             break;
           }
+          CHUNK_TRACE(0, n, 2);
           pend_key = key0;
           pend_g = g;
         }
@@ -397,8 +454,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       if (!mbar_wait(smem_u32(&q_full[qs]), (k >> 1) & 1, abort)) break;
       for (int c = 0; c < nchunk; ++c, ++n) {
         const int b = n & 1;
-        if (!mbar_wait(smem_u32(&s_empty[b]), ((n >> 1) & 1) ^ 1, abort) ||
-            !mbar_wait(smem_u32(&k_full[b]), (n >> 1) & 1, abort)) {
+        if (lane == 0) CHUNK_TRACE(1, n, 0);
+        if (!mbar_wait(smem_u32(&s_empty[b]), ((n >> 1) & 1) ^ 1, abort)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) CHUNK_TRACE(1, n, 1);
+        if (!mbar_wait(smem_u32(&k_full[b]), (n >> 1) & 1, abort)) {
           ok = false;
           break;
         }
@@ -416,6 +478,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           mma_commit(smem_u32(&k_empty[b]));
           if (c == nchunk - 1) mma_commit(smem_u32(&q_empty[qs]));
         }
+        if (lane == 0) CHUNK_TRACE(1, n, 2);
         __syncwarp();
       }
     }
@@ -433,8 +496,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       tile_keys(tb, lo, nchunk);
       for (int c = 0; c < nchunk; ++c, ++n) {
         const int b = n & 1;
-        if (!mbar_wait(smem_u32(&p_full[b]), (n >> 1) & 1, abort) ||
-            (c == 0 && !mbar_wait(smem_u32(&o_empty), (k & 1) ^ 1, abort)) ||
+        if (lane == 0) CHUNK_TRACE(2, n, 0);
+        if (!mbar_wait(smem_u32(&p_full[b]), (n >> 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) CHUNK_TRACE(2, n, 1);
+        if ((c == 0 && !mbar_wait(smem_u32(&o_empty), (k & 1) ^ 1, abort)) ||
             !mbar_wait(smem_u32(&v_full[b]), (n >> 1) & 1, abort)) {
           ok = false;
           break;
@@ -442,17 +510,17 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         __syncwarp();
         tc_fence_after();
         const uint64_t vd = mnmaj | ((sV + b * NCH * CH) >> 4);
-        const uint32_t aP = tmem + b * kChunkKeys;  // P: 8 columns per 16 keys
+        const uint32_t aP = tmem + p_col + b * HALF;  // P: 8 columns per 16 keys
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < kChunkKeys / 16; ++kk)
             mma_bf16_ts(tmem + o_col, aP + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv,
                         (c > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(smem_u32(&s_empty[b]));
+          mma_commit(smem_u32(&p_empty[b]));
           mma_commit(smem_u32(&v_empty[b]));
-          mma_commit(smem_u32(&pv_done));
           if (c == nchunk - 1) mma_commit(smem_u32(&o_full));
         }
+        if (lane == 0) CHUNK_TRACE(2, n, 2);
         __syncwarp();
       }
     }
@@ -460,6 +528,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  CHUNK_CTA(1);
   if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

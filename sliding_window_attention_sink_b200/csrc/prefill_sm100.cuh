@@ -74,6 +74,19 @@ __device__ __forceinline__ int first_key(const int32_t* cu, int num_seqs, int wi
   return lo;
 }
 
+// first_key with the bounds [s_lo, s_hi) of the last sequence looked up kept
+// by the caller: tokens of a thread advance monotonically, so cu_seqlens is
+// read again only when a token leaves that sequence. Start with s_lo > s_hi.
+__device__ __forceinline__ int first_key_cached(const int32_t* cu, int num_seqs, int window,
+                                                int t, int& s_lo, int& s_hi) {
+  if (t < s_lo || t >= s_hi) {
+    const int s = seq_of_token(cu, num_seqs, t);
+    s_lo = __ldg(cu + s);
+    s_hi = __ldg(cu + s + 1);
+  }
+  return window > 0 ? max(s_lo, t - window + 1) : s_lo;
+}
+
 __device__ __forceinline__ int first_visible_key(const PrefillParams& p, int t) {
   return first_key(p.cu_seqlens, p.num_seqs, p.window, t);
 }

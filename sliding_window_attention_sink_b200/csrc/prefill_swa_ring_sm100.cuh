@@ -50,19 +50,35 @@
 namespace swa {
 
 // Pipeline timeline hooks: compiled out unless SWA_RING_TRACE is defined (a
-// profiling build then supplies swa_ring_trace: clock64 stamps of CTA 0,
+// profiling build then supplies swa_ring_trace: clock64 stamps of one CTA,
 // [role][tile][event], roles 0 producer, 1 S issuer, 2 PV issuer, 3 softmax,
-// 4 epilogue).
+// 4 epilogue; and swa_ring_cta_ns: globaltimer and clock64 at each CTA's start
+// and end).
 #ifdef SWA_RING_TRACE
 __device__ unsigned long long* swa_ring_trace;
+__device__ unsigned long long* swa_ring_cta_ns;
+__device__ int swa_ring_trace_block;  // the CTA whose timeline is recorded
+#define RING_CTA(ev)                                                                      \
+  do {                                                                                    \
+    if (threadIdx.x == 0) {                                                               \
+      swa_ring_cta_ns[blockIdx.x * 4 + (ev)] = globaltimer_ns();                          \
+      swa_ring_cta_ns[blockIdx.x * 4 + 2 + (ev)] = static_cast<unsigned long long>(clock64()); \
+      unsigned smid_;                                                                     \
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));                                  \
+      swa_ring_cta_ns[160 * 4 + blockIdx.x] = smid_;                                      \
+    }                                                                                     \
+  } while (0)
 #define RING_TRACE(role, j, ev)                                                           \
   do {                                                                                    \
-    if (blockIdx.x == 0 && (j) < 128)                                                     \
+    if (blockIdx.x == swa_ring_trace_block && (j) < 128)                                 \
       swa_ring_trace[((role) * 128 + (j)) * 8 + (ev)] = static_cast<unsigned long long>(clock64()); \
   } while (0)
 #else
 #define RING_TRACE(role, j, ev) \
   do {                          \
+  } while (0)
+#define RING_CTA(ev) \
+  do {               \
   } while (0)
 #endif
 
@@ -70,6 +86,8 @@ constexpr int kRingMaxBlocks = 16;
 constexpr int kRingMaxQ = 4;
 constexpr int kRingThreads = 480;  // 15 warps
 constexpr int kRingMaxBN16 = 12;   // BN <= 192: a half row fits in registers
+constexpr int kRingRanges = 4;     // tile ranges queued between the producer and the rest
+constexpr int kRingRangeReaders = 14;  // warps other than the producer
 
 struct RingParams {
   const int32_t* cu_seqlens;
@@ -89,6 +107,14 @@ struct RingParams {
   uint32_t q_box_bytes;   // bytes of one 64-column Q box
   uint32_t s_stride;      // TMEM column of S / P buffer b is b * s_stride
   uint32_t o_col;         // TMEM column of O
+  // Tile schedule. Tiles f = g * n_tok_tiles + tb are taken in ranges of
+  // consecutive f: CTA c first takes [c * static_tiles, (c + 1) * static_tiles),
+  // then draws ranges of dyn_span tiles from dyn_base on through sched[0].
+  // sched[1] counts finished CTAs; the last one sets both back to zero.
+  unsigned int* sched;
+  int static_tiles;
+  int dyn_base;
+  int dyn_span;
 };
 
 // Smem bytes the ring kernel needs (1 KB alignment slack included).
@@ -118,6 +144,9 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], l_free[2];
   __shared__ __align__(8) uint64_t o_full, o_empty;
   __shared__ float red_max[2][128], red_lr[2][128], red_lx[2][128], l_s[2][128];
+  // ranges of tiles, from the producer to the 14 other warps
+  __shared__ __align__(8) uint64_t rq_full[kRingRanges], rq_empty[kRingRanges];
+  __shared__ int rq_lo[kRingRanges], rq_hi[kRingRanges];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -133,11 +162,6 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   const uint32_t sO = sQ + p.NQ * NCH * CH;                         // NCH x CH
   const uint32_t sK = sO + NCH * CH;                                // NCH x ring_ch
   const uint32_t sV = sK + NCH * ring_ch;
-
-  // ---- this CTA's span of (kv head, token tile) pairs ---------------------
-  const long long span_lo = static_cast<long long>(blockIdx.x) * p.n_tiles / gridDim.x;
-  const long long span_hi = static_cast<long long>(blockIdx.x + 1) * p.n_tiles / gridDim.x;
-  const int ntile = static_cast<int>(span_hi - span_lo);
 
   if (tid == 0) {
     for (int s = 0; s < p.NQ; ++s) {
@@ -156,6 +180,10 @@ __global__ void __launch_bounds__(kRingThreads, 1)
     }
     mbar_init(smem_u32(&o_full), 1);
     mbar_init(smem_u32(&o_empty), 4);
+    for (int q = 0; q < kRingRanges; ++q) {
+      mbar_init(smem_u32(&rq_full[q]), 1);
+      mbar_init(smem_u32(&rq_empty[q]), kRingRangeReaders);
+    }
     abort_sh = 0;
     fence_barrier_init();
   }
@@ -167,18 +195,26 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  RING_CTA(0);
 
-  // tile index j (0..ntile-1) -> (g, tb); new blocks it brings into the ring
-  auto tile_of = [&](int j, int& g, int& tb) {
-    const long long f = span_lo + j;
-    g = static_cast<int>(f / p.n_tok_tiles);
-    tb = static_cast<int>(f - static_cast<long long>(g) * p.n_tok_tiles);
+  // tile f -> (kv head g, token tile tb)
+  auto tile_of = [&](int f, int& g, int& tb) {
+    g = f / p.n_tok_tiles;
+    tb = f - g * p.n_tok_tiles;
   };
-  auto new_blocks = [&](int j) {
-    if (j == 0) return p.NWIN;
-    int g, tb;
-    tile_of(j, g, tb);
-    return tb == 0 ? p.NWIN : 1;  // a new kv head restarts the window
+  // key blocks tile tb brings into the ring: the whole window at the start of
+  // a range or of a kv head, else one
+  auto new_blocks = [&](bool range_start, int tb) { return range_start || tb == 0 ? p.NWIN : 1; };
+  // the q-th range of this CTA (every warp but the producer reads each one);
+  // false at the end of the schedule or when a wait gave up
+  auto next_range = [&](int q, int& f0, int& f1) -> bool {
+    const int s = q % kRingRanges;
+    if (!mbar_wait(smem_u32(&rq_full[s]), (q / kRingRanges) & 1, abort)) return false;
+    f0 = rq_lo[s];
+    f1 = rq_hi[s];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&rq_empty[s]));
+    return f0 < f1;
   };
 
   if (warp < 8) {
@@ -188,9 +224,20 @@ __global__ void __launch_bounds__(kRingThreads, 1)
     const int tok = r / p.G, hh = r - tok * p.G;
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-    for (int j = 0; j < ntile; ++j) {
+    // sequence bounds of this row's token and of the tile's last token, and
+    // this row's sink, carried from tile to tile
+    int row_s_lo = 1, row_s_hi = 0, last_s_lo = 1, last_s_hi = 0;
+    int sink_g = -1;
+    float sink_h = -INFINITY;
+    int j = 0;  // tiles done by this CTA: buffer parities
+    bool stop = false;
+    for (int q = 0; !stop; ++q) {
+     int f0 = 0, f1 = 0;
+     // every softmax thread leaves together (a named barrier follows)
+     if (named_bar_any(1, 256, !next_range(q, f0, f1))) break;
+     for (int f = f0; f < f1; ++f, ++j) {
       int g, tb;
-      tile_of(j, g, tb);
+      tile_of(f, g, tb);
       const int b = j & 1;
       const int t0 = tb * p.TM;
       const int i = t0 + tok;
@@ -198,7 +245,7 @@ __global__ void __launch_bounds__(kRingThreads, 1)
       const bool valid = i < p.total;
       int row_lo = 1, row_hi = 0;  // empty unless valid
       if (valid) {
-        row_lo = first_key(p.cu_seqlens, p.num_seqs, p.window, i);
+        row_lo = first_key_cached(p.cu_seqlens, p.num_seqs, p.window, i, row_s_lo, row_s_hi);
         row_hi = i;
       }
       const int c0 = (tb - p.KB) * p.TM + hw * HALF;  // key of this half's column 0
@@ -208,11 +255,16 @@ __global__ void __launch_bounds__(kRingThreads, 1)
       // columns visible to every valid row of the tile (uniform): from the
       // last valid token's first key to the first token itself
       const int t_last = min(t0 + p.TM, p.total) - 1;
-      const int all_lo = first_key(p.cu_seqlens, p.num_seqs, p.window, t_last) - c0;
+      const int all_lo =
+          first_key_cached(p.cu_seqlens, p.num_seqs, p.window, t_last, last_s_lo, last_s_hi) - c0;
       const int all_hi = t0 - c0;
-      const float sink2 = (valid && p.sink != nullptr) ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+      if (g != sink_g) {  // the sink changes with the kv head only
+        sink_g = g;
+        sink_h = p.sink != nullptr ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+      }
+      const float sink2 = valid ? sink_h : -INFINITY;
       if (tid == 0) RING_TRACE(3, j, 0);
-      if (!mbar_wait(smem_u32(&s_full[b]), (j >> 1) & 1, abort)) break;
+      const bool s_ok = mbar_wait(smem_u32(&s_full[b]), (j >> 1) & 1, abort);
       __syncwarp();
       tc_fence_after();
       if (tid == 0) RING_TRACE(3, j, 1);
@@ -242,7 +294,14 @@ __global__ void __launch_bounds__(kRingThreads, 1)
       const float mx = fmaxf(mx0, mx1);
       red_max[hw][r] = mx;
       if (tid == 0) RING_TRACE(3, j, 2);
-      named_bar_sync(1, 256);
+      // both halves have read S: P may go over it. A failed wait anywhere
+      // stops every softmax thread here.
+      tc_fence_before();
+      if (named_bar_any(1, 256, !s_ok || *abort != 0)) {
+        stop = true;
+        break;
+      }
+      tc_fence_after();
       if (tid == 0) RING_TRACE(3, j, 3);
       const float m = fmaxf(sink2, fmaxf(mx, red_max[hw ^ 1][r]) * p.scale_log2);
       const float mb = (m == -INFINITY) ? 0.f : m;
@@ -294,30 +353,40 @@ __global__ void __launch_bounds__(kRingThreads, 1)
           l_x += ts;
         }
         // l for the epilogue, once it has read this buffer's previous value
-        if (!mbar_wait(smem_u32(&l_free[b]), ((j >> 1) & 1) ^ 1, abort)) break;
-        l_s[b][r] = l_r;
+        // (on a failed wait the next tile's barrier stops the loop)
+        if (mbar_wait(smem_u32(&l_free[b]), ((j >> 1) & 1) ^ 1, abort)) l_s[b][r] = l_r;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&p_full[b]));
       if (tid == 0) RING_TRACE(3, j, 6);
       if (hw == 0 && valid && p.lse != nullptr)
         p.lse[static_cast<size_t>(h) * p.total + i] = (mb + lg2(l_x)) * kLn2;
+     }
     }
   } else if (warp < 12) {
     // ======================= epilogue (warps 8..11) ==========================
     const int r = 32 * (warp & 3) + lane;
     const bool issuer = tid == 256;
     const uint32_t tO = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + p.o_col;
-    for (int j = 0; j < ntile; ++j) {
+    int j = 0;
+    bool stop = false;
+    for (int q = 0; !stop; ++q) {
+     int f0 = 0, f1 = 0;
+     if (named_bar_any(2, 128, !next_range(q, f0, f1))) break;
+     for (int f = f0; f < f1; ++f, ++j) {
       int g, tb;
-      tile_of(j, g, tb);
+      tile_of(f, g, tb);
       const int b = j & 1;
       if (issuer) RING_TRACE(4, j, 0);
-      if (!mbar_wait(smem_u32(&o_full), j & 1, abort)) break;
-      if (issuer) RING_TRACE(4, j, 1);
       // p_full[b] of this tile completed before PV was issued; waiting on it
-      // here orders the softmax's write of l_s[b] before the read below
-      if (!mbar_wait(smem_u32(&p_full[b]), (j >> 1) & 1, abort)) break;
+      // too orders the softmax's write of l_s[b] before the read below
+      const bool ok = mbar_wait(smem_u32(&o_full), j & 1, abort) &&
+                      mbar_wait(smem_u32(&p_full[b]), (j >> 1) & 1, abort);
+      if (named_bar_any(2, 128, !ok)) {  // the epilogue warps leave together
+        stop = true;
+        break;
+      }
+      if (issuer) RING_TRACE(4, j, 1);
       __syncwarp();
       tc_fence_after();
       const float l = l_s[b][r];
@@ -361,63 +430,120 @@ __global__ void __launch_bounds__(kRingThreads, 1)
         }
       }
       if (issuer) RING_TRACE(4, j, 3);
+     }
     }
     if (issuer) tma_store_wait_all<0>();
   } else if (warp == 12) {
-    // ======================= TMA producer ====================================
+    // ================= TMA producer and tile scheduler ======================
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_o);
-      int nload = 0;
-      for (int j = 0; j < ntile && !*abort; ++j) {
-        int g, tb;
-        tile_of(j, g, tb);
-        const int st = j % p.NQ;
-        RING_TRACE(0, j, 0);
-        if (!mbar_wait(smem_u32(&q_empty[st]), ((j / p.NQ) & 1) ^ 1, abort)) break;
-        RING_TRACE(0, j, 1);
-        mbar_arrive_expect_tx(smem_u32(&q_full[st]), NCH * p.q_box_bytes);
+      int nload = 0, j = 0, q = 0;
+      // hand range [f0, f1) to the other warps as the q-th; f0 >= f1 ends
+      auto publish = [&](int f0, int f1) -> bool {
+        const int s = q % kRingRanges;
+        if (!mbar_wait(smem_u32(&rq_empty[s]), ((q / kRingRanges) & 1) ^ 1, abort)) return false;
+        rq_lo[s] = f0;
+        rq_hi[s] = f1;
+        mbar_arrive(smem_u32(&rq_full[s]));
+        ++q;
+        return true;
+      };
+      bool ok = true;
+      for (int k = 0; ok && !*abort; ++k) {
+        int f0, f1;
+        if (k == 0) {  // the static part
+          f0 = static_cast<int>(blockIdx.x) * p.static_tiles;
+          f1 = min(f0 + p.static_tiles, p.n_tiles);
+          if (f0 >= f1) continue;
+        } else {  // ranges drawn while any are left
+          const unsigned int d = atomicAdd(p.sched, 1u);
+          const long long s0 = p.dyn_base + static_cast<long long>(d) * p.dyn_span;
+          if (s0 >= p.n_tiles) break;
+          f0 = static_cast<int>(s0);
+          f1 = min(f0 + p.dyn_span, p.n_tiles);
+        }
+        if (!publish(f0, f1)) break;
+        for (int f = f0; f < f1 && ok; ++f, ++j) {
+          int g, tb;
+          tile_of(f, g, tb);
+          const int st = j % p.NQ;
+          RING_TRACE(0, j, 0);
+          if (!mbar_wait(smem_u32(&q_empty[st]), ((j / p.NQ) & 1) ^ 1, abort)) {
+            ok = false;
+            break;
+          }
+          RING_TRACE(0, j, 1);
+          mbar_arrive_expect_tx(smem_u32(&q_full[st]), NCH * p.q_box_bytes);
 #pragma unroll
-        for (int ch = 0; ch < NCH; ++ch)
-          tma_load_3d(sQ + (st * NCH + ch) * CH, &tm_q, smem_u32(&q_full[st]), ch * 64, g * p.G,
-                      tb * p.TM);
-        const int nnew = new_blocks(j);
-        const int first_kb = tb - nnew + 1;  // absolute key block of the first new block
-        for (int n = 0; n < nnew; ++n, ++nload) {
-          const int slot = nload % p.NB;
-          if (!mbar_wait(smem_u32(&kv_empty[slot]), ((nload / p.NB) & 1) ^ 1, abort)) break;
-          const uint32_t bar = smem_u32(&kv_full[slot]);
-          mbar_arrive_expect_tx(bar, 2u * NCH * blk_bytes);
-          const int key0 = (first_kb + n) * p.TM;  // may be negative: zero fill
+          for (int ch = 0; ch < NCH; ++ch)
+            tma_load_3d(sQ + (st * NCH + ch) * CH, &tm_q, smem_u32(&q_full[st]), ch * 64,
+                        g * p.G, tb * p.TM);
+          const int nnew = new_blocks(f == f0, tb);
+          const int first_kb = tb - nnew + 1;  // absolute key block of the first new block
+          for (int n = 0; n < nnew; ++n, ++nload) {
+            const int slot = nload % p.NB;
+            if (!mbar_wait(smem_u32(&kv_empty[slot]), ((nload / p.NB) & 1) ^ 1, abort)) {
+              ok = false;
+              break;
+            }
+            const uint32_t bar = smem_u32(&kv_full[slot]);
+            mbar_arrive_expect_tx(bar, 2u * NCH * blk_bytes);
+            const int key0 = (first_kb + n) * p.TM;  // may be negative: zero fill
 #pragma unroll
-          for (int ch = 0; ch < NCH; ++ch) {
-            tma_load_3d(sK + ch * ring_ch + slot * blk_bytes, &tm_k, bar, ch * 64, g, key0);
-            tma_load_3d(sV + ch * ring_ch + slot * blk_bytes, &tm_v, bar, ch * 64, g, key0);
+            for (int ch = 0; ch < NCH; ++ch) {
+              tma_load_3d(sK + ch * ring_ch + slot * blk_bytes, &tm_k, bar, ch * 64, g, key0);
+              tma_load_3d(sV + ch * ring_ch + slot * blk_bytes, &tm_v, bar, ch * 64, g, key0);
+            }
           }
         }
+      }
+      publish(0, 0);  // end of the schedule
+      // this CTA draws no more ranges; the last CTA to get here clears the
+      // call's scheduler slot for the next call that uses it
+      __threadfence();
+      if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+        __threadfence();
+        atomicExch(p.sched, 0u);
+        atomicExch(p.sched + 1, 0u);
       }
     }
   } else if (warp == 13) {
     // ======================= S = Q K^T issuer ================================
     // Descriptors are computed by the whole warp; one elected lane issues.
     const uint64_t kmaj = smem_desc_sw128(0, 16, 1024);  // layout bits, no address
-    int nload = 0;
-    for (int j = 0; j < ntile && !*abort; ++j) {
+    int nload = 0, j = 0;
+    bool stop = false;
+    for (int q = 0; !stop; ++q) {
+     int f0 = 0, f1 = 0;
+     if (!next_range(q, f0, f1)) break;
+     for (int f = f0; f < f1; ++f, ++j) {
+      int g, tb;
+      tile_of(f, g, tb);
       const int b = j & 1, st = j % p.NQ;
       const int first_new = nload;
-      nload += new_blocks(j);
+      nload += new_blocks(f == f0, tb);
       const int win_first = nload - p.NWIN;
       if (lane == 0) RING_TRACE(1, j, 0);
-      if (!mbar_wait(smem_u32(&s_empty[b]), ((j >> 1) & 1) ^ 1, abort)) break;
+      if (!mbar_wait(smem_u32(&s_empty[b]), ((j >> 1) & 1) ^ 1, abort)) {
+        stop = true;
+        break;
+      }
       if (lane == 0) RING_TRACE(1, j, 1);
-      if (!mbar_wait(smem_u32(&q_full[st]), (j / p.NQ) & 1, abort)) break;
+      if (!mbar_wait(smem_u32(&q_full[st]), (j / p.NQ) & 1, abort)) {
+        stop = true;
+        break;
+      }
       if (lane == 0) RING_TRACE(1, j, 2);
       bool ok = true;
       for (int s = first_new; s < nload && ok; ++s)
         ok = mbar_wait(smem_u32(&kv_full[s % p.NB]), (s / p.NB) & 1, abort);
-      if (!ok) break;
+      if (!ok) {
+        stop = true;
+        break;
+      }
       if (lane == 0) RING_TRACE(1, j, 3);
       __syncwarp();
       tc_fence_after();
@@ -449,6 +575,7 @@ __global__ void __launch_bounds__(kRingThreads, 1)
         RING_TRACE(1, j, 4);
       }
       __syncwarp();
+     }
     }
   } else if (warp == 14) {
     // ======================= O = P V issuer ==================================
@@ -457,17 +584,31 @@ __global__ void __launch_bounds__(kRingThreads, 1)
     // groups 1024 bytes apart (SBO)
     const uint64_t mnmaj = smem_desc_sw128(0, ring_ch, 1024);
     const uint32_t ring_keys = static_cast<uint32_t>(p.NB * p.TM);
-    int nload = 0;
-    for (int j = 0; j < ntile && !*abort; ++j) {
+    int nload = 0, j = 0;
+    bool stop = false;
+    for (int q = 0; !stop; ++q) {
+     int f0 = 0, f1 = 0;
+     if (!next_range(q, f0, f1)) break;
+     for (int f = f0; f < f1; ++f, ++j) {
+      int g, tb;
+      tile_of(f, g, tb);
       const int b = j & 1;
-      nload += new_blocks(j);
+      nload += new_blocks(f == f0, tb);
       const int win_first = nload - p.NWIN;
-      // first window block of the next tile: blocks before it are released
-      const int win_next = j + 1 < ntile ? nload + new_blocks(j + 1) - p.NWIN : win_first;
+      // first window block of the next tile (blocks before it are released):
+      // one block on within a range and a kv head, else the window restarts
+      const bool next_slides = f + 1 < f1 && tb + 1 < p.n_tok_tiles;
+      const int win_next = next_slides ? win_first + 1 : nload;
       if (lane == 0) RING_TRACE(2, j, 0);
-      if (!mbar_wait(smem_u32(&p_full[b]), (j >> 1) & 1, abort)) break;
+      if (!mbar_wait(smem_u32(&p_full[b]), (j >> 1) & 1, abort)) {
+        stop = true;
+        break;
+      }
       if (lane == 0) RING_TRACE(2, j, 1);
-      if (!mbar_wait(smem_u32(&o_empty), (j & 1) ^ 1, abort)) break;
+      if (!mbar_wait(smem_u32(&o_empty), (j & 1) ^ 1, abort)) {
+        stop = true;
+        break;
+      }
       if (lane == 0) RING_TRACE(2, j, 2);
       __syncwarp();
       tc_fence_after();
@@ -489,11 +630,13 @@ __global__ void __launch_bounds__(kRingThreads, 1)
         RING_TRACE(2, j, 3);
       }
       __syncwarp();
+     }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  RING_CTA(1);
   if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -3,8 +3,8 @@
 // sliding-window / global attention with a per-head sink on sm_100a.
 //
 // The operation and its sources are described in include/swa_sink.h. Every
-// argument error is returned before any launch; the library allocates no
-// device memory.
+// argument error is returned before any launch. The only device memory the
+// library allocates is the per-device tile-scheduler buffer (sched_slot).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -14,6 +14,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/swa_sink.h"
@@ -109,6 +110,56 @@ int sm_count() {
 
 size_t g_attr_ring[2][swa::kRingMaxBN16 + 1][kMaxDevices];
 
+// ---- tile scheduler state -----------------------------------------------------
+// The persistent prefill kernels draw tile ranges from a counter in device
+// memory: a slot of two words (next range, CTAs finished) that must read zero
+// when a launch starts and that the launch's last CTA sets back to zero. Each
+// call takes the next of kSchedSlots slots, so calls running at the same time
+// on different streams count separately (up to kSchedSlots of them).
+constexpr unsigned int kSchedSlots = 64;
+std::mutex g_sched_mu;
+unsigned int* g_sched[kMaxDevices];
+std::atomic<unsigned int> g_sched_seq{0};
+
+// This call's slot. The first call on a device allocates and zeroes the
+// slots (cudaMalloc, cudaMemset, then a device synchronisation).
+int sched_slot(unsigned int** slot) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail("cudaGetDevice", e);
+  {
+    std::lock_guard<std::mutex> lk(g_sched_mu);
+    if (g_sched[dev] == nullptr) {
+      void* ptr = nullptr;
+      const size_t bytes = 2 * kSchedSlots * sizeof(unsigned int);
+      e = cudaMalloc(&ptr, bytes);
+      if (e != cudaSuccess) return cuda_fail("cudaMalloc(scheduler slots)", e);
+      e = cudaMemset(ptr, 0, bytes);
+      if (e == cudaSuccess) e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) {
+        cudaFree(ptr);
+        return cuda_fail("cudaMemset(scheduler slots)", e);
+      }
+      g_sched[dev] = static_cast<unsigned int*>(ptr);
+    }
+  }
+  *slot = g_sched[dev] + 2 * (g_sched_seq.fetch_add(1u) % kSchedSlots);
+  return SWA_OK;
+}
+
+// Static share and dynamic range length of a persistent launch over n_tiles
+// tiles: each CTA first takes static_tiles consecutive tiles (about
+// kStaticShare of an even split), the rest goes out in short ranges to
+// whichever CTA is free, so SMs that run faster take more. (On B200 the same
+// tile stream ran up to 1.3x faster on some SMs than on others.) A ring range
+// of kRingDynSpan tiles refills the K/V window once (NWIN - 1 extra blocks).
+constexpr double kStaticShare = 0.75;
+constexpr int kRingDynSpan = 8;
+void split_schedule(int n_tiles, int grid, int* static_tiles, int* dyn_base) {
+  *static_tiles = static_cast<int>(kStaticShare * n_tiles / grid);
+  *dyn_base = *static_tiles * grid;
+}
+
 template <int D, int BN16>
 int run_ring(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const CUtensorMap& to, const swa::RingParams& p, size_t smem, int grid,
@@ -145,6 +196,8 @@ int launch_prefill_ring(const void* q, const void* k, const void* v, const int32
     else return SWA_ERR_UNSUPPORTED;
   }
   if (NB <= NWIN) return SWA_ERR_UNSUPPORTED;
+  unsigned int* slot = nullptr;
+  if (sched_slot(&slot) != SWA_OK) return SWA_ERR_CUDA;
   swa::RingParams p;
   p.cu_seqlens = cu;
   p.num_seqs = num_seqs;
@@ -177,6 +230,9 @@ int launch_prefill_ring(const void* q, const void* k, const void* v, const int32
   const int nsm = sm_count();
   if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)", 0);
   const int grid = std::min(nsm, p.n_tiles);
+  p.sched = slot;
+  p.dyn_span = kRingDynSpan;
+  split_schedule(p.n_tiles, grid, &p.static_tiles, &p.dyn_base);
   switch (BN / 16) {
 #define SWA_RING_CASE(N)                                                        \
   case N:                                                                       \

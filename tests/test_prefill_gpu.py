@@ -142,3 +142,28 @@ def test_prefill_full_workloads_sampled(wname):
     # every row written (the output was poisoned with NaN)
     assert torch.isfinite(o).all().item()
     assert torch.isfinite(lse).all().item()
+
+
+def test_prefill_repeated_calls_reuse_scheduler_slots():
+    # more calls than scheduler slots, on one stream and on two at once: each
+    # kernel must find its slot zeroed by the previous user of that slot, so
+    # every output equals the first one bit for bit
+    c = wl.prefill_case([700, 300], 16, 2, 128, 128, sigma=0.5, sink="normal", seed=5)
+    d = to_cuda(c)
+    ref_o, ref_l = B.attn_fwd(d["q"], d["k"], d["v"], d["cu_seqlens"], 128, sink=d["sink"])
+    g = wl.prefill_case([2000], 16, 2, 128, 0, sigma=0.5, sink="normal", seed=6)
+    dg = to_cuda(g)
+    ref_go, ref_gl = B.attn_fwd(dg["q"], dg["k"], dg["v"], dg["cu_seqlens"], 0, sink=dg["sink"])
+    torch.cuda.synchronize()
+    outs = []
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    for it in range(70):
+        with torch.cuda.stream(s1 if it % 2 else s2):
+            o, lse = B.attn_fwd(d["q"], d["k"], d["v"], d["cu_seqlens"], 128, sink=d["sink"])
+            go, gl = B.attn_fwd(dg["q"], dg["k"], dg["v"], dg["cu_seqlens"], 0, sink=dg["sink"])
+        outs.append((o, lse, go, gl))
+    torch.cuda.synchronize()
+    assert B.swa_sink_device_error() == 0
+    for o, lse, go, gl in outs:
+        assert torch.equal(o, ref_o) and torch.equal(lse, ref_l)
+        assert torch.equal(go, ref_go) and torch.equal(gl, ref_gl)
