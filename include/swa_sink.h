@@ -100,6 +100,42 @@ SWA_API int swa_sink_attn_fwd(const void *q, const void *k, const void *v,
                       float *lse, void *stream);
 
 /*
+ * swa_sink_attn_fwd without any device allocation.
+ *
+ * The pages have no counterpart: this is an interface variant. The arguments
+ * and the results (bit for bit) are those of swa_sink_attn_fwd; the only
+ * difference is where the tile scheduler of the sliding-window kernel keeps
+ * its two counters: in a static device array of the library (8 slots of two
+ * 32-bit words, 64 bytes in all) instead of the buffer that swa_sink_attn_fwd
+ * allocates with cudaMalloc on its first call on a device. For callers that
+ * must not allocate: work inside a CUDA stream capture (a first
+ * swa_sink_attn_fwd call there would call cudaMalloc), or a serving runtime
+ * that hands all device memory to its own pool at start-up.
+ *
+ *   slot   the static scheduler slot, 0 <= slot < 8. Any other value returns
+ *          SWA_ERR_SHAPE before anything is launched (the array holds 8).
+ *
+ * - Must start at zero: both words of the slot. They are zero when the
+ *   library's device code is loaded, and every launch leaves its slot zero
+ *   (the launch's last CTA clears it, also after a wait has timed out).
+ * - Calls whose kernels overlap in time (other streams, concurrently running
+ *   graphs) race on a shared slot and give wrong results: give each of them
+ *   its own slot.
+ * - The first call on each device also looks up the array's device address
+ *   (cudaGetSymbolAddress), raises the kernels' shared-memory limits and
+ *   fetches the driver's tensor-map entry point; make that first call before
+ *   any stream capture.
+ * - Only the sliding-window ring kernel has a scheduler; for shapes it does
+ *   not take, the call runs the same kernel as swa_sink_attn_fwd and `slot`
+ *   is not used.
+ */
+SWA_API int swa_sink_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                              const int32_t *cu_seqlens, int num_seqs, int max_seqlen,
+                              int total_tokens, int Hq, int Hkv, int D, int window,
+                              const float *sink, float softmax_scale, void *o,
+                              float *lse, int slot, void *stream);
+
+/*
  * Decode / draft verification over a W-slot KV ring per sequence.
  *
  * Source: section 2.3 "Lightweight MTP" of the report summary above (draft

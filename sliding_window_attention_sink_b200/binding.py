@@ -43,6 +43,9 @@ def load():
     lib.swa_sink_attn_fwd.restype = _i
     lib.swa_sink_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
                                       _f, _vp, _vp, _vp]
+    lib.swa_sink_attn_fwd_noalloc.restype = _i
+    lib.swa_sink_attn_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                              _vp, _f, _vp, _vp, _i, _vp]
     lib.swa_sink_attn_decode.restype = _i
     lib.swa_sink_attn_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                          _i, _vp, _f, _vp, _vp, _vp]
@@ -86,6 +89,14 @@ def swa_sink_attn_fwd(q, k, v, cu_seqlens, num_seqs, max_seqlen, total_tokens, H
         _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), int(num_seqs), int(max_seqlen),
         int(total_tokens), int(Hq), int(Hkv), int(D), int(window), _ptr(sink),
         float(softmax_scale), _ptr(o), _ptr(lse), _stream(stream))
+
+
+def swa_sink_attn_fwd_noalloc(q, k, v, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq, Hkv,
+                              D, window, sink, softmax_scale, o, lse, slot, stream=None):
+    return load().swa_sink_attn_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), int(num_seqs), int(max_seqlen),
+        int(total_tokens), int(Hq), int(Hkv), int(D), int(window), _ptr(sink),
+        float(softmax_scale), _ptr(o), _ptr(lse), int(slot), _stream(stream))
 
 
 def swa_sink_attn_decode(q, k_new, v_new, k_ring, v_ring, pos, B, n_q, Hq, Hkv, D, W, sink,

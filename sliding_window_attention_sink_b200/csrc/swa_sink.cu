@@ -147,6 +147,34 @@ int sched_slot(unsigned int** slot) {
   return SWA_OK;
 }
 
+// ---- scheduler slots that need no allocation ------------------------------------
+// swa_sink_attn_fwd_noalloc takes its tile-scheduler slot from this static
+// array instead of the per-device buffer that swa_sink_attn_fwd allocates on
+// its first call. Each slot is two words that must read zero when a launch
+// starts: they are zero when the module loads, and every launch leaves its
+// slot zero again (its last CTA clears it). 8 slots = 64 bytes.
+constexpr int kNoAllocSlots = 8;
+static __device__ __align__(256) unsigned int g_noalloc_sched[2 * kNoAllocSlots];
+std::mutex g_noalloc_mu;
+unsigned int* g_noalloc_base[kMaxDevices];
+
+// The device address of the slot, looked up once per device (with that device
+// current) by cudaGetSymbolAddress.
+int noalloc_slot(int slot, unsigned int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail("cudaGetDevice", e);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_base[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_sched);
+    if (e != cudaSuccess || ptr == nullptr) return cuda_fail("cudaGetSymbolAddress", e);
+    g_noalloc_base[dev] = static_cast<unsigned int*>(ptr);
+  }
+  *out = g_noalloc_base[dev] + 2 * slot;
+  return SWA_OK;
+}
+
 // Static share and dynamic range length of a persistent launch over n_tiles
 // tiles: each CTA first takes static_tiles consecutive tiles (about
 // kStaticShare of an even split), the rest goes out in short ranges to
@@ -176,11 +204,13 @@ constexpr size_t kRingSmemLimit = 232448 - 5120;
 
 // Sliding-window prefill on the persistent ring pipeline when the window's
 // keys for one tile fit one MMA (BN <= 256) and the S/P double buffer plus O
-// fit TMEM. Returns SWA_ERR_UNSUPPORTED (nothing launched) otherwise.
+// fit TMEM. Returns SWA_ERR_UNSUPPORTED (nothing launched) otherwise. The tile
+// scheduler uses static slot `noalloc` when it is >= 0, else the next slot of
+// the library's per-device buffer.
 template <int D>
 int launch_prefill_ring(const void* q, const void* k, const void* v, const int32_t* cu,
                         int num_seqs, int total, int Hq, int Hkv, int window, const float* sink,
-                        float scale, void* o, float* lse, cudaStream_t st) {
+                        float scale, void* o, float* lse, cudaStream_t st, int noalloc) {
   const int G = Hq / Hkv;
   if (window <= 0 || !(G == 2 || G == 4 || G == 8)) return SWA_ERR_UNSUPPORTED;
   const int TM = 128 / G;
@@ -197,7 +227,8 @@ int launch_prefill_ring(const void* q, const void* k, const void* v, const int32
   }
   if (NB <= NWIN) return SWA_ERR_UNSUPPORTED;
   unsigned int* slot = nullptr;
-  if (sched_slot(&slot) != SWA_OK) return SWA_ERR_CUDA;
+  if ((noalloc >= 0 ? noalloc_slot(noalloc, &slot) : sched_slot(&slot)) != SWA_OK)
+    return SWA_ERR_CUDA;
   swa::RingParams p;
   p.cu_seqlens = cu;
   p.num_seqs = num_seqs;
@@ -352,6 +383,54 @@ int launch_decode(const swa::DecodeParams& p, cudaStream_t st) {
   return e == cudaSuccess ? SWA_OK : cuda_fail("decode launch", e);
 }
 
+// swa_sink_attn_fwd and swa_sink_attn_fwd_noalloc: validation and kernel
+// choice. noalloc: the static scheduler slot of the ring kernel, or -1 for
+// the library's own buffer.
+int fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+             int num_seqs, int max_seqlen, int total_tokens, int Hq, int Hkv, int D, int window,
+             const float* sink, float softmax_scale, void* o, float* lse, void* stream,
+             int noalloc) {
+  if (num_seqs < 0 || max_seqlen < 0 || total_tokens < 0 || Hq <= 0 || Hkv <= 0)
+    return SWA_ERR_SHAPE;
+  if (Hq % Hkv != 0) return SWA_ERR_SHAPE;
+  if (total_tokens > 0 && num_seqs == 0) return SWA_ERR_SHAPE;
+  if (max_seqlen > total_tokens) return SWA_ERR_SHAPE;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 128) return SWA_ERR_UNSUPPORTED;
+  if (total_tokens == 0) return SWA_OK;
+  if (!q || !k || !v || !o || !cu_seqlens) return SWA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SWA_ERR_ALIGN;
+  if (!aligned4(cu_seqlens) || (sink && !aligned4(sink)) || (lse && !aligned4(lse)))
+    return SWA_ERR_ALIGN;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // sliding windows: the persistent ring pipeline when the shape allows it
+  if (window > 0) {
+    const int rc = D == 64 ? launch_prefill_ring<64>(q, k, v, cu_seqlens, num_seqs,
+                                                     total_tokens, Hq, Hkv, window, sink,
+                                                     softmax_scale, o, lse, st, noalloc)
+                           : launch_prefill_ring<128>(q, k, v, cu_seqlens, num_seqs,
+                                                      total_tokens, Hq, Hkv, window, sink,
+                                                      softmax_scale, o, lse, st, noalloc);
+    if (rc != SWA_ERR_UNSUPPORTED) return rc;
+  }
+  {
+    const int rc = D == 64 ? launch_prefill_chunked<64>(q, k, v, cu_seqlens, num_seqs,
+                                                        total_tokens, Hq, Hkv, window, sink,
+                                                        softmax_scale, o, lse, st)
+                           : launch_prefill_chunked<128>(q, k, v, cu_seqlens, num_seqs,
+                                                         total_tokens, Hq, Hkv, window, sink,
+                                                         softmax_scale, o, lse, st);
+    if (rc != SWA_ERR_UNSUPPORTED) return rc;
+  }
+  if (D == 64)
+    return launch_prefill<64>(q, k, v, cu_seqlens, num_seqs, total_tokens, Hq, Hkv, window, sink,
+                              softmax_scale, o, lse, st);
+  return launch_prefill<128>(q, k, v, cu_seqlens, num_seqs, total_tokens, Hq, Hkv, window, sink,
+                             softmax_scale, o, lse, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -374,45 +453,18 @@ int swa_sink_attn_fwd(const void* q, const void* k, const void* v, const int32_t
                       int num_seqs, int max_seqlen, int total_tokens, int Hq, int Hkv, int D,
                       int window, const float* sink, float softmax_scale, void* o, float* lse,
                       void* stream) {
-  if (num_seqs < 0 || max_seqlen < 0 || total_tokens < 0 || Hq <= 0 || Hkv <= 0)
-    return SWA_ERR_SHAPE;
-  if (Hq % Hkv != 0) return SWA_ERR_SHAPE;
-  if (total_tokens > 0 && num_seqs == 0) return SWA_ERR_SHAPE;
-  if (max_seqlen > total_tokens) return SWA_ERR_SHAPE;
-  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
-  if (Hq / Hkv > 128) return SWA_ERR_UNSUPPORTED;
-  if (total_tokens == 0) return SWA_OK;
-  if (!q || !k || !v || !o || !cu_seqlens) return SWA_ERR_NULL;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SWA_ERR_ALIGN;
-  if (!aligned4(cu_seqlens) || (sink && !aligned4(sink)) || (lse && !aligned4(lse)))
-    return SWA_ERR_ALIGN;
-  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-    softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // sliding windows: the persistent ring pipeline when the shape allows it
-  if (window > 0) {
-    const int rc = D == 64 ? launch_prefill_ring<64>(q, k, v, cu_seqlens, num_seqs,
-                                                     total_tokens, Hq, Hkv, window, sink,
-                                                     softmax_scale, o, lse, st)
-                           : launch_prefill_ring<128>(q, k, v, cu_seqlens, num_seqs,
-                                                      total_tokens, Hq, Hkv, window, sink,
-                                                      softmax_scale, o, lse, st);
-    if (rc != SWA_ERR_UNSUPPORTED) return rc;
-  }
-  {
-    const int rc = D == 64 ? launch_prefill_chunked<64>(q, k, v, cu_seqlens, num_seqs,
-                                                        total_tokens, Hq, Hkv, window, sink,
-                                                        softmax_scale, o, lse, st)
-                           : launch_prefill_chunked<128>(q, k, v, cu_seqlens, num_seqs,
-                                                         total_tokens, Hq, Hkv, window, sink,
-                                                         softmax_scale, o, lse, st);
-    if (rc != SWA_ERR_UNSUPPORTED) return rc;
-  }
-  if (D == 64)
-    return launch_prefill<64>(q, k, v, cu_seqlens, num_seqs, total_tokens, Hq, Hkv, window, sink,
-                              softmax_scale, o, lse, st);
-  return launch_prefill<128>(q, k, v, cu_seqlens, num_seqs, total_tokens, Hq, Hkv, window, sink,
-                             softmax_scale, o, lse, st);
+  return fwd_impl(q, k, v, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq, Hkv, D, window,
+                  sink, softmax_scale, o, lse, stream, -1);
+}
+
+int swa_sink_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                              const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+                              int total_tokens, int Hq, int Hkv, int D, int window,
+                              const float* sink, float softmax_scale, void* o, float* lse,
+                              int slot, void* stream) {
+  if (slot < 0 || slot >= kNoAllocSlots) return SWA_ERR_SHAPE;
+  return fwd_impl(q, k, v, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq, Hkv, D, window,
+                  sink, softmax_scale, o, lse, stream, slot);
 }
 
 int swa_sink_attn_decode(const void* q, const void* k_new, const void* v_new, const void* k_ring,

@@ -102,3 +102,18 @@ def test_header_is_plain_c():
                             "-I", os.path.join(ROOT, "include"), src],
                            capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
+
+
+def test_fwd_noalloc_argument_errors():
+    # the slot is checked first, then the arguments exactly as for
+    # swa_sink_attn_fwd; none of these calls reaches CUDA
+    a = dict(q=FAKE, k=FAKE, v=FAKE, cu_seqlens=FAKE, num_seqs=1, max_seqlen=8,
+             total_tokens=8, Hq=8, Hkv=2, D=128, window=128, sink=None,
+             softmax_scale=0.0, o=FAKE, lse=None, stream=0)
+    assert B.swa_sink_attn_fwd_noalloc(slot=8, **a) == -2
+    assert B.swa_sink_attn_fwd_noalloc(slot=-1, **a) == -2
+    assert B.swa_sink_attn_fwd_noalloc(slot=0, **dict(a, Hq=8, Hkv=3)) == -2
+    assert B.swa_sink_attn_fwd_noalloc(slot=7, **dict(a, D=96)) == -3
+    assert B.swa_sink_attn_fwd_noalloc(slot=0, **dict(a, q=None)) == -1
+    assert B.swa_sink_attn_fwd_noalloc(slot=0, **dict(a, o=FAKE + 2)) == -4
+    assert B.swa_sink_attn_fwd_noalloc(slot=3, **dict(a, total_tokens=0, max_seqlen=0)) == 0
