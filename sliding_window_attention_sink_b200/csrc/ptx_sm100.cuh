@@ -309,14 +309,6 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// The value x, hidden from the compiler's common-subexpression elimination
-// (so that values derived from it are computed again where they are used).
-__device__ __forceinline__ int opaque(int x) {
-  int y;
-  asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
 // Named barrier `id` (1..15) over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -370,32 +362,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return r;
 }
 
-// Base-2 exponential of a pair on the FMA pipe, for x in [-126.5, 128):
-// Cody and Waite's range reduction x = j + f with j = round(x) (by adding and
-// subtracting 1.5 * 2^23) and f in [-0.5, 0.5]; 2^f by a degree-3 polynomial
-// whose coefficients were fitted for this file by the Remez exchange
-// algorithm on [-0.5, 0.5] for least maximum relative error (7.5e-5); 2^j by
-// adding j to the exponent field, which the low bits of the rounded sum hold
-// after a left shift by 23. Inputs below -126.5 (masked keys: -inf) are
-// clamped there and give a tiny positive value (< 2^-126). Used for a share
-// of the softmax exponentials so that the MUFU pipe is not the only one busy.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  float a, b;
-  f2_unpack(x2, a, b);
-  const uint64_t xc = f2_pack(fmaxf(a, -126.5f), fmaxf(b, -126.5f));
-  const uint64_t r = f2_add(xc, f2_pack(12582912.f, 12582912.f));  // 1.5 * 2^23 + j
-  const uint64_t j = f2_add(r, f2_pack(-12582912.f, -12582912.f));
-  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), xc);
-  uint64_t p = f2_fma(f2_pack(0x1.c3f76p-5f, 0x1.c3f76p-5f), f,
-                      f2_pack(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
-  p = f2_fma(p, f, f2_pack(0x1.62f31ap-1f, 0x1.62f31ap-1f));
-  p = f2_fma(p, f, f2_pack(0x1.fff692p-1f, 0x1.fff692p-1f));
-  float p0, p1, r0, r1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(r, r0, r1);
-  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(r0) << 23)),
-                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(r1) << 23)));
-}
 // Three-input maximum.
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
