@@ -397,8 +397,9 @@ __global__ void __launch_bounds__(kRingThreads, 1)
       // staging chunk (128-byte swizzle: 16-byte unit u of row r at u ^ (r&7))
       // -> TMA store as its own bulk group. The staging chunk is reused once
       // its previous store has read it. TMEM O is released after the last
-      // chunk's load.
-#pragma unroll
+      // chunk's load. The chunk loop stays rolled (smaller code: the roles
+      // share each SM sub-partition's instruction cache).
+#pragma unroll 1
       for (int ch = 0; ch < NCH; ++ch) {
         uint32_t v[64];
 #pragma unroll
