@@ -9,21 +9,26 @@
 // the committed tokens at positions >= P + t - W + 1 (slot p mod W of the
 // ring) and the new tokens 0..t.
 //
-// Design (sm_100a): one CTA of 4 warps per (sequence, kv head); split-free.
+// Design (sm_100a): one CTA of 8 warps per (sequence, kv head); split-free.
 // * All G query heads of the kv head and all n_q tokens are one set of
 //   R = n_q * G query rows (32 for n_q = 4, G = 8), so each ring byte is read
 //   from HBM exactly once for all of them.
-// * The ring slice (W rows of D bf16, 2 KB apart in HBM) and the new rows go
-//   to shared memory with 16-byte cp.async; keys first, values in a second
-//   group that lands while the scores are computed.
+// * One thread issues all loads as TMA boxes into shared memory (128-byte
+//   swizzle, 64 head-dim columns per box): the ring slice (W rows of D bf16,
+//   Hkv * D apart in HBM) and the n_q new rows of K, then of V, plus the Q
+//   rows; K and Q complete on one mbarrier, V on a second one that lands
+//   while the scores are computed. (16-byte cp.async from every thread took
+//   about a third of a CTA's cycles just to issue.) The new rows go to row
+//   roundup8(W) so that every box starts on a 1024-byte swizzle atom.
 // * The contraction has ~25 flop per HBM byte, above what CUDA-core FMAs hide,
 //   so S = Q K^T and O = P V use the tensor cores through mma.sync m16n8k16
 //   (bf16, f32 accumulate); the tiles (32 rows) are too small for tcgen05.
-// * Softmax: the 4 warps split the keys for S; row maxima and sums are
+//   ldmatrix addresses follow the swizzle.
+// * Softmax: the 8 warps split the keys for S; row maxima and sums are
 //   reduced inside the quad that shares a row (warp shuffles), then across
 //   warps through shared memory. The max is seeded with the sink logit and
 //   the denominator gets the sink term exp(s - m). P goes to shared memory as
-//   bf16; the 4 warps then split the head dim for O = P V.
+//   bf16; the 8 warps then split the head dim for O = P V.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -37,23 +42,14 @@ struct DecodeParams {
   const int32_t* pos;
   int B, n_q, Hq, Hkv, G, W;
   int R;    // query rows per CTA = n_q * G (<= 32)
-  int KP;   // keys padded to a multiple of 16: roundup16(W + n_q)
+  int W8;   // first row of the new keys: roundup8(W)
+  int KP;   // key rows padded to a multiple of 16: roundup16(W8 + n_q)
   const float* sink;
   float scale_log2;
   __nv_bfloat16* o;
   float* lse;
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 __device__ __forceinline__ void st_shared_zero16(uint32_t dst) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
 }
@@ -92,36 +88,62 @@ __device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
-constexpr int kDecodeWarps = 8;
+// Warps per CTA: 4 when the keys fit 5 n8 tiles per warp (KP <= 160), with
+// one shared-memory buffer that holds K and then V, so that four CTAs share
+// an SM and overlap their loads; else 8 warps with separate K and V buffers.
+constexpr int kDecodeSmallWarps = 4;
+constexpr int kDecodeLargeWarps = 8;
+constexpr int kDecodeSmallMaxKP = 160;
 
-// Shared memory: K and V [KP][D+8], Q [32][D+8], P [32][KP+8] (bf16), then
-// per-warp row maxima and the two row sums [8][32] and per-row l [32] (fp32).
-__host__ __device__ constexpr int decode_row_stride(int D) { return D + 8; }
-__host__ __device__ inline size_t decode_smem_bytes(int D, int KP) {
-  const int ld = decode_row_stride(D);
-  return static_cast<size_t>(2 * KP * ld + 32 * ld + 32 * (KP + 8)) * 2 +
-         (kDecodeWarps * 32 * 3 + 32) * sizeof(float);
+// Shared memory (from a 1024-byte aligned base): K and V (or one buffer for
+// both) as D/64 blocks of [KP rows][128 bytes]; Q as D/64 blocks of [32 rows]
+// [128 bytes] (128-byte swizzle: 16-byte unit u of row r at u ^ (r & 7)),
+// later overwritten by P [32][KP+8] bf16; then per-warp row maxima and the two
+// row sums [NWP][32] and per-row l [32] (fp32).
+__host__ __device__ inline size_t decode_qp_bytes(int D, int KP) {
+  const size_t q = static_cast<size_t>(D / 64) * 32 * 128;
+  const size_t pb = static_cast<size_t>(32) * (KP + 8) * 2;
+  return q > pb ? q : pb;
+}
+__host__ __device__ inline size_t decode_smem_bytes(int D, int KP, int nwp) {
+  const size_t kv = static_cast<size_t>(D / 64) * KP * 128 * (nwp == kDecodeSmallWarps ? 1 : 2);
+  return 1024 + kv + decode_qp_bytes(D, KP) + (static_cast<size_t>(nwp) * 32 * 3 + 32) * sizeof(float);
 }
 
-template <int D, int MT>
-__global__ void __launch_bounds__(kDecodeWarps * 32, 2)
-    decode_sm100_kernel(const DecodeParams p) {
-  constexpr int NWP = kDecodeWarps;
+// Byte address of (row, col) in a tile stored as 64-column blocks of `rows`
+// 128-byte rows with the 128-byte swizzle; col a multiple of 8.
+__device__ __forceinline__ uint32_t sw128_addr(uint32_t base, int rows, int row, int col) {
+  return base + static_cast<uint32_t>((col >> 6) * rows * 128 + row * 128 +
+                                      ((((col & 63) >> 3) ^ (row & 7)) << 4));
+}
+
+template <int D, int MT, int NWP>
+__global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
+    decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_kr,
+                        const __grid_constant__ CUtensorMap tm_kn,
+                        const __grid_constant__ CUtensorMap tm_vr,
+                        const __grid_constant__ CUtensorMap tm_vn, const DecodeParams p) {
+  constexpr bool SHARE = NWP == kDecodeSmallWarps;  // one buffer for K, then V
   constexpr int NT_ = NWP * 32;
-  constexpr int LD = D + 8;        // bf16 elements per smem row (conflict-free ldmatrix)
-  constexpr int CPR = D / 8;       // 16-byte chunks per row
+  constexpr int NCH = D / 64;      // 64-column blocks of the head dim
   constexpr int RP = MT * 16;      // padded query rows
-  constexpr int NTW = 5;           // max n8 key tiles per warp (KP <= 272)
-  constexpr int DW = D / NWP;      // PV: head-dim columns per warp (16 or 8)
-  constexpr int NTO = DW / 8;      // n8 tiles per warp in PV (2 or 1)
+  constexpr int NTW = 5;           // max n8 key tiles per warp (KP <= 40 * NWP)
+  constexpr int DW = D / NWP;      // PV: head-dim columns per warp
+  constexpr int NTO = DW / 8;      // n8 tiles per warp in PV (1, 2 or 4)
   extern __shared__ __align__(16) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_qk, bar_v;
+  __shared__ int abort_sh;
+  volatile int* abort = &abort_sh;
   const int KP = p.KP;
-  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smem_raw);
-  __nv_bfloat16* Vs = Ks + KP * LD;
-  __nv_bfloat16* Qs = Vs + KP * LD;
-  __nv_bfloat16* Ps = Qs + 32 * LD;
+  const uint32_t sK = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sV = SHARE ? sK : sK + NCH * KP * 128;
+  const uint32_t sQ = sV + NCH * KP * 128;
+  // P takes Q's place once S is done
+  __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(smem_raw + (sQ - smem_u32(smem_raw)));
   const int LDP = KP + 8;
-  float* red_max = reinterpret_cast<float*>(Ps + 32 * LDP);  // [NWP][32]
+  float* red_max = reinterpret_cast<float*>(smem_raw + (sQ - smem_u32(smem_raw)) +
+                                              decode_qp_bytes(D, KP));  // [NWP][32]
   float* red_lr = red_max + NWP * 32;                         // [NWP][32]
   float* red_lx = red_lr + NWP * 32;                          // [NWP][32]
   float* row_l = red_lx + NWP * 32;                           // [32]
@@ -136,39 +158,51 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
   }
   const int W = p.W, n_q = p.n_q, G = p.G;
 
-  // ---- loads: group 0 = Q and K rows, group 1 = V rows ---------------------
-  const uint32_t sQ = smem_u32(Qs), sK = smem_u32(Ks), sV = smem_u32(Vs);
-  for (int idx = tid; idx < RP * CPR; idx += NT_) {
-    const int r = idx / CPR, c = idx - r * CPR;
-    const uint32_t dst = sQ + (r * LD + c * 8) * 2;
-    if (r < p.R) {
-      const int t = r / G, hh = r - t * G;
-      cp_async16(dst, p.q + ((static_cast<size_t>(b) * n_q + t) * p.Hq + g * G + hh) * D + c * 8);
-    } else {
-      st_shared_zero16(dst);
+  // ---- loads: Q and K on bar_qk, V on bar_v (one thread issues) ------------
+  const int W8 = p.W8;
+  if (tid == 0) {
+    mbar_init(smem_u32(&bar_qk), 1);
+    mbar_init(smem_u32(&bar_v), 1);
+    abort_sh = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kr);
+    tma_prefetch_desc(&tm_kn);
+    tma_prefetch_desc(&tm_vr);
+    tma_prefetch_desc(&tm_vn);
+    const uint32_t kv_bytes = NCH * (W + n_q) * 128;
+    mbar_arrive_expect_tx(smem_u32(&bar_qk), NCH * p.R * 128 + kv_bytes);
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+      tma_load_4d(sQ + ch * 32 * 128, &tm_q, smem_u32(&bar_qk), ch * 64, g * G, 0, b);
+      tma_load_4d(sK + ch * KP * 128, &tm_kr, smem_u32(&bar_qk), ch * 64, g, 0, b);
+      tma_load_4d(sK + ch * KP * 128 + W8 * 128, &tm_kn, smem_u32(&bar_qk), ch * 64, g, 0, b);
+    }
+    if (!SHARE) {
+      mbar_arrive_expect_tx(smem_u32(&bar_v), kv_bytes);
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch) {
+        tma_load_4d(sV + ch * KP * 128, &tm_vr, smem_u32(&bar_v), ch * 64, g, 0, b);
+        tma_load_4d(sV + ch * KP * 128 + W8 * 128, &tm_vn, smem_u32(&bar_v), ch * 64, g, 0, b);
+      }
     }
   }
-  const __nv_bfloat16* kr = p.k_ring + (static_cast<size_t>(b) * W * p.Hkv + g) * D;
-  const __nv_bfloat16* kn = p.k_new + (static_cast<size_t>(b) * n_q * p.Hkv + g) * D;
-  const __nv_bfloat16* vr = p.v_ring + (static_cast<size_t>(b) * W * p.Hkv + g) * D;
-  const __nv_bfloat16* vn = p.v_new + (static_cast<size_t>(b) * n_q * p.Hkv + g) * D;
-  const size_t kstride = static_cast<size_t>(p.Hkv) * D;  // elements between consecutive keys
-  for (int idx = tid; idx < KP * CPR; idx += NT_) {
-    const int key = idx / CPR, c = idx - key * CPR;
-    const uint32_t dst = sK + (key * LD + c * 8) * 2;
-    if (key < W) cp_async16(dst, kr + key * kstride + c * 8);
-    else if (key < W + n_q) cp_async16(dst, kn + (key - W) * kstride + c * 8);
-    else st_shared_zero16(dst);
+  // V rows no box writes (between the ring and the new rows, and after the
+  // new rows) are zeroed: P is 0 there, and 0 * V must stay 0 (with one
+  // buffer, K's boxes leave the same rows alone)
+  {
+    const int pad1 = W8 - W, pad2 = KP - (W8 + n_q);
+    for (int idx = tid; idx < NCH * (pad1 + pad2) * 8; idx += NT_) {
+      const int ch = idx / ((pad1 + pad2) * 8);
+      const int rem = idx - ch * (pad1 + pad2) * 8;
+      const int pr = rem >> 3;
+      const int row = pr < pad1 ? W + pr : W8 + n_q + (pr - pad1);
+      st_shared_zero16(sV + ch * KP * 128 + row * 128 + (rem & 7) * 16);
+    }
   }
-  cp_async_commit();
-  for (int idx = tid; idx < KP * CPR; idx += NT_) {
-    const int key = idx / CPR, c = idx - key * CPR;
-    const uint32_t dst = sV + (key * LD + c * 8) * 2;
-    if (key < W) cp_async16(dst, vr + key * kstride + c * 8);
-    else if (key < W + n_q) cp_async16(dst, vn + (key - W) * kstride + c * 8);
-    else st_shared_zero16(dst);
-  }
-  cp_async_commit();
 
   // ---- this thread's rows (fragment rows lane/4 and lane/4 + 8 per m-tile) --
   // ring slot s holds the token at position P - W + rel(s), rel(s) = (s - P) mod W;
@@ -185,8 +219,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
       thr[mt][hf] = t >= 0 ? max(t + 1, W - P) : 0x7fffffff;
     }
 
-  cp_async_wait<1>();
-  __syncthreads();
+  // Q and K in shared memory (the zeroing above is published by the same
+  // barrier); a wait that gave up ends every thread of the CTA here
+  if (!__syncthreads_and(mbar_wait(smem_u32(&bar_qk), 0, abort))) return;
 
   // ---- S = Q K^T: warp w takes key tiles w, w+8, w+16, ... ----------------
   const int NT = KP / 8;
@@ -204,7 +239,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
     for (int mt = 0; mt < MT; ++mt) {
       const int row = mt * 16 + (lane & 15);
       const int col = kk * 16 + (lane >> 4) * 8;
-      ldsm_x4(sQ + (row * LD + col) * 2, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
+      ldsm_x4(sw128_addr(sQ, 32, row, col), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
     }
 #pragma unroll
     for (int j = 0; j < NTW; ++j) {
@@ -213,10 +248,24 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
         uint32_t b0, b1;
         const int key = nt * 8 + (lane & 7);
         const int col = kk * 16 + ((lane >> 3) & 1) * 8;
-        ldsm_x2(sK + (key * LD + col) * 2, b0, b1);
+        ldsm_x2(sw128_addr(sK, KP, key, col), b0, b1);
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
           mma_16816(s[mt][j], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
+      }
+    }
+  }
+
+  if (SHARE) {
+    // K has been read: V goes into its buffer while the softmax runs
+    __syncthreads();
+    if (tid == 0) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(smem_u32(&bar_v), NCH * (W + n_q) * 128);
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch) {
+        tma_load_4d(sV + ch * KP * 128, &tm_vr, smem_u32(&bar_v), ch * 64, g, 0, b);
+        tma_load_4d(sV + ch * KP * 128 + W8 * 128, &tm_vn, smem_u32(&bar_v), ch * 64, g, 0, b);
       }
     }
   }
@@ -235,8 +284,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
       int rel = col - Pmod;
       if (rel < 0) rel += W;
       const bool ring = nt < NT && col < W;
-      const bool isnew = nt < NT && col >= W && col < W + n_q;
-      const int u = col - W;
+      const bool isnew = nt < NT && col >= W8 && col < W8 + n_q;
+      const int u = col - W8;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -313,8 +362,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
         red_lx[warp * 32 + mt * 16 + (lane >> 2) + hf * 8] = x;
       }
     }
-  cp_async_wait<0>();
-  __syncthreads();
+  // V in shared memory; a wait that gave up ends every thread here
+  if (!__syncthreads_and(mbar_wait(smem_u32(&bar_v), 0, abort))) return;
   // row sums over warps plus the sink term; LSE (one thread per row)
   if (tid < RP) {
     const int row = tid;
@@ -358,18 +407,21 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
       ldsm_x4(sP + (row * LDP + col) * 2, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
     }
     const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-    if (NTO == 2) {
-      uint32_t b0, b1, b2, b3;
-      const int col = warp * DW + (lane >> 4) * 8;
-      ldsm_x4_t(sV + (key * LD + col) * 2, b0, b1, b2, b3);
+    if (NTO >= 2) {
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        mma_16816(acc[mt][0], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
-        mma_16816(acc[mt][NTO - 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b2, b3);
+      for (int jp = 0; jp < NTO / 2; ++jp) {
+        uint32_t b0, b1, b2, b3;
+        const int col = warp * DW + jp * 16 + (lane >> 4) * 8;
+        ldsm_x4_t(sw128_addr(sV, KP, key, col), b0, b1, b2, b3);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          mma_16816(acc[mt][2 * jp], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
+          mma_16816(acc[mt][2 * jp + 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b2, b3);
+        }
       }
     } else {
       uint32_t b0, b1;
-      ldsm_x2_t(sV + (key * LD + warp * DW) * 2, b0, b1);
+      ldsm_x2_t(sw128_addr(sV, KP, key, warp * DW), b0, b1);
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
         mma_16816(acc[mt][0], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);

@@ -63,6 +63,22 @@ int encode_3d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t mid,
   return r == CUDA_SUCCESS ? SWA_OK : cuda_fail("cuTensorMapEncodeTiled", static_cast<int>(r));
 }
 
+// 4-D bf16 tensor [d3][d2][d1][d0] (d0 contiguous), 128-byte swizzle.
+int encode_4d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+              uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  auto fn = get_encode_fn();
+  if (!fn) return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", 0);
+  cuuint64_t dims[4] = {d0, d1, d2, d3};
+  cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  cuuint32_t box[4] = {b0, b1, b2, b3};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SWA_OK : cuda_fail("cuTensorMapEncodeTiled", static_cast<int>(r));
+}
+
 // With SWA_SINK_DEBUG set in the environment, failing CUDA calls are named
 // on stderr (the status code alone says only SWA_ERR_CUDA).
 int cuda_fail(const char* what, int err) {
@@ -91,7 +107,7 @@ int ensure_smem_attr(K kernel, size_t bytes, size_t (&done)[kMaxDevices]) {
 }
 
 size_t g_attr_prefill64[kMaxDevices], g_attr_prefill128[kMaxDevices];
-size_t g_attr_dec[2][2][kMaxDevices];
+size_t g_attr_dec[2][2][2][kMaxDevices];
 
 int next_pow2(int x) {
   int p = 32;
@@ -373,12 +389,25 @@ int launch_prefill(const void* q, const void* k, const void* v, const int32_t* c
   return e == cudaSuccess ? SWA_OK : cuda_fail("prefill launch", e);
 }
 
-template <int D, int MT>
+template <int D, int MT, int NWP>
 int launch_decode(const swa::DecodeParams& p, cudaStream_t st) {
-  const size_t smem = swa::decode_smem_bytes(D, p.KP);
-  auto kern = swa::decode_sm100_kernel<D, MT>;
-  if (ensure_smem_attr(kern, smem, g_attr_dec[D == 128][MT - 1]) != SWA_OK) return SWA_ERR_CUDA;
-  kern<<<static_cast<unsigned>(p.B) * p.Hkv, swa::kDecodeWarps * 32, smem, st>>>(p);
+  // boxes of 64 head-dim columns: Q [G heads x n_q tokens], ring [W rows],
+  // new rows [n_q rows], of one (sequence, kv head)
+  CUtensorMap tq, tkr, tkn, tvr, tvn;
+  const uint32_t G = static_cast<uint32_t>(p.G), nq = static_cast<uint32_t>(p.n_q);
+  const uint32_t W = static_cast<uint32_t>(p.W);
+  if (encode_4d(&tq, p.q, D, p.Hq, p.n_q, p.B, 64, G, nq, 1) != SWA_OK ||
+      encode_4d(&tkr, p.k_ring, D, p.Hkv, p.W, p.B, 64, 1, W, 1) != SWA_OK ||
+      encode_4d(&tkn, p.k_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK ||
+      encode_4d(&tvr, p.v_ring, D, p.Hkv, p.W, p.B, 64, 1, W, 1) != SWA_OK ||
+      encode_4d(&tvn, p.v_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK)
+    return SWA_ERR_CUDA;
+  const size_t smem = swa::decode_smem_bytes(D, p.KP, NWP);
+  auto kern = swa::decode_sm100_kernel<D, MT, NWP>;
+  if (ensure_smem_attr(kern, smem,
+                       g_attr_dec[D == 128][MT - 1][NWP == swa::kDecodeLargeWarps]) != SWA_OK)
+    return SWA_ERR_CUDA;
+  kern<<<static_cast<unsigned>(p.B) * p.Hkv, NWP * 32, smem, st>>>(tq, tkr, tkn, tvr, tvn, p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SWA_OK : cuda_fail("decode launch", e);
 }
@@ -497,7 +526,8 @@ int swa_sink_attn_decode(const void* q, const void* k_new, const void* v_new, co
   p.G = Hq / Hkv;
   p.W = W;
   p.R = n_q * p.G;
-  p.KP = round_up(W + n_q, 16);
+  p.W8 = round_up(W, 8);
+  p.KP = round_up(p.W8 + n_q, 16);
   p.sink = sink;
   p.scale_log2 = softmax_scale * swa::kLog2e;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -505,8 +535,14 @@ int swa_sink_attn_decode(const void* q, const void* k_new, const void* v_new, co
   if (static_cast<long long>(B) * Hkv > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool two = p.R > 16;
-  if (D == 64) return two ? launch_decode<64, 2>(p, st) : launch_decode<64, 1>(p, st);
-  return two ? launch_decode<128, 2>(p, st) : launch_decode<128, 1>(p, st);
+  if (p.KP <= swa::kDecodeSmallMaxKP) {
+    constexpr int S = swa::kDecodeSmallWarps;
+    if (D == 64) return two ? launch_decode<64, 2, S>(p, st) : launch_decode<64, 1, S>(p, st);
+    return two ? launch_decode<128, 2, S>(p, st) : launch_decode<128, 1, S>(p, st);
+  }
+  constexpr int L = swa::kDecodeLargeWarps;
+  if (D == 64) return two ? launch_decode<64, 2, L>(p, st) : launch_decode<64, 1, L>(p, st);
+  return two ? launch_decode<128, 2, L>(p, st) : launch_decode<128, 1, L>(p, st);
 }
 
 int swa_sink_kv_commit(void* k_ring, void* v_ring, const void* k_new, const void* v_new,

@@ -42,9 +42,15 @@ CASES = [  # (B, n_q, Hq, Hkv, D, W, sink)
     (8, 4, 32, 8, 128, 128, None),
     (8, 2, 8, 1, 128, 64, "normal"),
     (8, 3, 16, 2, 64, 40, "normal"),
-    # rings too large to double-buffer at D = 128 (single-buffer path)
+    # the largest rings
     (6, 2, 16, 2, 128, 256, "normal"),
     (6, 4, 32, 8, 128, 200, "uniform2"),
+    # rings that are not a multiple of 8 rows (new rows start at roundup8(W)),
+    # a one-slot ring, and 8 new tokens
+    (8, 4, 64, 8, 128, 127, "normal"),
+    (8, 3, 16, 2, 64, 13, "uniform2"),
+    (8, 1, 8, 1, 128, 1, "normal"),
+    (8, 8, 16, 4, 128, 100, "normal"),
     # more units than SMs with few rows per unit
     (400, 1, 8, 8, 64, 128, "normal"),
 ]
