@@ -9,7 +9,9 @@
 // the committed tokens at positions >= P + t - W + 1 (slot p mod W of the
 // ring) and the new tokens 0..t.
 //
-// Design (sm_100a): one CTA of 8 warps per (sequence, kv head); split-free.
+// Design (sm_100a): one CTA per (sequence, kv head); split-free. 4 warps and
+// one buffer for K then V when the keys fit (KP <= 160: four CTAs share an
+// SM), else 8 warps and separate K and V buffers.
 // * All G query heads of the kv head and all n_q tokens are one set of
 //   R = n_q * G query rows (32 for n_q = 4, G = 8), so each ring byte is read
 //   from HBM exactly once for all of them.
@@ -17,18 +19,19 @@
 //   swizzle, 64 head-dim columns per box): the ring slice (W rows of D bf16,
 //   Hkv * D apart in HBM) and the n_q new rows of K, then of V, plus the Q
 //   rows; K and Q complete on one mbarrier, V on a second one that lands
-//   while the scores are computed. (16-byte cp.async from every thread took
+//   while the scores are computed (with one buffer: V is loaded over K once
+//   S is done, while the softmax runs). (16-byte cp.async from every thread took
 //   about a third of a CTA's cycles just to issue.) The new rows go to row
 //   roundup8(W) so that every box starts on a 1024-byte swizzle atom.
 // * The contraction has ~25 flop per HBM byte, above what CUDA-core FMAs hide,
 //   so S = Q K^T and O = P V use the tensor cores through mma.sync m16n8k16
 //   (bf16, f32 accumulate); the tiles (32 rows) are too small for tcgen05.
 //   ldmatrix addresses follow the swizzle.
-// * Softmax: the 8 warps split the keys for S; row maxima and sums are
+// * Softmax: the warps split the keys for S; row maxima and sums are
 //   reduced inside the quad that shares a row (warp shuffles), then across
 //   warps through shared memory. The max is seeded with the sink logit and
 //   the denominator gets the sink term exp(s - m). P goes to shared memory as
-//   bf16; the 8 warps then split the head dim for O = P V.
+//   bf16 over Q's place; the warps then split the head dim for O = P V.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
