@@ -154,11 +154,6 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.x / p.Hkv;
   const int g = blockIdx.x - b * p.Hkv;
-  int P = __ldg(p.pos + b);
-  if (P < 0) {
-    if (tid == 0) flag_error(2u);
-    P = 0;
-  }
   const int W = p.W, n_q = p.n_q, G = p.G;
 
   // ---- loads: Q and K on bar_qk, V on bar_v (one thread issues) ------------
@@ -208,10 +203,19 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
   }
 
   // ---- this thread's rows (fragment rows lane/4 and lane/4 + 8 per m-tile) --
-  // ring slot s holds the token at position P - W + rel(s), rel(s) = (s - P) mod W;
-  // query t sees it iff rel >= max(t + 1, W - P); new token u iff u <= t.
+  // (read after the loads are on their way)
+  int P = __ldg(p.pos + b);
+  if (P < 0) {
+    if (tid == 0) flag_error(2u);
+    P = 0;
+  }
+  // Key ranks: ring slot s holds the token at position P - W + rel(s) with
+  // rel(s) = (s - P) mod W, rank rel(s); new token u has rank W + u. Query t
+  // sees ring tokens with rel >= max(t + 1, W - P) and new tokens u <= t: the
+  // ranks [lo_t, W + t], one contiguous range.
   const int Pmod = P % W;
-  int trow[MT][2], thr[MT][2];
+  int trow[MT][2], rlo[MT][2];
+  unsigned rspan[MT][2];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -219,7 +223,8 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
       const int row = mt * 16 + (lane >> 2) + hf * 8;
       const int t = row < p.R ? row / G : -1;  // -1: padding row, sees nothing
       trow[mt][hf] = t;
-      thr[mt][hf] = t >= 0 ? max(t + 1, W - P) : 0x7fffffff;
+      rlo[mt][hf] = t >= 0 ? max(t + 1, W - P) : 0x7fffffff;
+      rspan[mt][hf] = t >= 0 ? static_cast<unsigned>(W + t - rlo[mt][hf]) : 0u;
     }
 
   // Q and K in shared memory (the zeroing above is published by the same
@@ -283,17 +288,21 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
 #pragma unroll
     for (int e2 = 0; e2 < 2; ++e2) {
       const int col = nt * 8 + 2 * (lane & 3) + e2;
-      // kind of key: ring (visible iff rel >= thr), new (iff u <= t) or none
-      int rel = col - Pmod;
-      if (rel < 0) rel += W;
-      const bool ring = nt < NT && col < W;
-      const bool isnew = nt < NT && col >= W8 && col < W8 + n_q;
-      const int u = col - W8;
+      // this key's rank (0x3fffffff: padding, seen by no query)
+      int rank = 0x3fffffff;
+      if (nt < NT) {
+        if (col < W) {
+          rank = col - Pmod;
+          if (rank < 0) rank += W;
+        } else if (col >= W8 && col < W8 + n_q) {
+          rank = W + (col - W8);
+        }
+      }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-          const bool vis = (ring && rel >= thr[mt][hf]) || (isnew && u <= trow[mt][hf]);
+          const bool vis = static_cast<unsigned>(rank - rlo[mt][hf]) <= rspan[mt][hf];
           float& x = s[mt][j][hf * 2 + e2];
           x = vis ? x * p.scale_log2 : -INFINITY;
           mloc[mt][hf] = fmaxf(mloc[mt][hf], x);
