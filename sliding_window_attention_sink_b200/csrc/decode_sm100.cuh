@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
                         const __grid_constant__ CUtensorMap tm_kr,
                         const __grid_constant__ CUtensorMap tm_kn,
                         const __grid_constant__ CUtensorMap tm_vr,
-                        const __grid_constant__ CUtensorMap tm_vn, const DecodeParams p) {
+                        const __grid_constant__ CUtensorMap tm_vn,
+                        const __grid_constant__ CUtensorMap tm_o, const DecodeParams p) {
   constexpr bool SHARE = NWP == kDecodeSmallWarps;  // one buffer for K, then V
   constexpr int NT_ = NWP * 32;
   constexpr int NCH = D / 64;      // 64-column blocks of the head dim
@@ -226,6 +227,22 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
       rlo[mt][hf] = t >= 0 ? max(t + 1, W - P) : 0x7fffffff;
       rspan[mt][hf] = t >= 0 ? static_cast<unsigned>(W + t - rlo[mt][hf]) : 0u;
     }
+  // the sinks of this thread's rows (log2 units), fetched while the loads fly
+  float srow[MT][2];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int row = mt * 16 + (lane >> 2) + hf * 8;
+      srow[mt][hf] = (trow[mt][hf] >= 0 && p.sink != nullptr)
+                         ? __ldg(p.sink + g * G + (row - trow[mt][hf] * G)) * kLog2e
+                         : -INFINITY;
+    }
+  float sk_tid = -INFINITY;  // the sink of row tid, for the row sums below
+  if (tid < p.R && p.sink != nullptr) {
+    const int t = tid / G;
+    sk_tid = __ldg(p.sink + g * G + (tid - t * G)) * kLog2e;
+  }
 
   // Q and K in shared memory (the zeroing above is published by the same
   // barrier); a wait that gave up ends every thread of the CTA here
@@ -321,20 +338,16 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
   __syncthreads();
 
   // ---- row max over warps and the sink; P = exp2(x - m) -> smem; row sums --
-  float mrow[MT][2], srow[MT][2];
+  float mrow[MT][2];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const int row = mt * 16 + (lane >> 2) + hf * 8;
-      const float sk = (trow[mt][hf] >= 0 && p.sink != nullptr)
-                           ? __ldg(p.sink + g * G + (row - trow[mt][hf] * G)) * kLog2e
-                           : -INFINITY;
-      float m = sk;
+      float m = srow[mt][hf];
 #pragma unroll
       for (int w = 0; w < NWP; ++w) m = fmaxf(m, red_max[w * 32 + row]);
       mrow[mt][hf] = (m == -INFINITY) ? 0.f : m;
-      srow[mt][hf] = sk;
     }
   float lr[MT][2], lx[MT][2];
   const uint32_t sP = smem_u32(Ps);
@@ -379,10 +392,9 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
   // row sums over warps plus the sink term; LSE (one thread per row)
   if (tid < RP) {
     const int row = tid;
-    float m = -INFINITY, sk = -INFINITY;
     const int t = row < p.R ? row / G : -1;
-    if (t >= 0 && p.sink != nullptr) sk = __ldg(p.sink + g * G + (row - t * G)) * kLog2e;
-    m = sk;
+    const float sk = sk_tid;
+    float m = sk;
     for (int w = 0; w < NWP; ++w) m = fmaxf(m, red_max[w * 32 + row]);
     const float mb = (m == -INFINITY) ? 0.f : m;
     float l = 0.f, lxs = 0.f;
@@ -440,25 +452,36 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
     }
   }
 
-  // ---- O / l -> bf16 ----------------------------------------------------------
+  // ---- O / l -> bf16 into a swizzled staging tile (K/V's buffer, free once
+  // every warp is past PV), then one TMA box store per 64 columns ----------
+  __syncthreads();
+  const uint32_t sO = sK;  // NCH blocks of [32 rows][128 bytes]
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const int t = trow[mt][hf];
-      if (t >= 0) {
-        const int row = mt * 16 + (lane >> 2) + hf * 8;
+      const int row = mt * 16 + (lane >> 2) + hf * 8;
+      if (trow[mt][hf] >= 0) {
         const float inv_l = 1.f / row_l[row];
-        __nv_bfloat16* orow =
-            p.o + ((static_cast<size_t>(b) * n_q + t) * p.Hq + g * G + (row - t * G)) * D;
 #pragma unroll
         for (int jn = 0; jn < NTO; ++jn) {
-          const int col = warp * DW + jn * 8 + 2 * (lane & 3);
-          *reinterpret_cast<uint32_t*>(orow + col) =
-              pack_bf16x2(acc[mt][jn][2 * hf] * inv_l, acc[mt][jn][2 * hf + 1] * inv_l);
+          const int col = warp * DW + jn * 8;
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sw128_addr(sO, 32, row, col) +
+                                                        4 * (lane & 3)),
+                       "r"(pack_bf16x2(acc[mt][jn][2 * hf] * inv_l,
+                                       acc[mt][jn][2 * hf + 1] * inv_l))
+                       : "memory");
         }
       }
     }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (tid == 0) {
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) tma_store_4d(&tm_o, sO + ch * 32 * 128, ch * 64, g * G, 0, b);
+    tma_store_commit();
+    tma_store_wait_read<0>();  // the staging tile is read before the CTA leaves
+  }
 }
 
 // Copy accepted new tokens into their ring slots: block = (sequence, token).

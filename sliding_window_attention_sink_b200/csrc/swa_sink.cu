@@ -393,21 +393,23 @@ template <int D, int MT, int NWP>
 int launch_decode(const swa::DecodeParams& p, cudaStream_t st) {
   // boxes of 64 head-dim columns: Q [G heads x n_q tokens], ring [W rows],
   // new rows [n_q rows], of one (sequence, kv head)
-  CUtensorMap tq, tkr, tkn, tvr, tvn;
+  CUtensorMap tq, tkr, tkn, tvr, tvn, to;
   const uint32_t G = static_cast<uint32_t>(p.G), nq = static_cast<uint32_t>(p.n_q);
   const uint32_t W = static_cast<uint32_t>(p.W);
   if (encode_4d(&tq, p.q, D, p.Hq, p.n_q, p.B, 64, G, nq, 1) != SWA_OK ||
       encode_4d(&tkr, p.k_ring, D, p.Hkv, p.W, p.B, 64, 1, W, 1) != SWA_OK ||
       encode_4d(&tkn, p.k_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK ||
       encode_4d(&tvr, p.v_ring, D, p.Hkv, p.W, p.B, 64, 1, W, 1) != SWA_OK ||
-      encode_4d(&tvn, p.v_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK)
+      encode_4d(&tvn, p.v_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK ||
+      encode_4d(&to, p.o, D, p.Hq, p.n_q, p.B, 64, G, nq, 1) != SWA_OK)
     return SWA_ERR_CUDA;
   const size_t smem = swa::decode_smem_bytes(D, p.KP, NWP);
   auto kern = swa::decode_sm100_kernel<D, MT, NWP>;
   if (ensure_smem_attr(kern, smem,
                        g_attr_dec[D == 128][MT - 1][NWP == swa::kDecodeLargeWarps]) != SWA_OK)
     return SWA_ERR_CUDA;
-  kern<<<static_cast<unsigned>(p.B) * p.Hkv, NWP * 32, smem, st>>>(tq, tkr, tkn, tvr, tvn, p);
+  kern<<<static_cast<unsigned>(p.B) * p.Hkv, NWP * 32, smem, st>>>(tq, tkr, tkn, tvr, tvn, to,
+                                                                    p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SWA_OK : cuda_fail("decode launch", e);
 }
