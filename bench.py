@@ -79,24 +79,36 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+# The device sources (and the launch code in swa_sink.cu) that decide each
+# workload's kernel; a recorded DRAM traffic figure holds only while they are
+# unchanged.
+KERNEL_SOURCES = {
+    "ring": ["prefill_swa_ring_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
+    "chunked": ["prefill_chunked_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
+    "decode": ["decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
+}
+WORKLOAD_KERNEL = {"tiny_swa_prefill": "ring", "swa_prefill_32k": "ring",
+                   "varlen_swa_prefill": "ring", "global_prefill_8k": "chunked",
+                   "swa_decode_mtp": "decode"}
+
+
+def kernel_source_hash(workload):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sliding_window_attention_sink_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, fn), "rb").read())
+    for fn in KERNEL_SOURCES[WORKLOAD_KERNEL[workload]]:
+        h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+    the current sources of the workload's kernel; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         rec = json.load(open(path)).get(workload)
     except Exception:
         return None
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(workload):
         return None
     return rec.get("dram_bytes_per_launch")
 
