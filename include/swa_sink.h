@@ -47,6 +47,7 @@
 #ifndef SWA_SINK_H
 #define SWA_SINK_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -166,6 +167,43 @@ SWA_API int swa_sink_attn_decode(const void *q, const void *k_new, const void *v
                          const int32_t *pos, int B, int n_q, int Hq, int Hkv,
                          int D, int W, const float *sink, float softmax_scale,
                          void *o, float *lse, void *stream);
+
+/*
+ * Decode / draft verification over a long KV cache, split over the cached
+ * positions: the global-attention layers of section 2.2 of the report summary
+ * above (every earlier token visible) at decode, with the MTP verification of
+ * section 2.3 and the sink of section 2.2.2.
+ *
+ * The cache follows the ring convention of swa_sink_attn_decode (the token at
+ * position p in slot p mod W; query t sees cached positions
+ * max(0, pos[b]+t-W+1) .. pos[b]-1 and the new tokens 0..t), so the result is
+ * exactly what swa_sink_attn_decode defines, for any W that is a multiple of
+ * 64. With W at least the context length the cache is a plain array indexed
+ * by position and every earlier token is visible (a global layer).
+ *
+ *   k_cache, v_cache  bf16 [B, W, Hkv, D]
+ *   max_ctx   an upper bound on every pos[b] (the host does not read pos): it
+ *             sizes the split. A pos[b] beyond the cover is flagged (bit 1 of
+ *             swa_sink_device_error) and its excess positions are skipped.
+ *   workspace device memory of at least swa_sink_decode_splitkv_workspace()
+ *             bytes, 16-byte aligned, owned by the caller; it holds the
+ *             partial softmax states between the two kernels of a call, so
+ *             calls that overlap in time need separate workspaces.
+ *   the other arguments as for swa_sink_attn_decode (n_q 1..8,
+ *   n_q*(Hq/Hkv) <= 32, D 64 or 128).
+ *
+ * Returns SWA_OK or a negative swa_status_t (SWA_ERR_UNSUPPORTED when W is
+ * not a multiple of 64; SWA_ERR_SHAPE when the workspace is too small).
+ */
+SWA_API size_t swa_sink_decode_splitkv_workspace(int B, int n_q, int Hq, int Hkv, int D,
+                                                 int W, int max_ctx);
+SWA_API int swa_sink_attn_decode_splitkv(const void *q, const void *k_new, const void *v_new,
+                                         const void *k_cache, const void *v_cache,
+                                         const int32_t *pos, int B, int n_q, int Hq, int Hkv,
+                                         int D, int W, int max_ctx, const float *sink,
+                                         float softmax_scale, void *o, float *lse,
+                                         void *workspace, size_t workspace_bytes,
+                                         void *stream);
 
 /*
  * Commit accepted tokens into the ring after verification: for

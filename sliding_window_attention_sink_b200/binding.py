@@ -49,6 +49,12 @@ def load():
     lib.swa_sink_attn_decode.restype = _i
     lib.swa_sink_attn_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                          _i, _vp, _f, _vp, _vp, _vp]
+    lib.swa_sink_decode_splitkv_workspace.restype = ctypes.c_size_t
+    lib.swa_sink_decode_splitkv_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+    lib.swa_sink_attn_decode_splitkv.restype = _i
+    lib.swa_sink_attn_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                                 _i, _i, _i, _vp, _f, _vp, _vp, _vp,
+                                                 ctypes.c_size_t, _vp]
     lib.swa_sink_kv_commit.restype = _i
     lib.swa_sink_kv_commit.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
     lib.swa_sink_status_string.restype = ctypes.c_char_p
@@ -105,6 +111,21 @@ def swa_sink_attn_decode(q, k_new, v_new, k_ring, v_ring, pos, B, n_q, Hq, Hkv, 
         _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring), _ptr(v_ring), _ptr(pos), int(B),
         int(n_q), int(Hq), int(Hkv), int(D), int(W), _ptr(sink), float(softmax_scale),
         _ptr(o), _ptr(lse), _stream(stream))
+
+
+def swa_sink_decode_splitkv_workspace(B, n_q, Hq, Hkv, D, W, max_ctx):
+    return load().swa_sink_decode_splitkv_workspace(int(B), int(n_q), int(Hq), int(Hkv), int(D),
+                                                    int(W), int(max_ctx))
+
+
+def swa_sink_attn_decode_splitkv(q, k_new, v_new, k_cache, v_cache, pos, B, n_q, Hq, Hkv, D, W,
+                                 max_ctx, sink, softmax_scale, o, lse, workspace,
+                                 workspace_bytes, stream=None):
+    return load().swa_sink_attn_decode_splitkv(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(pos), int(B),
+        int(n_q), int(Hq), int(Hkv), int(D), int(W), int(max_ctx), _ptr(sink),
+        float(softmax_scale), _ptr(o), _ptr(lse), _ptr(workspace), int(workspace_bytes),
+        _stream(stream))
 
 
 def swa_sink_kv_commit(k_ring, v_ring, k_new, v_new, pos, n_accept, B, n_q, Hkv, D, W,
@@ -166,6 +187,30 @@ def attn_decode(q, k_new, v_new, k_ring, v_ring, pos, sink=None, softmax_scale=0
                               sink, softmax_scale, out, lse, stream)
     if rc != SWA_OK:
         raise SwaSinkError(rc, "swa_sink_attn_decode")
+    return out, lse
+
+
+def attn_decode_splitkv(q, k_new, v_new, k_cache, v_cache, pos, max_ctx, sink=None,
+                        softmax_scale=0.0, out=None, lse=None, want_lse=True, workspace=None,
+                        stream=None):
+    """Like attn_decode over a cache [B,W,Hkv,D] of any W that is a multiple of
+    64 (W >= the context: a global layer). The workspace (a uint8 CUDA tensor)
+    is allocated here when not given."""
+    B, n_q, Hq, D = q.shape
+    Hkv = k_new.shape[2]
+    W = k_cache.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q, Hq), dtype=torch.float32, device=q.device)
+    need = swa_sink_decode_splitkv_workspace(B, n_q, Hq, Hkv, D, W, max_ctx)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = swa_sink_attn_decode_splitkv(q, k_new, v_new, k_cache, v_cache, pos, B, n_q, Hq, Hkv,
+                                      D, W, max_ctx, sink, softmax_scale, out, lse, workspace,
+                                      workspace.numel(), stream)
+    if rc != SWA_OK:
+        raise SwaSinkError(rc, "swa_sink_attn_decode_splitkv")
     return out, lse
 
 

@@ -389,6 +389,15 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
     }
   // V in shared memory; a wait that gave up ends every thread here
   if (!__syncthreads_and(mbar_wait(smem_u32(&bar_v), 0, abort))) return;
+  // with fewer than W committed tokens the slots P .. W-1 were never written
+  // and may hold anything: their P is 0, and 0 * V must stay 0
+  if (P < W) {
+    for (int idx = tid; idx < NCH * (W - P) * 8; idx += NT_) {
+      const int ch = idx / ((W - P) * 8);
+      const int rem = idx - ch * (W - P) * 8;
+      st_shared_zero16(sV + ch * KP * 128 + (P + (rem >> 3)) * 128 + (rem & 7) * 16);
+    }
+  }
   // row sums over warps plus the sink term; LSE (one thread per row)
   if (tid < RP) {
     const int row = tid;

@@ -19,6 +19,7 @@
 
 #include "../../include/swa_sink.h"
 #include "decode_sm100.cuh"
+#include "decode_splitkv_sm100.cuh"
 #include "prefill_chunked_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "prefill_swa_ring_sm100.cuh"
@@ -462,6 +463,55 @@ int fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seql
                              softmax_scale, o, lse, st);
 }
 
+// ---- split-KV decode ------------------------------------------------------------
+// Ranges per (sequence, kv head) and their length: enough CTAs for a few waves
+// (a fixed target, so that the workspace size does not depend on the device),
+// no more ranges than 64-key tiles.
+constexpr long long kSplitTargetCtas = 1184;
+void split_shape(int B, int Hkv, int W, int max_ctx, int* S, int* chunk) {
+  const long long span = std::max(1, std::min(W, max_ctx));
+  const long long units = std::max(1LL, static_cast<long long>(B) * Hkv);
+  long long s = (kSplitTargetCtas + units - 1) / units;
+  s = std::max(1LL, std::min(s, (span + swa::kSplitTile - 1) / swa::kSplitTile));
+  long long c = (span + s - 1) / s;
+  c = (c + swa::kSplitTile - 1) / swa::kSplitTile * swa::kSplitTile;
+  *chunk = static_cast<int>(c);
+  *S = static_cast<int>((span + c - 1) / c);
+}
+
+size_t split_workspace_bytes(int B, int Hkv, int D, int W, int max_ctx) {
+  int S = 0, chunk = 0;
+  split_shape(B, Hkv, W, max_ctx, &S, &chunk);
+  return static_cast<size_t>(B) * Hkv * S * 32 * (D + 4) * sizeof(float);
+}
+
+size_t g_attr_split[2][2][kMaxDevices];
+
+template <int D, int MT>
+int launch_split(const swa::SplitParams& p, const void* q, const void* k_new, const void* v_new,
+                 const void* k_cache, const void* v_cache, cudaStream_t st) {
+  CUtensorMap tq, tkc, tvc, tkn, tvn;
+  const uint32_t G = static_cast<uint32_t>(p.G), nq = static_cast<uint32_t>(p.n_q);
+  if (encode_4d(&tq, q, D, p.Hq, p.n_q, p.B, 64, G, nq, 1) != SWA_OK ||
+      encode_4d(&tkc, k_cache, D, p.Hkv, p.W, p.B, 64, 1, swa::kSplitTile, 1) != SWA_OK ||
+      encode_4d(&tvc, v_cache, D, p.Hkv, p.W, p.B, 64, 1, swa::kSplitTile, 1) != SWA_OK ||
+      encode_4d(&tkn, k_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK ||
+      encode_4d(&tvn, v_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK)
+    return SWA_ERR_CUDA;
+  const size_t smem = swa::split_smem_bytes(D);
+  auto kern = swa::decode_split_kernel<D, MT>;
+  if (ensure_smem_attr(kern, smem, g_attr_split[D == 128][MT - 1]) != SWA_OK) return SWA_ERR_CUDA;
+  const long long units = static_cast<long long>(p.B) * p.Hkv;
+  if (units * p.S > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  kern<<<static_cast<unsigned>(units * p.S), swa::kSplitWarps * 32, smem, st>>>(tq, tkc, tvc, tkn,
+                                                                                 tvn, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("split-KV decode launch", e);
+  swa::decode_split_combine_kernel<D><<<static_cast<unsigned>(units), D, 0, st>>>(p);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SWA_OK : cuda_fail("split-KV combine launch", e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -545,6 +595,57 @@ int swa_sink_attn_decode(const void* q, const void* k_new, const void* v_new, co
   constexpr int L = swa::kDecodeLargeWarps;
   if (D == 64) return two ? launch_decode<64, 2, L>(p, st) : launch_decode<64, 1, L>(p, st);
   return two ? launch_decode<128, 2, L>(p, st) : launch_decode<128, 1, L>(p, st);
+}
+
+size_t swa_sink_decode_splitkv_workspace(int B, int n_q, int Hq, int Hkv, int D, int W,
+                                          int max_ctx) {
+  if (B < 0 || n_q <= 0 || Hq <= 0 || Hkv <= 0 || W <= 0 || max_ctx < 0) return 0;
+  if (D != 64 && D != 128) return 0;
+  return split_workspace_bytes(B, Hkv, D, W, max_ctx);
+}
+
+int swa_sink_attn_decode_splitkv(const void* q, const void* k_new, const void* v_new,
+                                 const void* k_cache, const void* v_cache, const int32_t* pos,
+                                 int B, int n_q, int Hq, int Hkv, int D, int W, int max_ctx,
+                                 const float* sink, float softmax_scale, void* o, float* lse,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 0 || n_q <= 0 || Hq <= 0 || Hkv <= 0 || W <= 0 || max_ctx < 0) return SWA_ERR_SHAPE;
+  if (Hq % Hkv != 0) return SWA_ERR_SHAPE;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (n_q > 8 || n_q * (Hq / Hkv) > 32) return SWA_ERR_UNSUPPORTED;
+  if (W % swa::kSplitTile != 0) return SWA_ERR_UNSUPPORTED;
+  if (B == 0) return SWA_OK;
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !pos || !o || !workspace)
+    return SWA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(o) || !aligned16(workspace))
+    return SWA_ERR_ALIGN;
+  if (!aligned4(pos) || (sink && !aligned4(sink)) || (lse && !aligned4(lse))) return SWA_ERR_ALIGN;
+  if (workspace_bytes < split_workspace_bytes(B, Hkv, D, W, max_ctx)) return SWA_ERR_SHAPE;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
+  swa::SplitParams p;
+  p.pos = pos;
+  p.B = B;
+  p.n_q = n_q;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.W = W;
+  p.R = n_q * p.G;
+  split_shape(B, Hkv, W, max_ctx, &p.S, &p.chunk);
+  p.sink = sink;
+  p.scale_log2 = softmax_scale * swa::kLog2e;
+  p.part = static_cast<float*>(workspace);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool two = p.R > 16;
+  if (D == 64)
+    return two ? launch_split<64, 2>(p, q, k_new, v_new, k_cache, v_cache, st)
+               : launch_split<64, 1>(p, q, k_new, v_new, k_cache, v_cache, st);
+  return two ? launch_split<128, 2>(p, q, k_new, v_new, k_cache, v_cache, st)
+             : launch_split<128, 1>(p, q, k_new, v_new, k_cache, v_cache, st);
 }
 
 int swa_sink_kv_commit(void* k_ring, void* v_ring, const void* k_new, const void* v_new,

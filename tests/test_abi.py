@@ -117,3 +117,20 @@ def test_fwd_noalloc_argument_errors():
     assert B.swa_sink_attn_fwd_noalloc(slot=0, **dict(a, q=None)) == -1
     assert B.swa_sink_attn_fwd_noalloc(slot=0, **dict(a, o=FAKE + 2)) == -4
     assert B.swa_sink_attn_fwd_noalloc(slot=3, **dict(a, total_tokens=0, max_seqlen=0)) == 0
+
+
+def test_splitkv_workspace_and_argument_errors():
+    ws = B.swa_sink_decode_splitkv_workspace(4, 4, 64, 8, 128, 4096, 4000)
+    assert ws > 0
+    assert B.swa_sink_decode_splitkv_workspace(4, 4, 64, 8, 96, 4096, 4000) == 0
+    a = dict(q=FAKE, k_new=FAKE, v_new=FAKE, k_cache=FAKE, v_cache=FAKE, pos=FAKE, B=4, n_q=4,
+             Hq=64, Hkv=8, D=128, W=4096, max_ctx=4000, sink=None, softmax_scale=0.0, o=FAKE,
+             lse=None, workspace=FAKE, workspace_bytes=ws, stream=0)
+    f = B.swa_sink_attn_decode_splitkv
+    assert f(**dict(a, W=4000)) == -3          # W not a multiple of 64
+    assert f(**dict(a, workspace_bytes=ws - 1)) == -2
+    assert f(**dict(a, workspace=None)) == -1
+    assert f(**dict(a, workspace=FAKE + 4)) == -4
+    assert f(**dict(a, n_q=9)) == -3
+    assert f(**dict(a, Hq=64, Hkv=6)) == -2
+    assert f(**dict(a, B=0)) == 0
