@@ -56,15 +56,18 @@ def prefill_work(seqlens, Hq, Hkv, D, window):
 
 
 def decode_work(pos, n_q, Hq, Hkv, D, W):
-    """FLOPs over visible pairs; bytes = ring K/V + new K/V + q + pos + sink
-    read once, o + lse written once."""
+    """FLOPs over visible pairs; bytes = the cached K/V rows of committed
+    tokens (min(pos, W) per sequence) + new K/V + q + pos + sink read once,
+    o + lse written once."""
     pairs = 0
+    cached = 0
     for P in pos:
+        cached += min(P, W)
         for t in range(n_q):
             pairs += min(P, W - 1 - t) + (t + 1)   # ring keys + new keys 0..t
     B = len(pos)
     flops = 4 * D * Hq * pairs
-    nbytes = (B * W * Hkv * D * 2 * 2 + B * n_q * Hkv * D * 2 * 2
+    nbytes = (cached * Hkv * D * 2 * 2 + B * n_q * Hkv * D * 2 * 2
               + B * n_q * Hq * D * 2 * 2 + B * n_q * Hq * 4 + B * 4 + Hq * 4)
     return flops, nbytes
 
@@ -86,10 +89,11 @@ KERNEL_SOURCES = {
     "ring": ["prefill_swa_ring_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "chunked": ["prefill_chunked_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "decode": ["decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
+    "splitkv": ["decode_splitkv_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
 }
 WORKLOAD_KERNEL = {"tiny_swa_prefill": "ring", "swa_prefill_32k": "ring",
                    "varlen_swa_prefill": "ring", "global_prefill_8k": "chunked",
-                   "swa_decode_mtp": "decode"}
+                   "swa_decode_mtp": "decode", "ga_decode_16k": "splitkv"}
 
 
 def kernel_source_hash(workload):
@@ -198,6 +202,7 @@ class PrefillRunner:
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
         self.units = c["total"]
+        self.launches_per_call = 2 if getattr(self, "full", False) else 1
 
     def call(self, stream):
         c = self.c
@@ -214,9 +219,9 @@ class PrefillRunner:
 
 
 class DecodeRunner:
-    """The decode batch reads ~170 MB, close to the 126 MB L2, so the timed
-    steps rotate over three independent input sets (> 500 MB together)."""
-    NSETS = 3
+    """The SWA decode batch reads ~170 MB, close to the 126 MB L2, so the
+    timed steps rotate over three independent input sets (> 500 MB together);
+    a global-layer batch (cache "full", split-KV call) is far larger than L2."""
 
     def __init__(self, case, rank, torch, B, wl):
         self.torch, self.B = torch, B
@@ -228,8 +233,16 @@ class DecodeRunner:
         dev = torch.device("cuda")
         names = ["q", "k_new", "v_new", "k_ring", "v_ring", "pos", "sink"]
         self.g = {n: d[n].to(dev) for n in names}
+        self.full = case.cache == "full"
+        self.max_ctx = case.pos_hi
+        self.NSETS = 1 if self.full else 3
         self.sets = [self.g] + [{n: (t.clone() if n != "pos" else t) for n, t in self.g.items()}
                                 for _ in range(self.NSETS - 1)]
+        self.ws = None
+        if self.full:
+            need = B.swa_sink_decode_splitkv_workspace(d["B"], d["n_q"], d["Hq"], d["Hkv"],
+                                                       d["D"], d["W"], self.max_ctx)
+            self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.turn = 0
         self.o = torch.empty_like(self.g["q"])
         self.lse = torch.empty((d["B"], d["n_q"], d["Hq"]), dtype=torch.float32, device=dev)
@@ -241,10 +254,19 @@ class DecodeRunner:
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
         self.units = d["B"]
+        self.launches_per_call = 2 if getattr(self, "full", False) else 1
 
     def call(self, stream):
         d, g = self.d, self.sets[self.turn]
         self.turn = (self.turn + 1) % self.NSETS
+        if self.full:
+            rc = self.B.swa_sink_attn_decode_splitkv(
+                g["q"], g["k_new"], g["v_new"], g["k_ring"], g["v_ring"], g["pos"], d["B"],
+                d["n_q"], d["Hq"], d["Hkv"], d["D"], d["W"], self.max_ctx, g["sink"], 0.0,
+                self.o, self.lse, self.ws, self.ws.numel(), stream)
+            if rc != 0:
+                raise RuntimeError("swa_sink_attn_decode_splitkv: %s" % self.B.status_string(rc))
+            return
         rc = self.B.swa_sink_attn_decode(g["q"], g["k_new"], g["v_new"], g["k_ring"],
                                          g["v_ring"], g["pos"], d["B"], d["n_q"], d["Hq"],
                                          d["Hkv"], d["D"], d["W"], g["sink"], 0.0, self.o,
@@ -255,7 +277,7 @@ class DecodeRunner:
     def describe(self):
         d = self.d
         return {"batch": d["B"], "n_q": d["n_q"], "Hq": d["Hq"], "Hkv": d["Hkv"],
-                "head_dim": d["D"], "ring": d["W"]}
+                "head_dim": d["D"], ("cache" if self.full else "ring"): d["W"]}
 
 
 # ------------------------------------------------------------ oracle timing --
@@ -538,7 +560,7 @@ def main():
                                    (runner.bytes / 1e6))},
                            **runner.describe()),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps, "clocks": clk.summary(), "device_error_flags": flag,
+            "gpu_launches": args.steps * runner.launches_per_call, "clocks": clk.summary(), "device_error_flags": flag,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -13,9 +13,10 @@
 //
 // Split-KV ("flash decoding"): the cached positions of a (sequence, kv head)
 // are cut into S ranges of `chunk` positions; one CTA per range streams its
-// K/V in 64-key tiles through a 2-stage TMA pipeline, keeps an online softmax
+// K/V in 64-key tiles through a 3-stage TMA pipeline, keeps an online softmax
 // over them (max in log2 units, unnormalised O, two row sums) and writes that
-// partial state. The last range also takes the n_q new tokens. A second
+// partial state. The last range also takes the n_q new tokens, as one more
+// tile through the same pipeline. A second
 // kernel merges the S partial states of each row and adds the sink term once:
 //   M = max(s, max_r m_r),  O = sum_r 2^(m_r - M) O_r / L,
 //   L = sum_r 2^(m_r - M) l_r + 2^(s - M),  LSE = (M + log2(same with l_x)) ln 2.
@@ -38,7 +39,7 @@ namespace swa {
 
 constexpr int kSplitWarps = 4;
 constexpr int kSplitTile = 64;    // keys per tile
-constexpr int kSplitStages = 2;   // K/V tiles in flight (two CTAs per SM at D = 128)
+constexpr int kSplitStages = 3;   // K/V tiles in flight (two CTAs per SM at D = 128)
 
 struct SplitParams {
   const int32_t* pos;
@@ -54,12 +55,12 @@ struct SplitParams {
 
 // Shared memory (1024-byte aligned base): kSplitStages stages of K and V tiles
 // (D/64 blocks of [64 rows][128 bytes] each, 128-byte swizzle), Q (D/64 blocks
-// of [32 rows][128 bytes]), the new-token tile of K and of V (same layout as a
-// stage), P [32][kSplitTile + 8] bf16, the row exchange [4][32] fp32.
+// of [32 rows][128 bytes]), P [32][kSplitTile + 8] bf16, the row exchange
+// [4][32] fp32.
 __host__ __device__ inline size_t split_smem_bytes(int D) {
   const size_t nch = D / 64;
   const size_t tile = nch * kSplitTile * 128;
-  return 1024 + (2 * kSplitStages + 2) * tile + nch * 32 * 128 +
+  return 1024 + 2 * kSplitStages * tile + nch * 32 * 128 +
          static_cast<size_t>(32) * (kSplitTile + 8) * 2 + 4 * 32 * sizeof(float);
 }
 
@@ -78,28 +79,28 @@ __global__ void __launch_bounds__(kSplitWarps * 32, 2)
   constexpr int NTO = DW / 8;                   // n8 tiles per warp in PV (2 or 4)
   constexpr int LDP = T + 8;                    // P row stride (bf16 elements)
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_q, bar_new, full[kSplitStages];
+  __shared__ __align__(8) uint64_t bar_q, full[kSplitStages];
   __shared__ int abort_sh;
   volatile int* abort = &abort_sh;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int unit = blockIdx.x;               // (b * Hkv + g) * S + s
-  const int bg = unit / p.S, s = unit - bg * p.S;
-  const int b = bg / p.Hkv, g = bg - b * p.Hkv;
+  // CTAs that run together take the same positions of all kv heads of a
+  // sequence (blockIdx = (b * S + s) * Hkv + g): a cached token's rows of the
+  // Hkv heads are adjacent in HBM and are then fetched at about the same time
+  const int bs = blockIdx.x / p.Hkv, g = blockIdx.x - bs * p.Hkv;
+  const int b = bs / p.S, s = bs - b * p.S;
+  const int unit = (b * p.Hkv + g) * p.S + s;  // partial-state slot
   const int W = p.W, n_q = p.n_q, G = p.G;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sKs = base;                           // stage st: sKs + st * 2 * TILE
-  const uint32_t sNK = base + 2 * kSplitStages * TILE; // new-token K, then V
-  const uint32_t sNV = sNK + TILE;
-  const uint32_t sQ = sNV + TILE;
+  const uint32_t sKs = base;  // stage st: K at sKs + st * 2 * TILE, V TILE further
+  const uint32_t sQ = base + 2 * kSplitStages * TILE;
   uint8_t* gen = smem_raw + (sQ + NCH * 32 * 128 - smem_u32(smem_raw));
   __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(gen);
   float* red = reinterpret_cast<float*>(gen + 32 * LDP * 2);  // [4][32]
 
   if (tid == 0) {
     mbar_init(smem_u32(&bar_q), 1);
-    mbar_init(smem_u32(&bar_new), 1);
     for (int i = 0; i < kSplitStages; ++i) mbar_init(smem_u32(&full[i]), 1);
     abort_sh = 0;
     fence_barrier_init();
@@ -119,17 +120,30 @@ __global__ void __launch_bounds__(kSplitWarps * 32, 2)
   const int t0 = (r0 / T) * T;                      // first tile start
   const int ntile = r1 > r0 ? (r1 - t0 + T - 1) / T : 0;
   const bool last = s == p.S - 1;                   // also takes the new tokens
+  const int nall = ntile + (last ? 1 : 0);          // tiles through the pipeline
 
   // loads: Q (and the new tokens) once; K/V tiles through the stages
-  auto issue_tile = [&](int i) {  // tile i -> stage i % kSplitStages
+  // tile i -> stage i % kSplitStages: cached positions, or for i == ntile the
+  // n_q new tokens in rows 0 .. n_q-1
+  auto issue_tile = [&](int i) {
     const int st = i % kSplitStages;
     const uint32_t bar = smem_u32(&full[st]);
-    const int slot = (t0 + i * T) % W;  // W % T == 0: a tile never wraps
-    mbar_arrive_expect_tx(bar, 2 * TILE);
+    const uint32_t dk = sKs + st * 2 * TILE, dv = dk + TILE;
+    if (i < ntile) {
+      const int slot = (t0 + i * T) % W;  // W % T == 0: a tile never wraps
+      mbar_arrive_expect_tx(bar, 2 * TILE);
 #pragma unroll
-    for (int ch = 0; ch < NCH; ++ch) {
-      tma_load_4d(sKs + st * 2 * TILE + ch * T * 128, &tm_kc, bar, ch * 64, g, slot, b);
-      tma_load_4d(sKs + st * 2 * TILE + TILE + ch * T * 128, &tm_vc, bar, ch * 64, g, slot, b);
+      for (int ch = 0; ch < NCH; ++ch) {
+        tma_load_4d(dk + ch * T * 128, &tm_kc, bar, ch * 64, g, slot, b);
+        tma_load_4d(dv + ch * T * 128, &tm_vc, bar, ch * 64, g, slot, b);
+      }
+    } else {
+      mbar_arrive_expect_tx(bar, 2 * NCH * n_q * 128);
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch) {
+        tma_load_4d(dk + ch * T * 128, &tm_kn, bar, ch * 64, g, 0, b);
+        tma_load_4d(dv + ch * T * 128, &tm_vn, bar, ch * 64, g, 0, b);
+      }
     }
   };
   if (tid == 0) {
@@ -140,25 +154,7 @@ __global__ void __launch_bounds__(kSplitWarps * 32, 2)
 #pragma unroll
     for (int ch = 0; ch < NCH; ++ch)
       tma_load_4d(sQ + ch * 32 * 128, &tm_q, smem_u32(&bar_q), ch * 64, g * G, 0, b);
-    if (last) {
-      mbar_arrive_expect_tx(smem_u32(&bar_new), 2 * NCH * n_q * 128);
-#pragma unroll
-      for (int ch = 0; ch < NCH; ++ch) {
-        tma_load_4d(sNK + ch * T * 128, &tm_kn, smem_u32(&bar_new), ch * 64, g, 0, b);
-        tma_load_4d(sNV + ch * T * 128, &tm_vn, smem_u32(&bar_new), ch * 64, g, 0, b);
-      }
-    }
-    for (int i = 0; i < min(ntile, kSplitStages); ++i) issue_tile(i);
-  }
-  // the new-token V tile's rows past n_q are zeroed (P is 0 there; 0 * V must
-  // stay 0 whatever those bytes are); so are a cached tile's rows past the
-  // range end, below
-  if (last) {
-    for (int idx = tid; idx < NCH * (T - n_q) * 8; idx += kSplitWarps * 32) {
-      const int ch = idx / ((T - n_q) * 8);
-      const int rem = idx - ch * (T - n_q) * 8;
-      st_shared_zero16(sNV + ch * T * 128 + (n_q + (rem >> 3)) * 128 + (rem & 7) * 16);
-    }
+    for (int i = 0; i < min(nall, kSplitStages); ++i) issue_tile(i);
   }
 
   // this thread's rows: fragment rows lane/4 and lane/4 + 8 of each m-tile
@@ -294,37 +290,34 @@ __global__ void __launch_bounds__(kSplitWarps * 32, 2)
     }
   };
 
-  // ---- cached tiles -----------------------------------------------------------
-  for (int i = 0; i < ntile; ++i) {
+  // ---- the tiles: cached positions, then (last range) the new tokens ---------
+  for (int i = 0; i < nall; ++i) {
     const int st = i % kSplitStages;
     if (!__syncthreads_and(mbar_wait(smem_u32(&full[st]), (i / kSplitStages) & 1, abort))) return;
-    const int tp0 = t0 + i * T;  // position of key 0 of the tile
-    // V rows of positions past the range end may hold anything (slots not
-    // written yet): zeroed, since P is 0 there and 0 * V must stay 0
-    if (tp0 + T > r1) {
-      const int first = r1 - tp0;
-      for (int idx = tid; idx < NCH * (T - first) * 8; idx += kSplitWarps * 32) {
-        const int ch = idx / ((T - first) * 8);
-        const int rem = idx - ch * (T - first) * 8;
-        st_shared_zero16(sKs + st * 2 * TILE + TILE + ch * T * 128 + (first + (rem >> 3)) * 128 +
-                         (rem & 7) * 16);
-      }
+    const uint32_t sK = sKs + st * 2 * TILE, sV = sK + TILE;
+    // V rows no key of this tile may use can hold anything (slots not written
+    // yet, stale or never-initialised shared memory): zeroed, since P is 0
+    // there and 0 * V must stay 0
+    const int tp0 = t0 + i * T;  // position of key 0 of a cached tile
+    const int first = i < ntile ? max(0, min(T, r1 - tp0)) : n_q;
+    for (int idx = tid; idx < NCH * (T - first) * 8; idx += kSplitWarps * 32) {
+      const int ch = idx / ((T - first) * 8);
+      const int rem = idx - ch * (T - first) * 8;
+      st_shared_zero16(sV + ch * T * 128 + (first + (rem >> 3)) * 128 + (rem & 7) * 16);
     }
-    process(sKs + st * 2 * TILE, sKs + st * 2 * TILE + TILE, [&](int mt, int hf, int key) {
-      const int pk = tp0 + key;
-      return pk >= vlo[mt][hf] && pk < r1;
-    });
+    if (i < ntile) {
+      process(sK, sV, [&](int mt, int hf, int key) {
+        const int pk = tp0 + key;
+        return pk >= vlo[mt][hf] && pk < r1;
+      });
+    } else {
+      process(sK, sV, [&](int mt, int hf, int key) { return key < n_q && key <= trow[mt][hf]; });
+    }
     __syncthreads();  // every warp is done with the stage and with P
-    if (tid == 0 && i + kSplitStages < ntile) {
+    if (tid == 0 && i + kSplitStages < nall) {
       fence_proxy_async_smem();
       issue_tile(i + kSplitStages);
     }
-  }
-  // ---- the new tokens (last range only) ---------------------------------------
-  if (last) {
-    if (!__syncthreads_and(mbar_wait(smem_u32(&bar_new), 0, abort))) return;
-    process(sNK, sNV, [&](int mt, int hf, int key) { return key < n_q && key <= trow[mt][hf]; });
-    __syncthreads();
   }
 
   // ---- partial state: row sums over the quad and the warps, then O, m, l ------
@@ -375,33 +368,60 @@ __global__ void __launch_bounds__(kSplitWarps * 32, 2)
     }
 }
 
-// Merge of the S partial states of each (sequence, kv head): one CTA, thread
-// d handles head-dim column d of every row.
+// Merge of the S partial states: one warp per (sequence, kv head, query row).
+// Lanes take the ranges for the max and the sums, then every lane adds 4
+// head-dim columns of each range's O (independent 16-byte loads).
 template <int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(32)
     decode_split_combine_kernel(const SplitParams p) {
-  const int bg = blockIdx.x;
+  const int lane = threadIdx.x;
+  const int bg = blockIdx.x / p.R, row = blockIdx.x - bg * p.R;
   const int b = bg / p.Hkv, g = bg - b * p.Hkv;
-  const int d = threadIdx.x;
+  const int t = row / p.G, hh = row - t * p.G;
+  const int h = g * p.G + hh;
   const float* part = p.part + static_cast<size_t>(bg) * p.S * 32 * (D + 4);
-  for (int row = 0; row < p.R; ++row) {
-    const int t = row / p.G, hh = row - t * p.G;
-    const int h = g * p.G + hh;
-    const float sk = p.sink != nullptr ? __ldg(p.sink + h) * kLog2e : -INFINITY;
-    float M = sk;
-    for (int r = 0; r < p.S; ++r) M = fmaxf(M, part[(r * 32 + row) * (D + 4) + D]);
-    const float mb = (M == -INFINITY) ? 0.f : M;
-    float L = sk != -INFINITY ? ex2(sk - mb) : 0.f, LX = L, acc = 0.f;
+  const float sk = p.sink != nullptr ? __ldg(p.sink + h) * kLog2e : -INFINITY;
+  float M = sk;
+  for (int r = lane; r < p.S; r += 32) M = fmaxf(M, part[(r * 32 + row) * (D + 4) + D]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  const float mb = (M == -INFINITY) ? 0.f : M;
+  float L = 0.f, LX = 0.f;
+  for (int r = lane; r < p.S; r += 32) {
+    const float* pr = part + (r * 32 + row) * (D + 4);
+    const float w = ex2(pr[D] - mb);  // an empty range has m = -inf: weight 0
+    L += w * pr[D + 1];
+    LX += w * pr[D + 2];
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    L += __shfl_xor_sync(0xffffffffu, L, off);
+    LX += __shfl_xor_sync(0xffffffffu, LX, off);
+  }
+  if (sk != -INFINITY) {
+    const float ts = ex2(sk - mb);
+    L += ts;
+    LX += ts;
+  }
+  // O: lane takes columns [4 lane, 4 lane + 4) (D / 4 lanes)
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane * 4 < D) {
     for (int r = 0; r < p.S; ++r) {
       const float* pr = part + (r * 32 + row) * (D + 4);
-      const float w = ex2(pr[D] - mb);  // an empty range has m = -inf: weight 0
-      L += w * pr[D + 1];
-      LX += w * pr[D + 2];
-      acc += w * pr[d];
+      const float w = ex2(__ldg(pr + D) - mb);
+      const float4 v = __ldg(reinterpret_cast<const float4*>(pr) + lane);
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
     }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
     const size_t orow = (static_cast<size_t>(b) * p.n_q + t) * p.Hq + h;
-    p.o[orow * D + d] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
-    if (d == 0 && p.lse != nullptr) p.lse[orow] = (mb + lg2(LX)) * kLn2;
+    uint2 pk;
+    pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(p.o + orow * D + lane * 4) = pk;
+    if (lane == 0 && p.lse != nullptr) p.lse[orow] = (mb + lg2(LX)) * kLn2;
   }
 }
 

@@ -507,7 +507,8 @@ int launch_split(const swa::SplitParams& p, const void* q, const void* k_new, co
                                                                                  tvn, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("split-KV decode launch", e);
-  swa::decode_split_combine_kernel<D><<<static_cast<unsigned>(units), D, 0, st>>>(p);
+  if (units * p.R > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  swa::decode_split_combine_kernel<D><<<static_cast<unsigned>(units * p.R), 32, 0, st>>>(p);
   e = cudaGetLastError();
   return e == cudaSuccess ? SWA_OK : cuda_fail("split-KV combine launch", e);
 }

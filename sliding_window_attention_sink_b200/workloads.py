@@ -48,10 +48,14 @@ class DecodeCase:
     seed: int
     pos_lo: int = 128
     pos_hi: int = 262144   # inclusive
+    # "ring": a W-slot ring (sliding-window layers); "full": a cache of W >=
+    # every context (global layers, split-KV decode with max_ctx = pos_hi)
+    cache: str = "ring"
 
 
-# The five workloads: a tiny parity case, one SWA layer, one global layer, a
-# packed varlen SWA batch and a decode / draft-verification batch.
+# The workloads: a tiny parity case, one SWA layer, one global layer, a packed
+# varlen SWA batch, a decode / draft-verification batch of the SWA layers and
+# one of a global layer over long contexts.
 WORKLOADS = {
     "tiny_swa_prefill": PrefillCase(
         "tiny_swa_prefill T=512 Hq=4 Hkv=1 D=64 W=128", [512], 4, 1, 64, 128,
@@ -68,6 +72,9 @@ WORKLOADS = {
     "swa_decode_mtp": DecodeCase(
         "swa_decode B=256 n_q=4 ring=128 Hq=64 Hkv=8 D=128", 256, 4, 64, 8,
         128, 128, 0.5, "normal", 5),
+    "ga_decode_16k": DecodeCase(
+        "ga_decode B=16 n_q=4 ctx~U[8192,16380] cache=16384 Hq=64 Hkv=8 D=128", 16, 4,
+        64, 8, 128, 16384, 0.5, "normal", 6, pos_lo=8192, pos_hi=16380, cache="full"),
 }
 
 
