@@ -4,6 +4,9 @@ per-head attention-sink logit.
 TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline / reference leg may import this package. The product
 library never imports it, and it imports nothing from the product package.
+
+``oracle.fp8`` adds the E4M3 code table and encoder and the decode / commit
+over a ring of E4M3 codes with per-kv-head scales (numpy, fp64).
 """
 from .oracle import (  # noqa: F401
     decode,

@@ -13,6 +13,8 @@ throughout this package):
   cu_seqlens [num_seqs + 1] int32 (first entry 0), sink [Hq] fp32.
 * decode: q [B, n_q, Hq, D], k_new/v_new [B, n_q, Hkv, D], ring k/v
   [B, W, Hkv, D] bf16, pos [B] int32, sink [Hq] fp32.
+* decode over an FP8 ring: the ring k/v are uint8 E4M3 codes [B, W, Hkv, D]
+  (drawn through torch's float8_e4m3fn cast) and kv_scale [2 * Hkv] fp32.
 """
 from dataclasses import dataclass, field
 from typing import List, Optional
@@ -51,6 +53,9 @@ class DecodeCase:
     # "ring": a W-slot ring (sliding-window layers); "full": a cache of W >=
     # every context (global layers, split-KV decode with max_ctx = pos_hi)
     cache: str = "ring"
+    # "bf16": the ring holds bf16 K/V; "fp8": E4M3 codes with one fp32 scale
+    # per kv head for K and one for V
+    kv: str = "bf16"
 
 
 # The workloads: a tiny parity case, one SWA layer, one global layer, a packed
@@ -75,6 +80,9 @@ WORKLOADS = {
     "ga_decode_16k": DecodeCase(
         "ga_decode B=16 n_q=4 ctx~U[8192,16380] cache=16384 Hq=64 Hkv=8 D=128", 16, 4,
         64, 8, 128, 16384, 0.5, "normal", 6, pos_lo=8192, pos_hi=16380, cache="full"),
+    "swa_decode_mtp_fp8": DecodeCase(
+        "swa_decode_fp8 B=256 n_q=4 ring=128 e4m3 Hq=64 Hkv=8 D=128", 256, 4, 64, 8,
+        128, 128, 0.5, "normal", 7, kv="fp8"),
 }
 
 
@@ -90,6 +98,19 @@ def _sink(kind, Hq, g):
     if kind == "normal":
         return torch.randn((Hq,), generator=g, dtype=torch.float32)
     raise ValueError(kind)
+
+
+def _fp8_codes(shape, g):
+    """Random E4M3 codes over the format's whole range: N(0, 64^2) draws
+    clamped to the largest finite magnitude, cast by torch."""
+    x = (torch.randn(shape, generator=g) * 64.0).clamp_(-448.0, 448.0)
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def _fp8_scales(Hkv, sigma, g):
+    """fp32 [2 * Hkv] (K scales, then V scales) around sigma / 64, so that the
+    dequantized ring values have about the spread of the bf16 draws."""
+    return (torch.rand((2 * Hkv,), generator=g, dtype=torch.float32) * 1.5 + 0.5) * (sigma / 64.0)
 
 
 def make_prefill(case: PrefillCase):
@@ -121,12 +142,19 @@ def make_decode(case: DecodeCase):
     q = _bf16(torch.randn((case.B, case.n_q, case.Hq, case.D), generator=g) * s)
     k_new = _bf16(torch.randn((case.B, case.n_q, case.Hkv, case.D), generator=g) * s)
     v_new = _bf16(torch.randn((case.B, case.n_q, case.Hkv, case.D), generator=g) * s)
-    k_ring = _bf16(torch.randn((case.B, case.W, case.Hkv, case.D), generator=g) * s)
-    v_ring = _bf16(torch.randn((case.B, case.W, case.Hkv, case.D), generator=g) * s)
+    ring_shape = (case.B, case.W, case.Hkv, case.D)
+    if case.kv == "fp8":
+        k_ring, v_ring = _fp8_codes(ring_shape, g), _fp8_codes(ring_shape, g)
+    else:
+        k_ring = _bf16(torch.randn(ring_shape, generator=g) * s)
+        v_ring = _bf16(torch.randn(ring_shape, generator=g) * s)
     sink = _sink(case.sink, case.Hq, g)
-    return dict(q=q, k_new=k_new, v_new=v_new, k_ring=k_ring, v_ring=v_ring,
-                pos=pos, sink=sink, B=case.B, n_q=case.n_q, Hq=case.Hq,
-                Hkv=case.Hkv, D=case.D, W=case.W)
+    out = dict(q=q, k_new=k_new, v_new=v_new, k_ring=k_ring, v_ring=v_ring,
+               pos=pos, sink=sink, B=case.B, n_q=case.n_q, Hq=case.Hq,
+               Hkv=case.Hkv, D=case.D, W=case.W)
+    if case.kv == "fp8":
+        out["kv_scale"] = _fp8_scales(case.Hkv, s, g)
+    return out
 
 
 def prefill_case(seqlens, Hq, Hkv, D, window, sigma=0.5, sink="normal", seed=0):
@@ -136,9 +164,9 @@ def prefill_case(seqlens, Hq, Hkv, D, window, sigma=0.5, sink="normal", seed=0):
 
 
 def decode_case(B, n_q, Hq, Hkv, D, W, sigma=0.5, sink="normal", seed=0,
-                pos_lo=128, pos_hi=262144):
+                pos_lo=128, pos_hi=262144, kv="bf16"):
     return make_decode(DecodeCase("adhoc", B, n_q, Hq, Hkv, D, W, sigma, sink,
-                                  seed, pos_lo, pos_hi))
+                                  seed, pos_lo, pos_hi, kv=kv))
 
 
 def shard_units(num_units: int, world_size: int, rank: int):
