@@ -55,9 +55,10 @@ def prefill_work(seqlens, Hq, Hkv, D, window):
     return flops, nbytes
 
 
-def decode_work(pos, n_q, Hq, Hkv, D, W):
+def decode_work(pos, n_q, Hq, Hkv, D, W, kv_bytes=2, Hkv_scales=0):
     """FLOPs over visible pairs; bytes = the cached K/V rows of committed
-    tokens (min(pos, W) per sequence) + new K/V + q + pos + sink read once,
+    tokens (min(pos, W) per sequence, kv_bytes per element: 2 for bf16, 1 for
+    E4M3 codes) + new K/V + q + pos + sink (+ the FP8 scales) read once,
     o + lse written once."""
     pairs = 0
     cached = 0
@@ -67,9 +68,15 @@ def decode_work(pos, n_q, Hq, Hkv, D, W):
             pairs += min(P, W - 1 - t) + (t + 1)   # ring keys + new keys 0..t
     B = len(pos)
     flops = 4 * D * Hq * pairs
-    nbytes = (cached * Hkv * D * 2 * 2 + B * n_q * Hkv * D * 2 * 2
-              + B * n_q * Hq * D * 2 * 2 + B * n_q * Hq * 4 + B * 4 + Hq * 4)
+    nbytes = (cached * Hkv * D * kv_bytes * 2 + B * n_q * Hkv * D * 2 * 2
+              + B * n_q * Hq * D * 2 * 2 + B * n_q * Hq * 4 + B * 4 + Hq * 4
+              + Hkv_scales * 2 * 4)
     return flops, nbytes
+
+
+def decode_work_of(d, fp8):
+    return decode_work(d["pos"].tolist(), d["n_q"], d["Hq"], d["Hkv"], d["D"], d["W"],
+                       kv_bytes=1 if fp8 else 2, Hkv_scales=d["Hkv"] if fp8 else 0)
 
 
 def load_peaks():
@@ -89,11 +96,13 @@ KERNEL_SOURCES = {
     "ring": ["prefill_swa_ring_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "chunked": ["prefill_chunked_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "decode": ["decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
+    "decode_fp8": ["decode_fp8_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "splitkv": ["decode_splitkv_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
 }
 WORKLOAD_KERNEL = {"tiny_swa_prefill": "ring", "swa_prefill_32k": "ring",
                    "varlen_swa_prefill": "ring", "global_prefill_8k": "chunked",
-                   "swa_decode_mtp": "decode", "ga_decode_16k": "splitkv"}
+                   "swa_decode_mtp": "decode", "ga_decode_16k": "splitkv",
+                   "swa_decode_mtp_fp8": "decode_fp8"}
 
 
 def kernel_source_hash(workload):
@@ -228,10 +237,12 @@ class DecodeRunner:
         case = wl.DecodeCase(**{**case.__dict__, "seed": case.seed + 1000 * rank})
         d = wl.make_decode(case)
         self.d = d
-        self.flops, self.bytes = decode_work(d["pos"].tolist(), d["n_q"], d["Hq"], d["Hkv"],
-                                             d["D"], d["W"])
+        self.fp8 = case.kv == "fp8"
+        self.flops, self.bytes = decode_work_of(d, self.fp8)
         dev = torch.device("cuda")
         names = ["q", "k_new", "v_new", "k_ring", "v_ring", "pos", "sink"]
+        if self.fp8:
+            names.append("kv_scale")
         self.g = {n: d[n].to(dev) for n in names}
         self.full = case.cache == "full"
         self.max_ctx = case.pos_hi
@@ -255,6 +266,10 @@ class DecodeRunner:
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
         self.units = d["B"]
         self.launches_per_call = 2 if getattr(self, "full", False) else 1
+        if self.NSETS > 1:
+            self.l2_note = ("%d input sets rotated, %.0f MB each, %.0f MB together (> L2): a "
+                            "step's inputs are not L2-resident" %
+                            (self.NSETS, self.bytes / 1e6, self.NSETS * self.bytes / 1e6))
 
     def call(self, stream):
         d, g = self.d, self.sets[self.turn]
@@ -267,6 +282,14 @@ class DecodeRunner:
             if rc != 0:
                 raise RuntimeError("swa_sink_attn_decode_splitkv: %s" % self.B.status_string(rc))
             return
+        if self.fp8:
+            rc = self.B.swa_sink_attn_decode_fp8kv(
+                g["q"], g["k_new"], g["v_new"], g["k_ring"], g["v_ring"], g["kv_scale"],
+                g["pos"], d["B"], d["n_q"], d["Hq"], d["Hkv"], d["D"], d["W"], g["sink"], 0.0,
+                self.o, self.lse, stream)
+            if rc != 0:
+                raise RuntimeError("swa_sink_attn_decode_fp8kv: %s" % self.B.status_string(rc))
+            return
         rc = self.B.swa_sink_attn_decode(g["q"], g["k_new"], g["v_new"], g["k_ring"],
                                          g["v_ring"], g["pos"], d["B"], d["n_q"], d["Hq"],
                                          d["Hkv"], d["D"], d["W"], g["sink"], 0.0, self.o,
@@ -276,8 +299,11 @@ class DecodeRunner:
 
     def describe(self):
         d = self.d
-        return {"batch": d["B"], "n_q": d["n_q"], "Hq": d["Hq"], "Hkv": d["Hkv"],
-                "head_dim": d["D"], ("cache" if self.full else "ring"): d["W"]}
+        out = {"batch": d["B"], "n_q": d["n_q"], "Hq": d["Hq"], "Hkv": d["Hkv"],
+               "head_dim": d["D"], ("cache" if self.full else "ring"): d["W"]}
+        if self.fp8:
+            out["kv_cache"] = "e4m3, one fp32 scale per kv head for K and for V"
+        return out
 
 
 # ------------------------------------------------------------ oracle timing --
@@ -294,7 +320,7 @@ def _cached_inputs(workload, wl):
 
 def oracle_sample(workload, wl, seconds, threads, seed=0):
     """Time the fp64 oracle on a bounded sample of the workload. Returns
-    (flops_done, bytes_equiv, elapsed_s, description)."""
+    (flops_done, bytes_equiv, elapsed_s, description, threads used)."""
     import numpy as np
     import oracle
     case = wl.WORKLOADS[workload]
@@ -314,17 +340,28 @@ def oracle_sample(workload, wl, seconds, threads, seed=0):
         unit = "random (token, head) rows"
     else:
         d = _cached_inputs(workload, wl)
-        F, Bt = decode_work(d["pos"].tolist(), d["n_q"], d["Hq"], d["Hkv"], d["D"], d["W"])
+        fp8 = case.kv == "fp8"
+        F, Bt = decode_work_of(d, fp8)
         total_rows = d["B"]
+        if fp8:
+            from oracle import fp8 as ofp8
+            threads = 1  # numpy, one thread
 
         def run(n):
             idx = np.sort(rng.choice(d["B"], size=min(n, d["B"]), replace=False))
             sub = {k: (d[k][idx] if k in ("q", "k_new", "v_new", "k_ring", "v_ring", "pos")
                        else d[k]) for k in d}
             t0 = time.perf_counter()
-            oracle.decode(sub["q"], sub["k_new"], sub["v_new"], sub["k_ring"], sub["v_ring"],
-                          sub["pos"], len(idx), d["n_q"], d["Hq"], d["Hkv"], d["D"], d["W"],
-                          sink=d["sink"], nthreads=threads)
+            if fp8:
+                f64 = lambda t: t.double().numpy()  # noqa: E731
+                ofp8.decode_fp8(f64(sub["q"]), f64(sub["k_new"]), f64(sub["v_new"]),
+                                sub["k_ring"].numpy(), sub["v_ring"].numpy(),
+                                d["kv_scale"].numpy(), sub["pos"].numpy(), len(idx), d["n_q"],
+                                d["Hq"], d["Hkv"], d["D"], d["W"], sink=d["sink"].numpy())
+            else:
+                oracle.decode(sub["q"], sub["k_new"], sub["v_new"], sub["k_ring"],
+                              sub["v_ring"], sub["pos"], len(idx), d["n_q"], d["Hq"], d["Hkv"],
+                              d["D"], d["W"], sink=d["sink"], nthreads=threads)
             return time.perf_counter() - t0
         unit = "sequences"
     # calibrate on a small sample, then size the timed sample to `seconds`
@@ -334,7 +371,7 @@ def oracle_sample(workload, wl, seconds, threads, seed=0):
     elapsed = run(n)
     frac = n / total_rows
     return F * frac, Bt * frac, elapsed, "%d of %d %s of %s, %d threads" % (
-        n, total_rows, unit, workload, threads)
+        n, total_rows, unit, workload, threads), threads
 
 
 def run_reference(args, wl):
@@ -354,7 +391,8 @@ def run_reference(args, wl):
     flops = nb = el = 0.0
     desc = ""
     for s in range(args.steps):
-        f, b, e, desc = oracle_sample(args.workload, wl, per_step, threads, seed=s + 1)
+        f, b, e, desc, threads_used = oracle_sample(args.workload, wl, per_step, threads,
+                                                    seed=s + 1)
         flops += f
         nb += b
         el += e
@@ -366,7 +404,7 @@ def run_reference(args, wl):
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": case.name, "impl_note": "fp64 CPU oracle, bounded samples"},
-        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads_used, "kind": "oracle",
                          "sample": desc + " per step"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -443,7 +481,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         threads = oracle.default_threads()
-        f, b, e, desc = oracle_sample(args.workload, wl, args.cpu_seconds, threads)
+        f, b, e, desc, threads = oracle_sample(args.workload, wl, args.cpu_seconds, threads)
         cpu = {"value": (f / e / 1e12) if is_prefill else (b / e / 1e9),
                "unit": "TFLOP/s" if is_prefill else "GB/s", "cores": threads,
                "kind": "oracle", "sample": desc + ", %.1f s" % e}
@@ -556,8 +594,9 @@ def main():
             "dtype": "bf16", "data": "synthetic",
             "config": dict({"workload": case.name,
                             "parallelism": "replicas" if world == 1 else "dp%d" % world,
-                            "l2": ("inputs larger than L2 (%.0f MB per step)" %
-                                   (runner.bytes / 1e6))},
+                            "l2": getattr(runner, "l2_note", None) or (
+                                "inputs larger than L2 (%.0f MB per step)" %
+                                (runner.bytes / 1e6))},
                            **runner.describe()),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * runner.launches_per_call, "clocks": clk.summary(), "device_error_flags": flag,

@@ -222,6 +222,44 @@ SWA_API int swa_sink_kv_commit(void *k_ring, void *v_ring, const void *k_new,
                        const int32_t *n_accept, int B, int n_q, int Hkv, int D,
                        int W, void *stream);
 
+/*
+ * Decode / draft verification and commit over an FP8 (E4M3) ring.
+ *
+ * Source: the KV cache of these models is sized as an FP8 cache (MiMo-V3 /
+ * HySparse2 news page, hao.cnyes.com, cost comparison at one million tokens),
+ * and inference runs in FP8 with the E4M3 format (MiMo-V2 blog review,
+ * kokolerk.github.io, sections 4.3 and 6). No page fixes the scale
+ * granularity; here it is one fp32 scale per kv head for K and one for V.
+ *
+ * The ring holds E4M3 codes (OCP E4M3FN: bias 7, no infinities, 0x7F / 0xFF
+ * NaN, largest finite 448): the ring value of code c of kv head g is
+ * value(c) * kv_scale[g] for K and value(c) * kv_scale[Hkv + g] for V. The
+ * decode is then exactly swa_sink_attn_decode over those values (positions,
+ * visibility, sink and outputs as there; the new tokens stay bf16).
+ *
+ *   k_ring, v_ring  uint8 E4M3 codes [B, W, Hkv, D], 16-byte aligned
+ *   kv_scale        fp32 [2 * Hkv] device: K scales, then V scales; each
+ *                   must be finite and > 0 (else flagged: bit 1 of
+ *                   swa_sink_device_error, results undefined)
+ *   the other arguments and limits as for swa_sink_attn_decode.
+ *
+ * swa_sink_kv_commit_fp8 writes accepted new token u (u < n_accept[b]) into
+ * slot (pos[b]+u) mod W as the E4M3 codes of x / scale: the quotient rounded
+ * to fp32 (IEEE division), then to the nearest E4M3 value (ties to even),
+ * magnitudes beyond 448 saturated to 448 (NaN stays NaN). n_accept and pos
+ * as for swa_sink_kv_commit.
+ */
+SWA_API int swa_sink_attn_decode_fp8kv(const void *q, const void *k_new, const void *v_new,
+                                       const void *k_ring, const void *v_ring,
+                                       const float *kv_scale, const int32_t *pos, int B,
+                                       int n_q, int Hq, int Hkv, int D, int W,
+                                       const float *sink, float softmax_scale, void *o,
+                                       float *lse, void *stream);
+SWA_API int swa_sink_kv_commit_fp8(void *k_ring, void *v_ring, const void *k_new,
+                                   const void *v_new, const float *kv_scale,
+                                   const int32_t *pos, const int32_t *n_accept, int B,
+                                   int n_q, int Hkv, int D, int W, void *stream);
+
 /* Human-readable text for a swa_status_t (static storage). */
 SWA_API const char *swa_sink_status_string(int status);
 

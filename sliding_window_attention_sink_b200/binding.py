@@ -57,6 +57,12 @@ def load():
                                                  ctypes.c_size_t, _vp]
     lib.swa_sink_kv_commit.restype = _i
     lib.swa_sink_kv_commit.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+    lib.swa_sink_attn_decode_fp8kv.restype = _i
+    lib.swa_sink_attn_decode_fp8kv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i,
+                                               _i, _i, _i, _vp, _f, _vp, _vp, _vp]
+    lib.swa_sink_kv_commit_fp8.restype = _i
+    lib.swa_sink_kv_commit_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                           _i, _vp]
     lib.swa_sink_status_string.restype = ctypes.c_char_p
     lib.swa_sink_status_string.argtypes = [_i]
     lib.swa_sink_device_error.restype = _i
@@ -133,6 +139,21 @@ def swa_sink_kv_commit(k_ring, v_ring, k_new, v_new, pos, n_accept, B, n_q, Hkv,
     return load().swa_sink_kv_commit(
         _ptr(k_ring), _ptr(v_ring), _ptr(k_new), _ptr(v_new), _ptr(pos), _ptr(n_accept),
         int(B), int(n_q), int(Hkv), int(D), int(W), _stream(stream))
+
+
+def swa_sink_attn_decode_fp8kv(q, k_new, v_new, k_ring, v_ring, kv_scale, pos, B, n_q, Hq, Hkv,
+                               D, W, sink, softmax_scale, o, lse, stream=None):
+    return load().swa_sink_attn_decode_fp8kv(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring), _ptr(v_ring), _ptr(kv_scale),
+        _ptr(pos), int(B), int(n_q), int(Hq), int(Hkv), int(D), int(W), _ptr(sink),
+        float(softmax_scale), _ptr(o), _ptr(lse), _stream(stream))
+
+
+def swa_sink_kv_commit_fp8(k_ring, v_ring, k_new, v_new, kv_scale, pos, n_accept, B, n_q, Hkv,
+                           D, W, stream=None):
+    return load().swa_sink_kv_commit_fp8(
+        _ptr(k_ring), _ptr(v_ring), _ptr(k_new), _ptr(v_new), _ptr(kv_scale), _ptr(pos),
+        _ptr(n_accept), int(B), int(n_q), int(Hkv), int(D), int(W), _stream(stream))
 
 
 def swa_sink_status_string(status):
@@ -221,3 +242,30 @@ def kv_commit(k_ring, v_ring, k_new, v_new, pos, n_accept, stream=None):
                             stream)
     if rc != SWA_OK:
         raise SwaSinkError(rc, "swa_sink_kv_commit")
+
+
+def attn_decode_fp8kv(q, k_new, v_new, k_ring, v_ring, kv_scale, pos, sink=None,
+                      softmax_scale=0.0, out=None, lse=None, want_lse=True, stream=None):
+    """attn_decode over an E4M3 ring: k_ring / v_ring uint8 codes [B,W,Hkv,D],
+    kv_scale fp32 [2*Hkv] (K scales, then V scales)."""
+    B, n_q, Hq, D = q.shape
+    Hkv = k_new.shape[2]
+    W = k_ring.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n_q, Hq), dtype=torch.float32, device=q.device)
+    rc = swa_sink_attn_decode_fp8kv(q, k_new, v_new, k_ring, v_ring, kv_scale, pos, B, n_q, Hq,
+                                    Hkv, D, W, sink, softmax_scale, out, lse, stream)
+    if rc != SWA_OK:
+        raise SwaSinkError(rc, "swa_sink_attn_decode_fp8kv")
+    return out, lse
+
+
+def kv_commit_fp8(k_ring, v_ring, k_new, v_new, kv_scale, pos, n_accept, stream=None):
+    B, W, Hkv, D = k_ring.shape
+    n_q = k_new.shape[1]
+    rc = swa_sink_kv_commit_fp8(k_ring, v_ring, k_new, v_new, kv_scale, pos, n_accept, B, n_q,
+                                Hkv, D, W, stream)
+    if rc != SWA_OK:
+        raise SwaSinkError(rc, "swa_sink_kv_commit_fp8")

@@ -18,6 +18,7 @@
 #include <mutex>
 
 #include "../../include/swa_sink.h"
+#include "decode_fp8_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "decode_splitkv_sm100.cuh"
 #include "prefill_chunked_sm100.cuh"
@@ -80,6 +81,24 @@ int encode_4d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint6
   return r == CUDA_SUCCESS ? SWA_OK : cuda_fail("cuTensorMapEncodeTiled", static_cast<int>(r));
 }
 
+// 4-D byte tensor [d3][d2][d1][d0] (E4M3 codes, d0 contiguous), boxes of b0
+// bytes inner: the 128-byte swizzle for 128-byte rows, the 64-byte one for
+// 64-byte rows.
+int encode_u8_4d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+                 uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  auto fn = get_encode_fn();
+  if (!fn) return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", 0);
+  cuuint64_t dims[4] = {d0, d1, d2, d3};
+  cuuint64_t strides[3] = {d0, d0 * d1, d0 * d1 * d2};
+  cuuint32_t box[4] = {b0, b1, b2, b3};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  b0 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SWA_OK : cuda_fail("cuTensorMapEncodeTiled", static_cast<int>(r));
+}
+
 // With SWA_SINK_DEBUG set in the environment, failing CUDA calls are named
 // on stderr (the status code alone says only SWA_ERR_CUDA).
 int cuda_fail(const char* what, int err) {
@@ -108,7 +127,7 @@ int ensure_smem_attr(K kernel, size_t bytes, size_t (&done)[kMaxDevices]) {
 }
 
 size_t g_attr_prefill64[kMaxDevices], g_attr_prefill128[kMaxDevices];
-size_t g_attr_dec[2][2][2][kMaxDevices];
+size_t g_attr_dec[2][2][2][2][kMaxDevices];
 
 int next_pow2(int x) {
   int p = 32;
@@ -390,29 +409,104 @@ int launch_prefill(const void* q, const void* k, const void* v, const int32_t* c
   return e == cudaSuccess ? SWA_OK : cuda_fail("prefill launch", e);
 }
 
-template <int D, int MT, int NWP>
-int launch_decode(const swa::DecodeParams& p, cudaStream_t st) {
+template <int D, int MT, int NWP, bool KV8>
+int launch_decode(const swa::DecodeFp8Params& p, cudaStream_t st) {
   // boxes of 64 head-dim columns: Q [G heads x n_q tokens], ring [W rows],
-  // new rows [n_q rows], of one (sequence, kv head)
+  // new rows [n_q rows], of one (sequence, kv head); an FP8 ring as one box
+  // of W rows x D codes
   CUtensorMap tq, tkr, tkn, tvr, tvn, to;
   const uint32_t G = static_cast<uint32_t>(p.G), nq = static_cast<uint32_t>(p.n_q);
   const uint32_t W = static_cast<uint32_t>(p.W);
-  if (encode_4d(&tq, p.q, D, p.Hq, p.n_q, p.B, 64, G, nq, 1) != SWA_OK ||
-      encode_4d(&tkr, p.k_ring, D, p.Hkv, p.W, p.B, 64, 1, W, 1) != SWA_OK ||
+  const bool ring_ok =
+      KV8 ? (encode_u8_4d(&tkr, p.k_ring, D, p.Hkv, p.W, p.B, D, 1, W, 1) == SWA_OK &&
+             encode_u8_4d(&tvr, p.v_ring, D, p.Hkv, p.W, p.B, D, 1, W, 1) == SWA_OK)
+          : (encode_4d(&tkr, p.k_ring, D, p.Hkv, p.W, p.B, 64, 1, W, 1) == SWA_OK &&
+             encode_4d(&tvr, p.v_ring, D, p.Hkv, p.W, p.B, 64, 1, W, 1) == SWA_OK);
+  if (!ring_ok || encode_4d(&tq, p.q, D, p.Hq, p.n_q, p.B, 64, G, nq, 1) != SWA_OK ||
       encode_4d(&tkn, p.k_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK ||
-      encode_4d(&tvr, p.v_ring, D, p.Hkv, p.W, p.B, 64, 1, W, 1) != SWA_OK ||
       encode_4d(&tvn, p.v_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK ||
       encode_4d(&to, p.o, D, p.Hq, p.n_q, p.B, 64, G, nq, 1) != SWA_OK)
     return SWA_ERR_CUDA;
-  const size_t smem = swa::decode_smem_bytes(D, p.KP, NWP);
-  auto kern = swa::decode_sm100_kernel<D, MT, NWP>;
-  if (ensure_smem_attr(kern, smem,
-                       g_attr_dec[D == 128][MT - 1][NWP == swa::kDecodeLargeWarps]) != SWA_OK)
-    return SWA_ERR_CUDA;
-  kern<<<static_cast<unsigned>(p.B) * p.Hkv, NWP * 32, smem, st>>>(tq, tkr, tkn, tvr, tvn, to,
-                                                                    p);
+  const unsigned grid = static_cast<unsigned>(p.B) * p.Hkv;
+  auto& attr = g_attr_dec[KV8][D == 128][MT - 1][NWP == swa::kDecodeLargeWarps];
+  if constexpr (KV8) {
+    const size_t smem = swa::decode_fp8_smem_bytes(D, p.KP, p.W8, NWP);
+    auto kern = swa::decode_fp8_sm100_kernel<D, MT, NWP>;
+    if (ensure_smem_attr(kern, smem, attr) != SWA_OK)
+      return SWA_ERR_CUDA;
+    kern<<<grid, NWP * 32, smem, st>>>(tq, tkr, tkn, tvr, tvn, to, p);
+  } else {  // the bf16 ring (the kernel takes the DecodeParams part)
+    const size_t smem = swa::decode_smem_bytes(D, p.KP, NWP);
+    auto kern = swa::decode_sm100_kernel<D, MT, NWP>;
+    if (ensure_smem_attr(kern, smem, attr) != SWA_OK)
+      return SWA_ERR_CUDA;
+    kern<<<grid, NWP * 32, smem, st>>>(tq, tkr, tkn, tvr, tvn, to, p);
+  }
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SWA_OK : cuda_fail("decode launch", e);
+}
+
+template <bool KV8>
+int pick_decode(const swa::DecodeFp8Params& p, int D, cudaStream_t st) {
+  const bool two = p.R > 16;
+  if (p.KP <= swa::kDecodeSmallMaxKP) {
+    constexpr int S = swa::kDecodeSmallWarps;
+    if (D == 64)
+      return two ? launch_decode<64, 2, S, KV8>(p, st) : launch_decode<64, 1, S, KV8>(p, st);
+    return two ? launch_decode<128, 2, S, KV8>(p, st) : launch_decode<128, 1, S, KV8>(p, st);
+  }
+  constexpr int L = swa::kDecodeLargeWarps;
+  if (D == 64)
+    return two ? launch_decode<64, 2, L, KV8>(p, st) : launch_decode<64, 1, L, KV8>(p, st);
+  return two ? launch_decode<128, 2, L, KV8>(p, st) : launch_decode<128, 1, L, KV8>(p, st);
+}
+
+// swa_sink_attn_decode (kv_scale NULL: bf16 ring) and
+// swa_sink_attn_decode_fp8kv (E4M3 ring with per-kv-head scales).
+int decode_impl(const void* q, const void* k_new, const void* v_new, const void* k_ring,
+                const void* v_ring, const float* kv_scale, const int32_t* pos, int B, int n_q,
+                int Hq, int Hkv, int D, int W, const float* sink, float softmax_scale, void* o,
+                float* lse, void* stream) {
+  if (B < 0 || n_q <= 0 || Hq <= 0 || Hkv <= 0 || W <= 0) return SWA_ERR_SHAPE;
+  if (Hq % Hkv != 0) return SWA_ERR_SHAPE;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (n_q > 8 || W > 256 || n_q * (Hq / Hkv) > 32) return SWA_ERR_UNSUPPORTED;
+  if (B == 0) return SWA_OK;
+  if (!q || !k_new || !v_new || !k_ring || !v_ring || !pos || !o) return SWA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_ring) ||
+      !aligned16(v_ring) || !aligned16(o))
+    return SWA_ERR_ALIGN;
+  if (!aligned4(pos) || (sink && !aligned4(sink)) || (lse && !aligned4(lse)) ||
+      (kv_scale && !aligned4(kv_scale)))
+    return SWA_ERR_ALIGN;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
+  swa::DecodeFp8Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.k_ring = static_cast<const __nv_bfloat16*>(k_ring);
+  p.v_ring = static_cast<const __nv_bfloat16*>(v_ring);
+  p.kv_scale = kv_scale;
+  p.pos = pos;
+  p.B = B;
+  p.n_q = n_q;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.W = W;
+  p.R = n_q * p.G;
+  // the new tokens' columns start at a multiple of 8 (16 for an FP8 ring,
+  // whose kernel gives them a 16-key block of their own)
+  p.W8 = round_up(W, kv_scale ? 16 : 8);
+  p.KP = round_up(p.W8 + n_q, 16);
+  p.sink = sink;
+  p.scale_log2 = softmax_scale * swa::kLog2e;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  if (static_cast<long long>(B) * Hkv > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return kv_scale ? pick_decode<true>(p, D, st) : pick_decode<false>(p, D, st);
 }
 
 // swa_sink_attn_fwd and swa_sink_attn_fwd_noalloc: validation and kernel
@@ -553,49 +647,18 @@ int swa_sink_attn_decode(const void* q, const void* k_new, const void* v_new, co
                          const void* v_ring, const int32_t* pos, int B, int n_q, int Hq, int Hkv,
                          int D, int W, const float* sink, float softmax_scale, void* o,
                          float* lse, void* stream) {
-  if (B < 0 || n_q <= 0 || Hq <= 0 || Hkv <= 0 || W <= 0) return SWA_ERR_SHAPE;
-  if (Hq % Hkv != 0) return SWA_ERR_SHAPE;
-  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
-  if (n_q > 8 || W > 256 || n_q * (Hq / Hkv) > 32) return SWA_ERR_UNSUPPORTED;
-  if (B == 0) return SWA_OK;
-  if (!q || !k_new || !v_new || !k_ring || !v_ring || !pos || !o) return SWA_ERR_NULL;
-  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_ring) ||
-      !aligned16(v_ring) || !aligned16(o))
-    return SWA_ERR_ALIGN;
-  if (!aligned4(pos) || (sink && !aligned4(sink)) || (lse && !aligned4(lse))) return SWA_ERR_ALIGN;
-  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-    softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
-  swa::DecodeParams p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
-  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
-  p.k_ring = static_cast<const __nv_bfloat16*>(k_ring);
-  p.v_ring = static_cast<const __nv_bfloat16*>(v_ring);
-  p.pos = pos;
-  p.B = B;
-  p.n_q = n_q;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.W = W;
-  p.R = n_q * p.G;
-  p.W8 = round_up(W, 8);
-  p.KP = round_up(p.W8 + n_q, 16);
-  p.sink = sink;
-  p.scale_log2 = softmax_scale * swa::kLog2e;
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  if (static_cast<long long>(B) * Hkv > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool two = p.R > 16;
-  if (p.KP <= swa::kDecodeSmallMaxKP) {
-    constexpr int S = swa::kDecodeSmallWarps;
-    if (D == 64) return two ? launch_decode<64, 2, S>(p, st) : launch_decode<64, 1, S>(p, st);
-    return two ? launch_decode<128, 2, S>(p, st) : launch_decode<128, 1, S>(p, st);
-  }
-  constexpr int L = swa::kDecodeLargeWarps;
-  if (D == 64) return two ? launch_decode<64, 2, L>(p, st) : launch_decode<64, 1, L>(p, st);
-  return two ? launch_decode<128, 2, L>(p, st) : launch_decode<128, 1, L>(p, st);
+  return decode_impl(q, k_new, v_new, k_ring, v_ring, nullptr, pos, B, n_q, Hq, Hkv, D, W, sink,
+                     softmax_scale, o, lse, stream);
+}
+
+int swa_sink_attn_decode_fp8kv(const void* q, const void* k_new, const void* v_new,
+                               const void* k_ring, const void* v_ring, const float* kv_scale,
+                               const int32_t* pos, int B, int n_q, int Hq, int Hkv, int D, int W,
+                               const float* sink, float softmax_scale, void* o, float* lse,
+                               void* stream) {
+  if (B > 0 && !kv_scale) return SWA_ERR_NULL;
+  return decode_impl(q, k_new, v_new, k_ring, v_ring, kv_scale, pos, B, n_q, Hq, Hkv, D, W,
+                     sink, softmax_scale, o, lse, stream);
 }
 
 size_t swa_sink_decode_splitkv_workspace(int B, int n_q, int Hq, int Hkv, int D, int W,
@@ -666,6 +729,27 @@ int swa_sink_kv_commit(void* k_ring, void* v_ring, const void* k_new, const void
       static_cast<__nv_bfloat16*>(k_ring), static_cast<__nv_bfloat16*>(v_ring),
       static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), pos,
       n_accept, n_q, Hkv, D, W);
+  return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int swa_sink_kv_commit_fp8(void* k_ring, void* v_ring, const void* k_new, const void* v_new,
+                           const float* kv_scale, const int32_t* pos, const int32_t* n_accept,
+                           int B, int n_q, int Hkv, int D, int W, void* stream) {
+  if (B < 0 || n_q <= 0 || Hkv <= 0 || W <= 0) return SWA_ERR_SHAPE;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (B == 0) return SWA_OK;
+  if (!k_ring || !v_ring || !k_new || !v_new || !kv_scale || !pos || !n_accept)
+    return SWA_ERR_NULL;
+  if (!aligned16(k_ring) || !aligned16(v_ring) || !aligned16(k_new) || !aligned16(v_new))
+    return SWA_ERR_ALIGN;
+  if (!aligned4(kv_scale) || !aligned4(pos) || !aligned4(n_accept)) return SWA_ERR_ALIGN;
+  const long long grid = static_cast<long long>(B) * n_q;
+  if (grid > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  swa::kv_commit_fp8_kernel<<<static_cast<unsigned>(grid), 128, 0, st>>>(
+      static_cast<uint8_t*>(k_ring), static_cast<uint8_t*>(v_ring),
+      static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
+      kv_scale, pos, n_accept, n_q, Hkv, D, W);
   return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 

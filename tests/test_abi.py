@@ -134,3 +134,26 @@ def test_splitkv_workspace_and_argument_errors():
     assert f(**dict(a, n_q=9)) == -3
     assert f(**dict(a, Hq=64, Hkv=6)) == -2
     assert f(**dict(a, B=0)) == 0
+
+
+def test_fp8_decode_and_commit_argument_errors():
+    a = dict(q=FAKE, k_new=FAKE, v_new=FAKE, k_ring=FAKE, v_ring=FAKE, kv_scale=FAKE, pos=FAKE,
+             B=4, n_q=4, Hq=64, Hkv=8, D=128, W=128, sink=None, softmax_scale=0.0, o=FAKE,
+             lse=None, stream=0)
+    f = B.swa_sink_attn_decode_fp8kv
+    assert f(**dict(a, kv_scale=None)) == -1
+    assert f(**dict(a, kv_scale=FAKE + 2)) == -4
+    assert f(**dict(a, k_ring=FAKE + 8)) == -4
+    assert f(**dict(a, W=257)) == -3
+    assert f(**dict(a, D=96)) == -3
+    assert f(**dict(a, n_q=0)) == -2
+    assert f(**dict(a, B=0, kv_scale=None)) == 0
+    c = dict(k_ring=FAKE, v_ring=FAKE, k_new=FAKE, v_new=FAKE, kv_scale=FAKE, pos=FAKE,
+             n_accept=FAKE, B=2, n_q=4, Hkv=8, D=128, W=128, stream=0)
+    g = B.swa_sink_kv_commit_fp8
+    assert g(**dict(c, kv_scale=None)) == -1
+    assert g(**dict(c, kv_scale=FAKE + 1)) == -4
+    assert g(**dict(c, v_ring=FAKE + 8)) == -4
+    assert g(**dict(c, D=32)) == -3
+    assert g(**dict(c, W=0)) == -2
+    assert g(**dict(c, B=0)) == 0
