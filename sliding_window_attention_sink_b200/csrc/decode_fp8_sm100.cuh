@@ -27,23 +27,24 @@
 //   fragments are loaded.
 // * S = Q K^T: the order of the 16 head-dim columns of each k-step is
 //   permuted alike in Q and K (logical 2c, 2c+1, 2c+8, 2c+9 <-> stored
-//   4c .. 4c+3), so one 32-bit load of 4 codes gives a thread both of its K
-//   fragment registers, and one 64-bit load of Q gives two A registers.
-// * O = P V: a thread loads 4 codes of one key row (stored head-dim columns
-//   4c .. 4c+3 of a 16-column group), converts them to two bf16 pairs and
-//   movmatrix-transposes each 8x8 tile into the B fragment. The two tiles of
-//   a group hold the stored columns {4c, 4c+1} and {4c+2, 4c+3}, which the
-//   epilogue writes back in place.
+//   4c .. 4c+3). An ldmatrix over the code tile hands each thread 4
+//   consecutive codes of one key row per 8x8 (16-bit) matrix, i.e. both of
+//   its K fragment registers; one ldmatrix.x4 covers four k-steps. Q is
+//   stored reordered (in its f16 conversion) so that plain ldmatrix A
+//   fragments come out in the same order.
+// * O = P V: an ldmatrix over the V code tile gives a thread 4 codes of one
+//   key row (stored head-dim columns 4c .. 4c+3 of a 16-column group); they
+//   become two f16 pairs, and movmatrix transposes each 8x8 tile into the B
+//   fragment. The two tiles of a group hold the stored columns {4c, 4c+1}
+//   and {4c+2, 4c+3}, which the epilogue writes back in place.
 // * K's scale multiplies the logits of the ring columns. V's scale is applied
 //   in fp32: the new tokens (a 16-key block of their own: the ring's columns
 //   are padded to a multiple of 16) are accumulated first, the accumulator
 //   is divided by the scale, the ring's blocks follow, and O is multiplied by
 //   the scale at the end.
-// * Never-written slots (pos < W) and the padding rows read as zero codes
-//   (a predicated load), so NaN bytes there cannot reach O.
+// * The V rows of never-written slots (pos < W) and of the padding are set
+//   to zero codes in shared memory, so NaN bytes there cannot reach O.
 #pragma once
-#include <cuda_fp16.h>
-
 #include "decode_sm100.cuh"
 
 namespace swa {
@@ -57,11 +58,11 @@ __host__ __device__ inline size_t round1024(size_t x) { return (x + 1023) / 1024
 // Shared memory (from a 1024-byte aligned base): Q [D/64][32 rows][128 B]
 // (later P [32][KP+8] bf16, then the O staging tile); the K and V code tiles
 // [W8 rows][D bytes] (swizzled); the new K and V rows [D/64][16 rows][128 B];
-// per-warp row maxima and the two row sums [NWP][32] and row l [32] (fp32).
+// per-warp row maxima and row sums [NWP][32] and row l [32] (fp32).
 __host__ __device__ inline size_t decode_fp8_smem_bytes(int D, int KP, int W8, int nwp) {
   return 1024 + round1024(decode_qp_bytes(D, KP)) + 2 * round1024(static_cast<size_t>(W8) * D) +
          2 * static_cast<size_t>(D / 64) * 2048 +
-         (static_cast<size_t>(nwp) * 32 * 3 + 32) * sizeof(float);
+         (static_cast<size_t>(nwp) * 32 * 2 + 32) * sizeof(float);
 }
 
 // Byte address of (row, byte) in a code tile of D-byte rows written by TMA
@@ -91,24 +92,24 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
       : "f"(bf16hi_to_f32(x)), "f"(bf16lo_to_f32(x)));
   return r;
 }
+// bf16 pair x s -> f16 pair (round to nearest; beyond 65504 saturated).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t x, float s) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;"
+      : "=r"(r)
+      : "f"(bf16hi_to_f32(x) * s), "f"(bf16lo_to_f32(x) * s));
+  return r;
+}
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-__device__ __forceinline__ float f16x2_sum(uint32_t x) {
-  const __half2 h = *reinterpret_cast<const __half2*>(&x);
-  const float2 f = __half22float2(h);
-  return f.x + f.y;
-}
 
-// Shared-memory reads as plain loads (not asm), so that the compiler may
-// schedule them ahead of the conversions and MMAs of earlier tiles; the
-// barrier waits (asm with a memory clobber) keep them after the data lands.
+// A shared-memory read as a plain load (not asm), so that the compiler may
+// schedule it ahead of the conversions and MMAs of earlier tiles; the
+// barrier waits (asm with a memory clobber) keep it after the data lands.
 // (smem: the dynamic shared array; addr: a shared-window address in it)
-__device__ __forceinline__ uint32_t lds32(const uint8_t* smem, uint32_t addr) {
-  return *reinterpret_cast<const uint32_t*>(smem + (addr - smem_u32(smem)));
-}
 __device__ __forceinline__ void lds64(const uint8_t* smem, uint32_t addr, uint32_t& lo,
                                       uint32_t& hi) {
   const uint2 v = *reinterpret_cast<const uint2*>(smem + (addr - smem_u32(smem)));
@@ -165,8 +166,7 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
   __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(smem_raw + (sQ - smem_u32(smem_raw)));
   const int LDP = KP + 8;
   float* red_max = reinterpret_cast<float*>(smem_raw + (sVn + NCH * 2048 - smem_u32(smem_raw)));
-  float* red_lr = red_max + NWP * 32;  // [NWP][32]
-  float* red_lx = red_lr + NWP * 32;   // [NWP][32]
+  float* red_lx = red_max + NWP * 32;  // [NWP][32]
   float* row_l = red_lx + NWP * 32;    // [32]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -262,7 +262,11 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
   __syncthreads();
 
   // ---- S = Q K^T: warp w takes key tiles w, w + NWP, ... ----------------------
-  const int NT = KP / 8;
+  // Tiles at or past NTS hold padding only: no S, and P = 0 there. The new
+  // keys are divided by K's scale as they are converted, so that every
+  // column's logit is S x sc_ring.
+  const int NT = KP / 8, NTS = (W8 + n_q + 7) / 8;
+  const float k_inv = 1.f / k_sc;
   float s[MT][NTW][4];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
@@ -288,7 +292,7 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
 #pragma unroll
     for (int j = 0; j < NTW; ++j) {
       const int nt = warp + NWP * j;
-      if (nt < NT) {
+      if (nt < NTS) {
         uint32_t b[4][2];
         if (nt * 8 < W8) {  // ring keys: codes
           uint32_t w[4];
@@ -301,8 +305,8 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
           for (int i = 0; i < 4; ++i) {
             lds64(sm, bf16_addr(sKn, 16, nt * 8 - W8 + gq, (kq * 4 + i) * 16 + 4 * c4), b[i][0],
                   b[i][1]);
-            b[i][0] = bf16x2_to_f16x2(b[i][0]);
-            b[i][1] = bf16x2_to_f16x2(b[i][1]);
+            b[i][0] = bf16x2_to_f16x2_scaled(b[i][0], k_inv);
+            b[i][1] = bf16x2_to_f16x2_scaled(b[i][1], k_inv);
           }
         }
 #pragma unroll
@@ -315,36 +319,51 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
     }
   }
 
-  // ---- mask, scale to log2 units, per-warp row max --------------------------
+  // ---- mask (raw logits) and per-warp row max -------------------------------
+  // The scale sc_ring > 0 goes into the exponent below. A ring tile whose
+  // slots all have rank >= thr = max(n_q, W - P) is seen whole by every query
+  // row (query t hides ranks < max(t + 1, W - P)): a warp vote skips its mask.
+  const int thr = max(n_q, W - P);
   float mloc[MT][2];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) mloc[mt][0] = mloc[mt][1] = -INFINITY;
 #pragma unroll
   for (int j = 0; j < NTW; ++j) {
     const int nt = warp + NWP * j;
+    if (nt >= NTS) continue;  // warp-uniform
+    int rank[2];
+    bool hidden = false;
 #pragma unroll
     for (int e2 = 0; e2 < 2; ++e2) {
       const int col = nt * 8 + 2 * c4 + e2;
-      int rank = 0x3fffffff;  // padding: seen by no query
-      if (nt < NT) {
-        if (col < W) {
-          rank = col - Pmod;
-          if (rank < 0) rank += W;
-        } else if (col >= W8 && col < W8 + n_q) {
-          rank = W + (col - W8);
-        }
+      rank[e2] = 0x3fffffff;  // padding: seen by no query
+      if (col < W) {
+        rank[e2] = col - Pmod;
+        if (rank[e2] < 0) rank[e2] += W;
+      } else if (col >= W8 && col < W8 + n_q) {
+        rank[e2] = W + (col - W8);
       }
-      const float csc = col < W ? sc_ring : p.scale_log2;
+      hidden |= rank[e2] < thr || rank[e2] >= W;
+    }
+    if (!__any_sync(0xffffffffu, hidden)) {
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+          mloc[mt][hf] = max3(mloc[mt][hf], s[mt][j][hf * 2], s[mt][j][hf * 2 + 1]);
+      continue;
+    }
+#pragma unroll
+    for (int e2 = 0; e2 < 2; ++e2)
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-          const bool vis = static_cast<unsigned>(rank - rlo[mt][hf]) <= rspan[mt][hf];
+          const bool vis = static_cast<unsigned>(rank[e2] - rlo[mt][hf]) <= rspan[mt][hf];
           float& x = s[mt][j][hf * 2 + e2];
-          x = vis ? x * csc : -INFINITY;
+          x = vis ? x : -INFINITY;
           mloc[mt][hf] = fmaxf(mloc[mt][hf], x);
         }
-    }
   }
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
@@ -357,23 +376,26 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
     }
   __syncthreads();
 
-  // ---- row max over warps and the sink; P = exp2(x - m) -> smem; row sums --
+  // ---- row max over warps and the sink (log2 units); P = exp2(x sc - m) ->
+  // smem (f16); row sums of the unrounded P (f16 P is close enough that O
+  // needs no sum of the rounded weights) ------------------------------------
   float mrow[MT][2];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const int row = mt * 16 + gq + hf * 8;
-      float m = srow[mt][hf];
+      float m = -INFINITY;
 #pragma unroll
       for (int w = 0; w < NWP; ++w) m = fmaxf(m, red_max[w * 32 + row]);
+      m = fmaxf(srow[mt][hf], m * sc_ring);
       mrow[mt][hf] = (m == -INFINITY) ? 0.f : m;
     }
-  float lr[MT][2], lx[MT][2];
+  float lx[MT][2];
   const uint32_t sP = smem_u32(Ps);
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
-    lr[mt][0] = lr[mt][1] = lx[mt][0] = lx[mt][1] = 0.f;
+    lx[mt][0] = lx[mt][1] = 0.f;
 #pragma unroll
     for (int j = 0; j < NTW; ++j) {
       const int nt = warp + NWP * j;
@@ -382,11 +404,13 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
         for (int hf = 0; hf < 2; ++hf) {
           const int row = mt * 16 + gq + hf * 8;
           const int col = nt * 8 + 2 * c4;
-          const float p0 = ex2(s[mt][j][2 * hf] - mrow[mt][hf]);
-          const float p1 = ex2(s[mt][j][2 * hf + 1] - mrow[mt][hf]);
-          const uint32_t pk = pack_f16x2(p0, p1);
-          lr[mt][hf] += f16x2_sum(pk);
-          lx[mt][hf] += p0 + p1;
+          uint32_t pk = 0u;
+          if (nt < NTS) {
+            const float p0 = ex2(fmaf(s[mt][j][2 * hf], sc_ring, -mrow[mt][hf]));
+            const float p1 = ex2(fmaf(s[mt][j][2 * hf + 1], sc_ring, -mrow[mt][hf]));
+            pk = pack_f16x2(p0, p1);
+            lx[mt][hf] += p0 + p1;
+          }
           asm volatile("st.shared.b32 [%0], %1;" ::"r"(sP + (row * LDP + col) * 2), "r"(pk)
                        : "memory");
         }
@@ -397,15 +421,10 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      float v = lr[mt][hf], x = lx[mt][hf];
-      v += __shfl_xor_sync(0xffffffffu, v, 1);
-      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      float x = lx[mt][hf];
       x += __shfl_xor_sync(0xffffffffu, x, 1);
       x += __shfl_xor_sync(0xffffffffu, x, 2);
-      if (c4 == 0) {
-        red_lr[warp * 32 + mt * 16 + gq + hf * 8] = v;
-        red_lx[warp * 32 + mt * 16 + gq + hf * 8] = x;
-      }
+      if (c4 == 0) red_lx[warp * 32 + mt * 16 + gq + hf * 8] = x;
     }
   // V's codes and new rows in shared memory; a wait that gave up ends every
   // thread here (the barrier also publishes P and the row sums)
@@ -421,20 +440,14 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
     const int row = tid;
     const int t = row < p.R ? row / G : -1;
     const float sk = sk_tid;
-    float m = sk;
+    float m = -INFINITY;
     for (int w = 0; w < NWP; ++w) m = fmaxf(m, red_max[w * 32 + row]);
+    m = fmaxf(sk, m * sc_ring);
     const float mb = (m == -INFINITY) ? 0.f : m;
-    float l = 0.f, lxs = 0.f;
-    for (int w = 0; w < NWP; ++w) {
-      l += red_lr[w * 32 + row];
-      lxs += red_lx[w * 32 + row];
-    }
-    if (sk != -INFINITY) {
-      const float ts = ex2(sk - mb);
-      l += ts;
-      lxs += ts;
-    }
-    row_l[row] = l;
+    float lxs = 0.f;
+    for (int w = 0; w < NWP; ++w) lxs += red_lx[w * 32 + row];
+    if (sk != -INFINITY) lxs += ex2(sk - mb);
+    row_l[row] = lxs;
     if (t >= 0 && p.lse != nullptr)
       p.lse[(static_cast<size_t>(b) * n_q + t) * p.Hq + g * G + (row - t * G)] =
           (mb + lg2(lxs)) * kLn2;

@@ -432,8 +432,7 @@ int launch_decode(const swa::DecodeFp8Params& p, cudaStream_t st) {
   if constexpr (KV8) {
     const size_t smem = swa::decode_fp8_smem_bytes(D, p.KP, p.W8, NWP);
     auto kern = swa::decode_fp8_sm100_kernel<D, MT, NWP>;
-    if (ensure_smem_attr(kern, smem, attr) != SWA_OK)
-      return SWA_ERR_CUDA;
+    if (ensure_smem_attr(kern, smem, attr) != SWA_OK) return SWA_ERR_CUDA;
     kern<<<grid, NWP * 32, smem, st>>>(tq, tkr, tkn, tvr, tvn, to, p);
   } else {  // the bf16 ring (the kernel takes the DecodeParams part)
     const size_t smem = swa::decode_smem_bytes(D, p.KP, NWP);
@@ -449,6 +448,7 @@ int launch_decode(const swa::DecodeFp8Params& p, cudaStream_t st) {
 template <bool KV8>
 int pick_decode(const swa::DecodeFp8Params& p, int D, cudaStream_t st) {
   const bool two = p.R > 16;
+  // 4 warps up to 160 keys, else 8
   if (p.KP <= swa::kDecodeSmallMaxKP) {
     constexpr int S = swa::kDecodeSmallWarps;
     if (D == 64)
