@@ -7,6 +7,8 @@ library never imports it, and it imports nothing from the product package.
 
 ``oracle.fp8`` adds the E4M3 code table and encoder and the decode / commit
 over a ring of E4M3 codes with per-kv-head scales (numpy, fp64).
+``oracle.rope`` adds the rotary position embedding applied before the
+attention (fp64 rotation, bf16 rounding) and the ring the prefill writes.
 """
 from .oracle import (  # noqa: F401
     decode,
