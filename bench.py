@@ -94,12 +94,15 @@ def load_peaks():
 # unchanged.
 KERNEL_SOURCES = {
     "ring": ["prefill_swa_ring_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
+    "ring_rope": ["prefill_swa_ring_sm100.cuh", "rope_sm100.cuh", "prefill_sm100.cuh",
+                  "ptx_sm100.cuh", "swa_sink.cu"],
     "chunked": ["prefill_chunked_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "decode": ["decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "decode_fp8": ["decode_fp8_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "splitkv": ["decode_splitkv_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
 }
 WORKLOAD_KERNEL = {"tiny_swa_prefill": "ring", "swa_prefill_32k": "ring",
+                   "swa_prefill_32k_rope": "ring_rope",
                    "varlen_swa_prefill": "ring", "global_prefill_8k": "chunked",
                    "swa_decode_mtp": "decode", "ga_decode_16k": "splitkv",
                    "swa_decode_mtp_fp8": "decode_fp8"}
@@ -192,7 +195,19 @@ class PrefillRunner:
         self.c = c
         self.flops, self.bytes = prefill_work(c["seqlens"], c["Hq"], c["Hkv"], c["D"],
                                               c["window"])
+        self.rope = c["rope_base"] > 0
         dev = torch.device("cuda")
+        self.k_ring = self.v_ring = self.ws = None
+        if self.rope:
+            # the ring the call writes: rotated K and V of each sequence's last
+            # ring_W tokens
+            S, W = len(c["seqlens"]), c["ring_W"]
+            self.k_ring = torch.empty((S, W, c["Hkv"], c["D"]), dtype=torch.bfloat16, device=dev)
+            self.v_ring = torch.empty_like(self.k_ring)
+            self.bytes += sum(min(L, W) for L in c["seqlens"]) * c["Hkv"] * c["D"] * 2 * 2
+            need = B.swa_sink_attn_fwd_rope_workspace(c["total"], c["Hq"], c["Hkv"], c["D"],
+                                                      c["window"])
+            self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.q, self.k, self.v = c["q"].to(dev), c["k"].to(dev), c["v"].to(dev)
         self.cu = c["cu_seqlens"].to(dev)
         self.sink = c["sink"].to(dev) if c["sink"] is not None else None
@@ -215,6 +230,15 @@ class PrefillRunner:
 
     def call(self, stream):
         c = self.c
+        if self.rope:
+            rc = self.B.swa_sink_attn_fwd_rope(
+                self.q, self.k, self.v, self.cu, len(c["seqlens"]), c["max_seqlen"], c["total"],
+                c["Hq"], c["Hkv"], c["D"], c["window"], self.sink, 0.0, c["rope_base"], 0, None,
+                self.k_ring, self.v_ring, c["ring_W"], self.ws, self.ws.numel(), self.o,
+                self.lse, stream)
+            if rc != 0:
+                raise RuntimeError("swa_sink_attn_fwd_rope: %s" % self.B.status_string(rc))
+            return
         rc = self.B.swa_sink_attn_fwd(self.q, self.k, self.v, self.cu, len(c["seqlens"]),
                                       c["max_seqlen"], c["total"], c["Hq"], c["Hkv"], c["D"],
                                       c["window"], self.sink, 0.0, self.o, self.lse, stream)
@@ -223,8 +247,11 @@ class PrefillRunner:
 
     def describe(self):
         c = self.c
-        return {"Hq": c["Hq"], "Hkv": c["Hkv"], "head_dim": c["D"], "window": c["window"],
-                "num_seqs": len(c["seqlens"]), "tokens": c["total"]}
+        out = {"Hq": c["Hq"], "Hkv": c["Hkv"], "head_dim": c["D"], "window": c["window"],
+               "num_seqs": len(c["seqlens"]), "tokens": c["total"]}
+        if self.rope:
+            out.update(rope_base=c["rope_base"], ring=c["ring_W"])
+        return out
 
 
 class DecodeRunner:
@@ -334,8 +361,15 @@ def oracle_sample(workload, wl, seconds, threads, seed=0):
             rt = rng.integers(0, c["total"], n)
             rh = rng.integers(0, c["Hq"], n).astype(np.int32)
             t0 = time.perf_counter()
-            oracle.prefill_rows(c["q"], c["k"], c["v"], c["cu_seqlens"], c["Hq"], c["Hkv"],
-                                c["D"], c["window"], rt, rh, sink=c["sink"], nthreads=threads)
+            if c["rope_base"] > 0:
+                from oracle import rope as orope
+                orope.prefill_rope_rows(c["q"], c["k"], c["v"], c["cu_seqlens"], c["Hq"],
+                                        c["Hkv"], c["D"], c["window"], c["rope_base"], rt, rh,
+                                        sink=c["sink"], nthreads=threads)
+            else:
+                oracle.prefill_rows(c["q"], c["k"], c["v"], c["cu_seqlens"], c["Hq"], c["Hkv"],
+                                    c["D"], c["window"], rt, rh, sink=c["sink"],
+                                    nthreads=threads)
             return time.perf_counter() - t0
         unit = "random (token, head) rows"
     else:

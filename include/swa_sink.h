@@ -137,6 +137,64 @@ SWA_API int swa_sink_attn_fwd_noalloc(const void *q, const void *k, const void *
                               float *lse, int slot, void *stream);
 
 /*
+ * Packed varlen prefill with the rotary position embedding (RoPE) applied to q
+ * and k inside the call, and the decode ring of each sequence written from it.
+ *
+ * Source: the RoPE base per layer type is given in section 3.1 "Data
+ * Scheduler" of the report summary above (SWA 10,000; global 640,000, raised
+ * to 5,000,000 for the 256K extension); the Q&A of the ICML 2026 talk
+ * write-up (hzrcw.cc) says the position index keeps increasing while the
+ * window slides. No page prints the rotation: it is the standard rotary
+ * embedding over the whole head dim. Pair c (0 <= c < D/2) of a row at
+ * absolute position p turns by p * base^(-2c/D):
+ *   (x_a, x_b) -> (x_a cos - x_b sin, x_b cos + x_a sin)
+ * with (a, b) = (c, c + D/2) when rope_interleaved = 0 ("rotate half"), or
+ * (2c, 2c + 1) when rope_interleaved = 1. The rotated q and k are rounded to
+ * bf16 (round to nearest even) and then attended exactly as
+ * swa_sink_attn_fwd does, so the result is that of rotating, storing in bf16
+ * and calling swa_sink_attn_fwd (up to rare 1-ulp differences of a rotated
+ * element lying within ~1e-7 relative of a bf16 rounding boundary).
+ *
+ *   q, k, v, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq, Hkv, D,
+ *   window, sink, softmax_scale, o, lse   as for swa_sink_attn_fwd; q and k
+ *               are NOT rotated (they are read only).
+ *   rope_base   the base (> 0, finite), e.g. 1e4 for SWA layers.
+ *   rope_interleaved  0 or 1 (the pairing above).
+ *   pos0        int32 [num_seqs] device: the position of each sequence's
+ *               first token (token i of sequence s is at pos0[s] + i), or NULL
+ *               for 0. Positions must lie in [0, 2^24); others are clamped
+ *               and flagged (bit 1 of swa_sink_device_error). The attention
+ *               itself still sees only the tokens of this call.
+ *   k_ring, v_ring  bf16 [num_seqs, ring_W, Hkv, D], 16-byte aligned, or
+ *               both NULL. For the last min(L_s, ring_W) tokens of sequence
+ *               s, the rotated key row and the value row of position p go to
+ *               slot p mod ring_W (the layout swa_sink_attn_decode reads);
+ *               the other slots are not touched. ring_W >= pos0[s] + L_s gives
+ *               a plain position-indexed cache (the global layers' layout for
+ *               swa_sink_attn_decode_splitkv).
+ *   workspace   device memory of swa_sink_attn_fwd_rope_workspace() bytes,
+ *               16-byte aligned, owned by the caller (NULL allowed when that
+ *               is 0). Zero for sliding windows on the fused ring kernel
+ *               (Hq/Hkv in {2, 4, 8}, window + 128/(Hq/Hkv) - 1 <= 192 keys):
+ *               it rotates each Q tile and K block in shared memory. For the
+ *               other shapes (global layers among them) a separate pass first
+ *               writes rotated copies of q and k there, then the prefill runs
+ *               on them. Calls that overlap in time need separate workspaces.
+ *
+ * Returns SWA_OK or a negative swa_status_t (SWA_ERR_SHAPE for a bad base,
+ * pairing flag, ring_W or a workspace that is too small).
+ */
+SWA_API size_t swa_sink_attn_fwd_rope_workspace(int total_tokens, int Hq, int Hkv, int D,
+                                                int window);
+SWA_API int swa_sink_attn_fwd_rope(const void *q, const void *k, const void *v,
+                                   const int32_t *cu_seqlens, int num_seqs, int max_seqlen,
+                                   int total_tokens, int Hq, int Hkv, int D, int window,
+                                   const float *sink, float softmax_scale, float rope_base,
+                                   int rope_interleaved, const int32_t *pos0, void *k_ring,
+                                   void *v_ring, int ring_W, void *workspace,
+                                   size_t workspace_bytes, void *o, float *lse, void *stream);
+
+/*
  * Decode / draft verification over a W-slot KV ring per sequence.
  *
  * Source: section 2.3 "Lightweight MTP" of the report summary above (draft

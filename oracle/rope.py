@@ -128,11 +128,15 @@ def prefill_rope(q, k, v, cu_seqlens, Hq, Hkv, D, window, base, pos0=None,
 
 def prefill_rope_rows(q, k, v, cu_seqlens, Hq, Hkv, D, window, base, row_tok, row_head,
                       pos0=None, sink=None, scale=None, interleaved=False, nthreads=None):
-    """prefill_rope on a sample of (token, head) rows: (o [n,D], lse [n])."""
+    """prefill_rope on a sample of (token, head) rows: (o [n,D], lse [n]).
+    Only the sampled tokens' query rows are rotated (no other query row is
+    read); every key row is."""
     pos = token_positions(cu_seqlens, pos0)
-    qr = rope_bf16(q, pos, base, interleaved)
+    qb = _core._bits(q).copy()
+    toks = np.unique(np.asarray(row_tok, dtype=np.int64))
+    qb[toks] = rope_bf16(qb[toks], pos[toks], base, interleaved)
     kr = rope_bf16(k, pos, base, interleaved)
-    o, lse, _ = _core.prefill_rows(qr, kr, v, cu_seqlens, Hq, Hkv, D, window, row_tok,
+    o, lse, _ = _core.prefill_rows(qb, kr, v, cu_seqlens, Hq, Hkv, D, window, row_tok,
                                    row_head, sink=sink, scale=scale, nthreads=nthreads)
     return o, lse
 

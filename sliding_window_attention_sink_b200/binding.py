@@ -5,7 +5,7 @@ integer device pointers) and only marshal arguments; every step of the
 computation runs in the library's CUDA kernels. There is no CPU fallback: if
 the library is missing, loading raises.
 
-Convenience wrappers (`attn_fwd`, `attn_decode`, `kv_commit`) allocate the
+Convenience wrappers (`attn_fwd`, `attn_fwd_rope`, `attn_decode`, `kv_commit`, ...) allocate the
 outputs with torch and raise `SwaSinkError` on a non-zero status.
 """
 import ctypes
@@ -46,6 +46,12 @@ def load():
     lib.swa_sink_attn_fwd_noalloc.restype = _i
     lib.swa_sink_attn_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                               _vp, _f, _vp, _vp, _i, _vp]
+    lib.swa_sink_attn_fwd_rope_workspace.restype = ctypes.c_size_t
+    lib.swa_sink_attn_fwd_rope_workspace.argtypes = [_i, _i, _i, _i, _i]
+    lib.swa_sink_attn_fwd_rope.restype = _i
+    lib.swa_sink_attn_fwd_rope.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
+                                           _f, _f, _i, _vp, _vp, _vp, _i, _vp, ctypes.c_size_t,
+                                           _vp, _vp, _vp]
     lib.swa_sink_attn_decode.restype = _i
     lib.swa_sink_attn_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                          _i, _vp, _f, _vp, _vp, _vp]
@@ -109,6 +115,23 @@ def swa_sink_attn_fwd_noalloc(q, k, v, cu_seqlens, num_seqs, max_seqlen, total_t
         _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), int(num_seqs), int(max_seqlen),
         int(total_tokens), int(Hq), int(Hkv), int(D), int(window), _ptr(sink),
         float(softmax_scale), _ptr(o), _ptr(lse), int(slot), _stream(stream))
+
+
+def swa_sink_attn_fwd_rope_workspace(total_tokens, Hq, Hkv, D, window):
+    return load().swa_sink_attn_fwd_rope_workspace(int(total_tokens), int(Hq), int(Hkv), int(D),
+                                                   int(window))
+
+
+def swa_sink_attn_fwd_rope(q, k, v, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq, Hkv, D,
+                           window, sink, softmax_scale, rope_base, rope_interleaved, pos0,
+                           k_ring, v_ring, ring_W, workspace, workspace_bytes, o, lse,
+                           stream=None):
+    return load().swa_sink_attn_fwd_rope(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), int(num_seqs), int(max_seqlen),
+        int(total_tokens), int(Hq), int(Hkv), int(D), int(window), _ptr(sink),
+        float(softmax_scale), float(rope_base), int(rope_interleaved), _ptr(pos0), _ptr(k_ring),
+        _ptr(v_ring), int(ring_W), _ptr(workspace), int(workspace_bytes), _ptr(o), _ptr(lse),
+        _stream(stream))
 
 
 def swa_sink_attn_decode(q, k_new, v_new, k_ring, v_ring, pos, B, n_q, Hq, Hkv, D, W, sink,
@@ -191,6 +214,37 @@ def attn_fwd(q, k, v, cu_seqlens, window, sink=None, softmax_scale=0.0, max_seql
                            window, sink, softmax_scale, out, lse, stream)
     if rc != SWA_OK:
         raise SwaSinkError(rc, "swa_sink_attn_fwd")
+    return out, lse
+
+
+def attn_fwd_rope(q, k, v, cu_seqlens, window, rope_base, sink=None, pos0=None,
+                  interleaved=False, k_ring=None, v_ring=None, softmax_scale=0.0,
+                  max_seqlen=None, out=None, lse=None, want_lse=True, workspace=None,
+                  stream=None):
+    """attn_fwd with RoPE applied to q and k inside the call (q, k are read
+    only). pos0: int32 CUDA [num_seqs] first position of each sequence (None:
+    0). k_ring / v_ring: bf16 [num_seqs, ring_W, Hkv, D] written with the last
+    ring_W tokens of each sequence (rotated K, V), or None. The workspace (a
+    uint8 CUDA tensor) is allocated here when the shape needs one."""
+    total, Hq, D = q.shape
+    Hkv = k.shape[1]
+    num_seqs = cu_seqlens.numel() - 1
+    if max_seqlen is None:
+        max_seqlen = total
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device)
+    need = swa_sink_attn_fwd_rope_workspace(total, Hq, Hkv, D, window)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ring_W = 0 if k_ring is None else k_ring.shape[1]
+    rc = swa_sink_attn_fwd_rope(q, k, v, cu_seqlens, num_seqs, max_seqlen, total, Hq, Hkv, D,
+                                window, sink, softmax_scale, rope_base, 1 if interleaved else 0,
+                                pos0, k_ring, v_ring, ring_W, workspace,
+                                0 if workspace is None else workspace.numel(), out, lse, stream)
+    if rc != SWA_OK:
+        raise SwaSinkError(rc, "swa_sink_attn_fwd_rope")
     return out, lse
 
 

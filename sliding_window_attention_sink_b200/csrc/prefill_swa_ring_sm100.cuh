@@ -46,6 +46,7 @@
 
 #include "prefill_sm100.cuh"
 #include "ptx_sm100.cuh"
+#include "rope_sm100.cuh"
 
 namespace swa {
 
@@ -126,12 +127,23 @@ __host__ __device__ inline size_t ring_smem_bytes(int D, int TM, int NB, int NQ)
 
 // BN16 = BN / 16 is fixed at compile time so a half row of scores lives in
 // registers.
-template <int D, int BN16>
+//
+// ROPE: q and k arrive before the rotary embedding. The epilogue warpgroup
+// rotates each Q tile in its stage and each new K block in its ring slot (in
+// shared memory, in place, rounded to bf16) before the S issuer may use them
+// (barriers q_rot / k_rot instead of the TMA barriers), then drains the
+// previous tile's O: per tile it does rotate(j), drain(j - 1). Thread item
+// (token, 8-pair group) computes the group's 8 angles once and rotates the G
+// query rows of that token and the token's key row (the tile's own key block
+// holds the tile's tokens). For the last ring_W tokens of each sequence it
+// also writes the rotated key row and the value row into the caller's ring.
+template <int D, int BN16, bool ROPE>
 __global__ void __launch_bounds__(kRingThreads, 1)
     prefill_swa_ring_kernel(const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v,
-                            const __grid_constant__ CUtensorMap tm_o, const RingParams p) {
+                            const __grid_constant__ CUtensorMap tm_o, const RingParams p,
+                            const __grid_constant__ RopeArgs rope) {
   constexpr int NCH = D / 64;
   constexpr uint32_t CH = 16384;  // one 128-row x 128-byte chunk
   constexpr int BN = BN16 * 16;
@@ -143,6 +155,8 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   __shared__ __align__(8) uint64_t kv_full[kRingMaxBlocks], kv_empty[kRingMaxBlocks];
   __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], l_free[2];
   __shared__ __align__(8) uint64_t o_full, o_empty;
+  // ROPE only: Q stage / K block rotated in place
+  __shared__ __align__(8) uint64_t q_rot[kRingMaxQ], k_rot[kRingMaxBlocks];
   __shared__ float red_max[2][128], red_lr[2][128], red_lx[2][128], l_s[2][128];
   // ranges of tiles, from the producer to the 14 other warps
   __shared__ __align__(8) uint64_t rq_full[kRingRanges], rq_empty[kRingRanges];
@@ -183,6 +197,10 @@ __global__ void __launch_bounds__(kRingThreads, 1)
     for (int q = 0; q < kRingRanges; ++q) {
       mbar_init(smem_u32(&rq_full[q]), 1);
       mbar_init(smem_u32(&rq_empty[q]), kRingRangeReaders);
+    }
+    if (ROPE) {
+      for (int s = 0; s < p.NQ; ++s) mbar_init(smem_u32(&q_rot[s]), 4);
+      for (int s = 0; s < p.NB; ++s) mbar_init(smem_u32(&k_rot[s]), 4);
     }
     abort_sh = 0;
     fence_barrier_init();
@@ -368,25 +386,17 @@ __global__ void __launch_bounds__(kRingThreads, 1)
     const int r = 32 * (warp & 3) + lane;
     const bool issuer = tid == 256;
     const uint32_t tO = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + p.o_col;
-    int j = 0;
-    bool stop = false;
-    for (int q = 0; !stop; ++q) {
-     int f0 = 0, f1 = 0;
-     if (named_bar_any(2, 128, !next_range(q, f0, f1))) break;
-     for (int f = f0; f < f1; ++f, ++j) {
-      int g, tb;
-      tile_of(f, g, tb);
-      const int b = j & 1;
-      if (issuer) RING_TRACE(4, j, 0);
+    // O of tile jd (kv head gd, token tile tbd) to HBM; false when a wait gave
+    // up (the epilogue warps then leave together)
+    auto drain = [&](int jd, int gd, int tbd) -> bool {
+      const int b = jd & 1;
+      if (issuer) RING_TRACE(4, jd, 0);
       // p_full[b] of this tile completed before PV was issued; waiting on it
       // too orders the softmax's write of l_s[b] before the read below
-      const bool ok = mbar_wait(smem_u32(&o_full), j & 1, abort) &&
-                      mbar_wait(smem_u32(&p_full[b]), (j >> 1) & 1, abort);
-      if (named_bar_any(2, 128, !ok)) {  // the epilogue warps leave together
-        stop = true;
-        break;
-      }
-      if (issuer) RING_TRACE(4, j, 1);
+      const bool ok = mbar_wait(smem_u32(&o_full), jd & 1, abort) &&
+                      mbar_wait(smem_u32(&p_full[b]), (jd >> 1) & 1, abort);
+      if (named_bar_any(2, 128, !ok)) return false;
+      if (issuer) RING_TRACE(4, jd, 1);
       __syncwarp();
       tc_fence_after();
       const float l = l_s[b][r];
@@ -409,7 +419,7 @@ __global__ void __launch_bounds__(kRingThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&o_empty));
-          if (issuer) RING_TRACE(4, j, 2);
+          if (issuer) RING_TRACE(4, jd, 2);
         }
         if (issuer) tma_store_wait_read<NCH - 1>();
         named_bar_sync(2, 128);
@@ -426,12 +436,139 @@ __global__ void __launch_bounds__(kRingThreads, 1)
         fence_proxy_async_smem();
         named_bar_sync(2, 128);
         if (issuer) {
-          tma_store_3d(&tm_o, sO + ch * CH, ch * 64, g * p.G, tb * p.TM);
+          tma_store_3d(&tm_o, sO + ch * CH, ch * 64, gd * p.G, tbd * p.TM);
           tma_store_commit();
         }
       }
-      if (issuer) RING_TRACE(4, j, 3);
-     }
+      if (issuer) RING_TRACE(4, jd, 3);
+      return true;
+    };
+    int j = 0;
+    bool stop = false;
+    if constexpr (!ROPE) {
+      for (int q = 0; !stop; ++q) {
+        int f0 = 0, f1 = 0;
+        if (named_bar_any(2, 128, !next_range(q, f0, f1))) break;
+        for (int f = f0; f < f1; ++f, ++j) {
+          int g, tb;
+          tile_of(f, g, tb);
+          if (!drain(j, g, tb)) {
+            stop = true;
+            break;
+          }
+        }
+      }
+    } else {
+      constexpr int NK = D / 16;  // 8-pair groups per row
+      const bool inter = rope.interleaved != 0;
+      // cached sequence of the last token looked up
+      int s_lo = 1, s_hi = 0, s_idx = 0, s_p0 = 0;
+      // unit u of row `row` in a 1024-byte-aligned 128-byte-swizzled block
+      auto unit_addr = [](uint32_t blk, int row, int u) -> uint32_t {
+        return blk + row * 128 + ((u ^ (row & 7)) << 4);
+      };
+      // rotate tile jr's Q stage and its new K blocks [first_new, last_new)
+      auto rotate = [&](int jr, int first_new, int last_new, int gr, int tbr) -> bool {
+        const int st = jr % p.NQ;
+        bool ok = mbar_wait(smem_u32(&q_full[st]), (jr / p.NQ) & 1, abort);
+        for (int s = first_new; s < last_new && ok; ++s)
+          ok = mbar_wait(smem_u32(&kv_full[s % p.NB]), (s / p.NB) & 1, abort);
+        if (named_bar_any(2, 128, !ok)) return false;
+        const int t0 = tbr * p.TM;
+        const int nnew = last_new - first_new;
+        const int first_kb = tbr - nnew + 1;
+        const uint32_t qst = sQ + st * NCH * CH;
+        const uint32_t kslot = static_cast<uint32_t>((last_new - 1) % p.NB) * blk_bytes;
+        for (int it = r; it < p.TM * NK; it += 128) {
+          const int tok = it / NK, k = it - tok * NK;
+          int da, db;
+          rope_units<D>(k, inter, da, db);
+          const int cha = da >> 6, ua = (da & 63) >> 3, chb = db >> 6, ub = (db & 63) >> 3;
+          float cs[8], sn[8];
+          uint32_t a[4], bq[4];
+          const int t = t0 + tok;
+          if (t < p.total) {
+            const int ps = rope_token_pos(p.cu_seqlens, p.num_seqs, rope.pos0, t, s_lo, s_hi,
+                                          s_idx, s_p0);
+            rope_cos_sin8(rope, ps, 8 * k, cs, sn);
+            // the token's G query rows
+            for (int hh = 0; hh < p.G; ++hh) {
+              const int row = tok * p.G + hh;
+              const uint32_t aa = unit_addr(qst + cha * CH, row, ua);
+              const uint32_t ab = unit_addr(qst + chb * CH, row, ub);
+              ld_shared_v4(aa, a);
+              ld_shared_v4(ab, bq);
+              rope_rotate8(a, bq, cs, sn, inter);
+              st_shared_v4(aa, a[0], a[1], a[2], a[3]);
+              st_shared_v4(ab, bq[0], bq[1], bq[2], bq[3]);
+            }
+            // its key row in the tile's own (last new) block
+            const uint32_t ka = unit_addr(sK + cha * ring_ch + kslot, tok, ua);
+            const uint32_t kb = unit_addr(sK + chb * ring_ch + kslot, tok, ub);
+            ld_shared_v4(ka, a);
+            ld_shared_v4(kb, bq);
+            rope_rotate8(a, bq, cs, sn, inter);
+            st_shared_v4(ka, a[0], a[1], a[2], a[3]);
+            st_shared_v4(kb, bq[0], bq[1], bq[2], bq[3]);
+            if (rope.k_ring != nullptr && t - s_lo >= (s_hi - s_lo) - rope.ring_W) {
+              const size_t rrow = (static_cast<size_t>(s_idx) * rope.ring_W +
+                                   static_cast<size_t>(ps) % rope.ring_W) * p.Hkv + gr;
+              __nv_bfloat16* kr = rope.k_ring + rrow * D;
+              __nv_bfloat16* vr = rope.v_ring + rrow * D;
+              st_global_v4(kr + da, a);
+              st_global_v4(kr + db, bq);
+              ld_shared_v4(unit_addr(sV + cha * ring_ch + kslot, tok, ua), a);
+              ld_shared_v4(unit_addr(sV + chb * ring_ch + kslot, tok, ub), bq);
+              st_global_v4(vr + da, a);
+              st_global_v4(vr + db, bq);
+            }
+          }
+          // earlier blocks of a window loaded whole (range or kv-head start)
+          for (int n = 0; n + 1 < nnew; ++n) {
+            const int tk = (first_kb + n) * p.TM + tok;
+            if (tk < 0 || tk >= p.total) continue;  // zero fill
+            const int ps = rope_token_pos(p.cu_seqlens, p.num_seqs, rope.pos0, tk, s_lo, s_hi,
+                                          s_idx, s_p0);
+            rope_cos_sin8(rope, ps, 8 * k, cs, sn);
+            const uint32_t sl = static_cast<uint32_t>((first_new + n) % p.NB) * blk_bytes;
+            const uint32_t ka = unit_addr(sK + cha * ring_ch + sl, tok, ua);
+            const uint32_t kb = unit_addr(sK + chb * ring_ch + sl, tok, ub);
+            ld_shared_v4(ka, a);
+            ld_shared_v4(kb, bq);
+            rope_rotate8(a, bq, cs, sn, inter);
+            st_shared_v4(ka, a[0], a[1], a[2], a[3]);
+            st_shared_v4(kb, bq[0], bq[1], bq[2], bq[3]);
+          }
+        }
+        // the rotated tiles go to the tensor cores (async proxy)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(smem_u32(&q_rot[st]));
+          for (int s = first_new; s < last_new; ++s) mbar_arrive(smem_u32(&k_rot[s % p.NB]));
+        }
+        return true;
+      };
+      int nload = 0;
+      int pj = -1, pg = 0, ptb = 0;  // the tile whose O is still to drain
+      for (int q = 0; !stop; ++q) {
+        int f0 = 0, f1 = 0;
+        if (named_bar_any(2, 128, !next_range(q, f0, f1))) break;
+        for (int f = f0; f < f1; ++f, ++j) {
+          int g, tb;
+          tile_of(f, g, tb);
+          const int first_new = nload;
+          nload += new_blocks(f == f0, tb);
+          if (!rotate(j, first_new, nload, g, tb) || (pj >= 0 && !drain(pj, pg, ptb))) {
+            stop = true;
+            break;
+          }
+          pj = j;
+          pg = g;
+          ptb = tb;
+        }
+      }
+      if (!stop && pj >= 0) drain(pj, pg, ptb);
     }
     if (issuer) tma_store_wait_all<0>();
   } else if (warp == 12) {
@@ -533,14 +670,16 @@ __global__ void __launch_bounds__(kRingThreads, 1)
         break;
       }
       if (lane == 0) RING_TRACE(1, j, 1);
-      if (!mbar_wait(smem_u32(&q_full[st]), (j / p.NQ) & 1, abort)) {
+      // with ROPE, Q and the new K blocks once the epilogue has rotated them
+      if (!mbar_wait(smem_u32(ROPE ? &q_rot[st] : &q_full[st]), (j / p.NQ) & 1, abort)) {
         stop = true;
         break;
       }
       if (lane == 0) RING_TRACE(1, j, 2);
       bool ok = true;
       for (int s = first_new; s < nload && ok; ++s)
-        ok = mbar_wait(smem_u32(&kv_full[s % p.NB]), (s / p.NB) & 1, abort);
+        ok = mbar_wait(smem_u32(ROPE ? &k_rot[s % p.NB] : &kv_full[s % p.NB]), (s / p.NB) & 1,
+                       abort);
       if (!ok) {
         stop = true;
         break;

@@ -24,6 +24,7 @@
 #include "prefill_chunked_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "prefill_swa_ring_sm100.cuh"
+#include "rope_sm100.cuh"
 
 namespace {
 
@@ -144,7 +145,7 @@ int sm_count() {
   return n;
 }
 
-size_t g_attr_ring[2][swa::kRingMaxBN16 + 1][kMaxDevices];
+size_t g_attr_ring[2][2][swa::kRingMaxBN16 + 1][kMaxDevices];
 
 // ---- tile scheduler state -----------------------------------------------------
 // The persistent prefill kernels draw tile ranges from a counter in device
@@ -224,13 +225,14 @@ void split_schedule(int n_tiles, int grid, int* static_tiles, int* dyn_base) {
   *dyn_base = *static_tiles * grid;
 }
 
-template <int D, int BN16>
+template <int D, int BN16, bool ROPE>
 int run_ring(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-             const CUtensorMap& to, const swa::RingParams& p, size_t smem, int grid,
-             cudaStream_t st) {
-  auto kern = swa::prefill_swa_ring_kernel<D, BN16>;
-  if (ensure_smem_attr(kern, smem, g_attr_ring[D == 128][BN16]) != SWA_OK) return SWA_ERR_CUDA;
-  kern<<<grid, swa::kRingThreads, smem, st>>>(tq, tk, tv, to, p);
+             const CUtensorMap& to, const swa::RingParams& p, const swa::RopeArgs& rope,
+             size_t smem, int grid, cudaStream_t st) {
+  auto kern = swa::prefill_swa_ring_kernel<D, BN16, ROPE>;
+  if (ensure_smem_attr(kern, smem, g_attr_ring[ROPE][D == 128][BN16]) != SWA_OK)
+    return SWA_ERR_CUDA;
+  kern<<<grid, swa::kRingThreads, smem, st>>>(tq, tk, tv, to, p, rope);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SWA_OK : cuda_fail("ring prefill launch", e);
 }
@@ -238,30 +240,46 @@ int run_ring(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
 // Dynamic shared memory available next to the ring kernel's static barriers.
 constexpr size_t kRingSmemLimit = 232448 - 5120;
 
-// Sliding-window prefill on the persistent ring pipeline when the window's
-// keys for one tile fit one MMA (BN <= 256) and the S/P double buffer plus O
-// fit TMEM. Returns SWA_ERR_UNSUPPORTED (nothing launched) otherwise. The tile
-// scheduler uses static slot `noalloc` when it is >= 0, else the next slot of
-// the library's per-device buffer.
+// Shape of the ring pipeline for head dim D, group G and window W > 0: tile
+// tokens TM, key blocks per window NWIN (BN = NWIN * TM keys), S column
+// stride, Q stages NQ and ring blocks NB. False when the window's keys for
+// one tile do not fit one MMA (BN <= 192), the S/P double buffer plus O do
+// not fit TMEM, or the stages do not fit shared memory.
+struct RingShape {
+  int TM, KB, NWIN, BN, scol, NQ, NB;
+};
+bool ring_shape(int D, int G, int window, RingShape* r) {
+  if (window <= 0 || !(G == 2 || G == 4 || G == 8)) return false;
+  r->TM = 128 / G;
+  r->KB = (window - 1 + r->TM - 1) / r->TM;
+  r->NWIN = r->KB + 1;
+  r->BN = r->NWIN * r->TM;
+  r->scol = round_up(r->BN, 32);
+  if (r->BN > 16 * swa::kRingMaxBN16 || 2 * r->scol + D > 512) return false;
+  r->NQ = 3;
+  r->NB = std::min(swa::kRingMaxBlocks, r->NWIN + 3);
+  while (swa::ring_smem_bytes(D, r->TM, r->NB, r->NQ) > kRingSmemLimit) {
+    if (r->NB > r->NWIN + 1) --r->NB;
+    else if (r->NQ > 2) --r->NQ;
+    else return false;
+  }
+  return r->NB > r->NWIN;
+}
+
+// Sliding-window prefill on the persistent ring pipeline when ring_shape
+// accepts the shape; SWA_ERR_UNSUPPORTED (nothing launched) otherwise. The
+// tile scheduler uses static slot `noalloc` when it is >= 0, else the next
+// slot of the library's per-device buffer. With `rope` the kernel rotates q
+// and k itself (and writes the ring it names).
 template <int D>
 int launch_prefill_ring(const void* q, const void* k, const void* v, const int32_t* cu,
                         int num_seqs, int total, int Hq, int Hkv, int window, const float* sink,
-                        float scale, void* o, float* lse, cudaStream_t st, int noalloc) {
+                        float scale, void* o, float* lse, cudaStream_t st, int noalloc,
+                        const swa::RopeArgs* rope = nullptr) {
   const int G = Hq / Hkv;
-  if (window <= 0 || !(G == 2 || G == 4 || G == 8)) return SWA_ERR_UNSUPPORTED;
-  const int TM = 128 / G;
-  const int KB = (window - 1 + TM - 1) / TM;
-  const int NWIN = KB + 1;
-  const int BN = NWIN * TM;
-  const int scol = round_up(BN, 32);
-  if (BN > 16 * swa::kRingMaxBN16 || 2 * scol + D > 512) return SWA_ERR_UNSUPPORTED;
-  int NQ = 3, NB = std::min(swa::kRingMaxBlocks, NWIN + 3);
-  while (swa::ring_smem_bytes(D, TM, NB, NQ) > kRingSmemLimit) {
-    if (NB > NWIN + 1) --NB;
-    else if (NQ > 2) --NQ;
-    else return SWA_ERR_UNSUPPORTED;
-  }
-  if (NB <= NWIN) return SWA_ERR_UNSUPPORTED;
+  RingShape rs;
+  if (!ring_shape(D, G, window, &rs)) return SWA_ERR_UNSUPPORTED;
+  const int TM = rs.TM, BN = rs.BN;
   unsigned int* slot = nullptr;
   if ((noalloc >= 0 ? noalloc_slot(noalloc, &slot) : sched_slot(&slot)) != SWA_OK)
     return SWA_ERR_CUDA;
@@ -274,18 +292,18 @@ int launch_prefill_ring(const void* q, const void* k, const void* v, const int32
   p.G = G;
   p.TM = TM;
   p.window = window;
-  p.KB = KB;
-  p.NWIN = NWIN;
-  p.NB = NB;
-  p.NQ = NQ;
+  p.KB = rs.KB;
+  p.NWIN = rs.NWIN;
+  p.NB = rs.NB;
+  p.NQ = rs.NQ;
   p.n_tok_tiles = (total + TM - 1) / TM;
   p.n_tiles = p.n_tok_tiles * Hkv;
   p.sink = sink;
   p.scale_log2 = scale * swa::kLog2e;
   p.lse = lse;
   p.q_box_bytes = 128u * TM * G;
-  p.s_stride = static_cast<uint32_t>(scol);
-  p.o_col = static_cast<uint32_t>(2 * scol);
+  p.s_stride = static_cast<uint32_t>(rs.scol);
+  p.o_col = static_cast<uint32_t>(2 * rs.scol);
 
   CUtensorMap tq, tk, tv, to;
   if (encode_3d(&tq, q, D, Hq, total, 64, G, TM) != SWA_OK) return SWA_ERR_CUDA;
@@ -293,17 +311,19 @@ int launch_prefill_ring(const void* q, const void* k, const void* v, const int32
   if (encode_3d(&tv, v, D, Hkv, total, 64, 1, TM) != SWA_OK) return SWA_ERR_CUDA;
   if (encode_3d(&to, o, D, Hq, total, 64, G, TM) != SWA_OK) return SWA_ERR_CUDA;
 
-  const size_t smem = swa::ring_smem_bytes(D, TM, NB, NQ);
+  const size_t smem = swa::ring_smem_bytes(D, TM, rs.NB, rs.NQ);
   const int nsm = sm_count();
   if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)", 0);
   const int grid = std::min(nsm, p.n_tiles);
   p.sched = slot;
   p.dyn_span = kRingDynSpan;
   split_schedule(p.n_tiles, grid, &p.static_tiles, &p.dyn_base);
+  static const swa::RopeArgs no_rope{};
   switch (BN / 16) {
-#define SWA_RING_CASE(N)                                                        \
-  case N:                                                                       \
-    return run_ring<D, N>(tq, tk, tv, to, p, smem, grid, st);
+#define SWA_RING_CASE(N)                                                              \
+  case N:                                                                             \
+    return rope ? run_ring<D, N, true>(tq, tk, tv, to, p, *rope, smem, grid, st)      \
+                : run_ring<D, N, false>(tq, tk, tv, to, p, no_rope, smem, grid, st);
     SWA_RING_CASE(1) SWA_RING_CASE(2) SWA_RING_CASE(3) SWA_RING_CASE(4) SWA_RING_CASE(5)
     SWA_RING_CASE(6) SWA_RING_CASE(7) SWA_RING_CASE(8) SWA_RING_CASE(9) SWA_RING_CASE(10)
     SWA_RING_CASE(11) SWA_RING_CASE(12)
@@ -557,6 +577,114 @@ int fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seql
                              softmax_scale, o, lse, st);
 }
 
+// ---- prefill with the rotary embedding ------------------------------------------
+// The ring kernel rotates q and k in shared memory (no workspace); the other
+// prefill kernels read q and k through TMA straight into the MMAs, so for them
+// a standalone pass first writes rotated copies into the caller's workspace
+// (q then k, the k copy 256-byte aligned).
+size_t rope_k_offset(int total, int Hq, int D) {
+  const size_t qb = static_cast<size_t>(total) * Hq * D * 2;
+  return (qb + 255) / 256 * 256;
+}
+
+size_t rope_workspace_bytes(int total, int Hq, int Hkv, int D, int window) {
+  if (total <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (D != 64 && D != 128)) return 0;
+  RingShape rs;
+  if (ring_shape(D, Hq / Hkv, window, &rs)) return 0;
+  return rope_k_offset(total, Hq, D) + static_cast<size_t>(total) * Hkv * D * 2;
+}
+
+int fwd_rope_impl(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                  int num_seqs, int max_seqlen, int total_tokens, int Hq, int Hkv, int D,
+                  int window, const float* sink, float softmax_scale, float rope_base,
+                  int rope_interleaved, const int32_t* pos0, void* k_ring, void* v_ring,
+                  int ring_W, void* workspace, size_t workspace_bytes, void* o, float* lse,
+                  void* stream) {
+  if (num_seqs < 0 || max_seqlen < 0 || total_tokens < 0 || Hq <= 0 || Hkv <= 0)
+    return SWA_ERR_SHAPE;
+  if (Hq % Hkv != 0) return SWA_ERR_SHAPE;
+  if (total_tokens > 0 && num_seqs == 0) return SWA_ERR_SHAPE;
+  if (max_seqlen > total_tokens) return SWA_ERR_SHAPE;
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return SWA_ERR_SHAPE;
+  if (rope_interleaved != 0 && rope_interleaved != 1) return SWA_ERR_SHAPE;
+  if ((k_ring == nullptr) != (v_ring == nullptr)) return SWA_ERR_NULL;
+  if (k_ring != nullptr && ring_W < 1) return SWA_ERR_SHAPE;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 128) return SWA_ERR_UNSUPPORTED;
+  if (total_tokens == 0) return SWA_OK;
+  if (!q || !k || !v || !o || !cu_seqlens) return SWA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SWA_ERR_ALIGN;
+  if (k_ring != nullptr && (!aligned16(k_ring) || !aligned16(v_ring))) return SWA_ERR_ALIGN;
+  if (!aligned4(cu_seqlens) || (sink && !aligned4(sink)) || (lse && !aligned4(lse)) ||
+      (pos0 && !aligned4(pos0)))
+    return SWA_ERR_ALIGN;
+  const size_t need = rope_workspace_bytes(total_tokens, Hq, Hkv, D, window);
+  if (need > 0) {
+    if (workspace == nullptr) return SWA_ERR_NULL;
+    if (workspace_bytes < need) return SWA_ERR_SHAPE;
+    if (!aligned16(workspace)) return SWA_ERR_ALIGN;
+  }
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  swa::RopeArgs ra{};
+  ra.pos0 = pos0;
+  ra.interleaved = rope_interleaved;
+  // theta_c / (2 pi) = base^(-2c/D) / (2 pi), split into two floats
+  for (int c = 0; c < D / 2; ++c) {
+    const double f = std::pow(static_cast<double>(rope_base), -2.0 * c / D) /
+                     (2.0 * 3.14159265358979323846);
+    ra.f_hi[c] = static_cast<float>(f);
+    ra.f_lo[c] = static_cast<float>(f - static_cast<double>(ra.f_hi[c]));
+  }
+  ra.k_ring = static_cast<__nv_bfloat16*>(k_ring);
+  ra.v_ring = static_cast<__nv_bfloat16*>(v_ring);
+  ra.ring_W = k_ring != nullptr ? ring_W : 0;
+
+  if (need == 0) {  // the ring kernel, fused
+    return D == 64 ? launch_prefill_ring<64>(q, k, v, cu_seqlens, num_seqs, total_tokens, Hq,
+                                             Hkv, window, sink, softmax_scale, o, lse, st, -1,
+                                             &ra)
+                   : launch_prefill_ring<128>(q, k, v, cu_seqlens, num_seqs, total_tokens, Hq,
+                                              Hkv, window, sink, softmax_scale, o, lse, st, -1,
+                                              &ra);
+  }
+  // rotate into the workspace, then the plain prefill on the rotated copies
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  swa::RopePassParams pp;
+  pp.q = static_cast<const __nv_bfloat16*>(q);
+  pp.k = static_cast<const __nv_bfloat16*>(k);
+  pp.v = static_cast<const __nv_bfloat16*>(v);
+  pp.q_out = reinterpret_cast<__nv_bfloat16*>(ws);
+  pp.k_out = reinterpret_cast<__nv_bfloat16*>(ws + rope_k_offset(total_tokens, Hq, D));
+  pp.cu_seqlens = cu_seqlens;
+  pp.num_seqs = num_seqs;
+  pp.total = total_tokens;
+  pp.Hq = Hq;
+  pp.Hkv = Hkv;
+  if (D == 64) swa::rope_pass_kernel<64><<<total_tokens, 128, 0, st>>>(pp, ra);
+  else swa::rope_pass_kernel<128><<<total_tokens, 128, 0, st>>>(pp, ra);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("rope pass launch", e);
+  const void* qr = pp.q_out;
+  const void* kr = pp.k_out;
+  {
+    const int rc = D == 64 ? launch_prefill_chunked<64>(qr, kr, v, cu_seqlens, num_seqs,
+                                                        total_tokens, Hq, Hkv, window, sink,
+                                                        softmax_scale, o, lse, st)
+                           : launch_prefill_chunked<128>(qr, kr, v, cu_seqlens, num_seqs,
+                                                         total_tokens, Hq, Hkv, window, sink,
+                                                         softmax_scale, o, lse, st);
+    if (rc != SWA_ERR_UNSUPPORTED) return rc;
+  }
+  if (D == 64)
+    return launch_prefill<64>(qr, kr, v, cu_seqlens, num_seqs, total_tokens, Hq, Hkv, window,
+                              sink, softmax_scale, o, lse, st);
+  return launch_prefill<128>(qr, kr, v, cu_seqlens, num_seqs, total_tokens, Hq, Hkv, window, sink,
+                             softmax_scale, o, lse, st);
+}
+
 // ---- split-KV decode ------------------------------------------------------------
 // Ranges per (sequence, kv head) and their length: enough CTAs for a few waves
 // (a fixed target, so that the workspace size does not depend on the device),
@@ -641,6 +769,21 @@ int swa_sink_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   if (slot < 0 || slot >= kNoAllocSlots) return SWA_ERR_SHAPE;
   return fwd_impl(q, k, v, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq, Hkv, D, window,
                   sink, softmax_scale, o, lse, stream, slot);
+}
+
+size_t swa_sink_attn_fwd_rope_workspace(int total_tokens, int Hq, int Hkv, int D, int window) {
+  return rope_workspace_bytes(total_tokens, Hq, Hkv, D, window);
+}
+
+int swa_sink_attn_fwd_rope(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                           int num_seqs, int max_seqlen, int total_tokens, int Hq, int Hkv, int D,
+                           int window, const float* sink, float softmax_scale, float rope_base,
+                           int rope_interleaved, const int32_t* pos0, void* k_ring, void* v_ring,
+                           int ring_W, void* workspace, size_t workspace_bytes, void* o,
+                           float* lse, void* stream) {
+  return fwd_rope_impl(q, k, v, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq, Hkv, D,
+                       window, sink, softmax_scale, rope_base, rope_interleaved, pos0, k_ring,
+                       v_ring, ring_W, workspace, workspace_bytes, o, lse, stream);
 }
 
 int swa_sink_attn_decode(const void* q, const void* k_new, const void* v_new, const void* k_ring,

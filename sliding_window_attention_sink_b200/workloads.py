@@ -34,6 +34,11 @@ class PrefillCase:
     sink: Optional[str]    # "uniform2" (U(-2,2)), "normal" (N(0,1)) or None
     seed: int
     varlen_draw: Optional[tuple] = None  # (num_seqs, lo, hi) drawn from seed
+    # > 0: q and k are given before the rotary embedding with this base (token
+    # i of a sequence at position i), and the call writes a ring of ring_W
+    # slots per sequence
+    rope_base: float = 0.0
+    ring_W: int = 0
 
 
 @dataclass
@@ -58,7 +63,9 @@ class DecodeCase:
     kv: str = "bf16"
 
 
-# The workloads: a tiny parity case, one SWA layer, one global layer, a packed
+# The workloads: a tiny parity case, one SWA layer (also with the rotary
+# embedding applied inside the call and the decode ring written), one global
+# layer, a packed
 # varlen SWA batch, a decode / draft-verification batch of the SWA layers and
 # one of a global layer over long contexts.
 WORKLOADS = {
@@ -68,6 +75,9 @@ WORKLOADS = {
     "swa_prefill_32k": PrefillCase(
         "swa_prefill T=32768 Hq=64 Hkv=8 D=128 W=128", [32768], 64, 8, 128,
         128, 0.5, "normal", 2),
+    "swa_prefill_32k_rope": PrefillCase(
+        "swa_prefill_rope T=32768 Hq=64 Hkv=8 D=128 W=128 rope_base=1e4 ring=128", [32768],
+        64, 8, 128, 128, 0.5, "normal", 2, rope_base=1e4, ring_W=128),
     "global_prefill_8k": PrefillCase(
         "global_prefill T=8192 Hq=64 Hkv=8 D=128 full-causal", [8192], 64, 8,
         128, 0, 0.5, "normal", 3),
@@ -130,7 +140,8 @@ def make_prefill(case: PrefillCase):
     sink = _sink(case.sink, case.Hq, g)
     return dict(q=q, k=k, v=v, cu_seqlens=cu, sink=sink, seqlens=seqlens,
                 total=total, Hq=case.Hq, Hkv=case.Hkv, D=case.D,
-                window=case.window, max_seqlen=max(seqlens) if seqlens else 0)
+                window=case.window, max_seqlen=max(seqlens) if seqlens else 0,
+                rope_base=case.rope_base, ring_W=case.ring_W)
 
 
 def make_decode(case: DecodeCase):

@@ -157,3 +157,46 @@ def test_fp8_decode_and_commit_argument_errors():
     assert g(**dict(c, D=32)) == -3
     assert g(**dict(c, W=0)) == -2
     assert g(**dict(c, B=0)) == 0
+
+
+def fwd_rope(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, cu_seqlens=FAKE, num_seqs=1, max_seqlen=8,
+             total_tokens=8, Hq=8, Hkv=2, D=128, window=128, sink=None,
+             softmax_scale=0.0, rope_base=1e4, rope_interleaved=0, pos0=None,
+             k_ring=None, v_ring=None, ring_W=0, workspace=None, workspace_bytes=0,
+             o=FAKE, lse=None, stream=0)
+    a.update(kw)
+    return B.swa_sink_attn_fwd_rope(**a)
+
+
+def test_fwd_rope_argument_errors():
+    assert fwd_rope(rope_base=0.0) == -2
+    assert fwd_rope(rope_base=float("inf")) == -2
+    assert fwd_rope(rope_base=float("nan")) == -2
+    assert fwd_rope(rope_interleaved=2) == -2
+    assert fwd_rope(k_ring=FAKE) == -1                     # v_ring missing
+    assert fwd_rope(k_ring=FAKE, v_ring=FAKE, ring_W=0) == -2
+    assert fwd_rope(k_ring=FAKE + 8, v_ring=FAKE, ring_W=4) == -4
+    assert fwd_rope(pos0=FAKE + 2) == -4
+    assert fwd_rope(Hq=8, Hkv=3) == -2
+    assert fwd_rope(D=96) == -3
+    assert fwd_rope(q=None) == -1
+    # shapes that need a workspace: a global layer, G = 1
+    assert fwd_rope(window=0) == -1
+    assert fwd_rope(window=0, workspace=FAKE, workspace_bytes=16) == -2
+    assert fwd_rope(window=0, workspace=FAKE + 4, workspace_bytes=1 << 20) == -4
+    assert fwd_rope(total_tokens=0, max_seqlen=0) == 0
+
+
+def test_fwd_rope_workspace_sizes():
+    ws = B.swa_sink_attn_fwd_rope_workspace
+    # the fused ring kernel needs none
+    assert ws(32768, 64, 8, 128, 128) == 0
+    assert ws(1000, 8, 2, 128, 128) == 0
+    assert ws(1000, 4, 2, 64, 20) == 0
+    # the others: rotated q (padded to 256 bytes) + rotated k
+    q_bytes = 8192 * 64 * 128 * 2
+    assert ws(8192, 64, 8, 128, 0) == q_bytes + 8192 * 8 * 128 * 2
+    assert ws(300, 2, 2, 64, 128) == (300 * 2 * 64 * 2 + 255) // 256 * 256 + 300 * 2 * 64 * 2
+    assert ws(600, 8, 1, 64, 300) > 0          # window too wide for the ring
+    assert ws(0, 64, 8, 128, 0) == 0
