@@ -97,12 +97,14 @@ KERNEL_SOURCES = {
     "ring_rope": ["prefill_swa_ring_sm100.cuh", "rope_sm100.cuh", "prefill_sm100.cuh",
                   "ptx_sm100.cuh", "swa_sink.cu"],
     "chunked": ["prefill_chunked_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
+    "chunked_rope": ["prefill_chunked_sm100.cuh", "rope_sm100.cuh", "prefill_sm100.cuh",
+                     "ptx_sm100.cuh", "swa_sink.cu"],
     "decode": ["decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "decode_fp8": ["decode_fp8_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "splitkv": ["decode_splitkv_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
 }
 WORKLOAD_KERNEL = {"tiny_swa_prefill": "ring", "swa_prefill_32k": "ring",
-                   "swa_prefill_32k_rope": "ring_rope",
+                   "swa_prefill_32k_rope": "ring_rope", "global_prefill_8k_rope": "chunked_rope",
                    "varlen_swa_prefill": "ring", "global_prefill_8k": "chunked",
                    "swa_decode_mtp": "decode", "ga_decode_16k": "splitkv",
                    "swa_decode_mtp_fp8": "decode_fp8"}
@@ -208,6 +210,7 @@ class PrefillRunner:
             need = B.swa_sink_attn_fwd_rope_workspace(c["total"], c["Hq"], c["Hkv"], c["D"],
                                                       c["window"])
             self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+            self.rope_pass = need > 0  # a rotation pass into the workspace, then the prefill
         self.q, self.k, self.v = c["q"].to(dev), c["k"].to(dev), c["v"].to(dev)
         self.cu = c["cu_seqlens"].to(dev)
         self.sink = c["sink"].to(dev) if c["sink"] is not None else None
@@ -226,7 +229,7 @@ class PrefillRunner:
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
         self.units = c["total"]
-        self.launches_per_call = 2 if getattr(self, "full", False) else 1
+        self.launches_per_call = 2 if getattr(self, "rope_pass", False) else 1
 
     def call(self, stream):
         c = self.c
@@ -281,6 +284,7 @@ class DecodeRunner:
             need = B.swa_sink_decode_splitkv_workspace(d["B"], d["n_q"], d["Hq"], d["Hkv"],
                                                        d["D"], d["W"], self.max_ctx)
             self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+            self.rope_pass = need > 0  # a rotation pass into the workspace, then the prefill
         self.turn = 0
         self.o = torch.empty_like(self.g["q"])
         self.lse = torch.empty((d["B"], d["n_q"], d["Hq"]), dtype=torch.float32, device=dev)

@@ -63,9 +63,9 @@ class DecodeCase:
     kv: str = "bf16"
 
 
-# The workloads: a tiny parity case, one SWA layer (also with the rotary
-# embedding applied inside the call and the decode ring written), one global
-# layer, a packed
+# The workloads: a tiny parity case, one SWA layer and one global layer (each
+# also with the rotary embedding applied inside the call and the decode ring /
+# position-indexed cache written), a packed
 # varlen SWA batch, a decode / draft-verification batch of the SWA layers and
 # one of a global layer over long contexts.
 WORKLOADS = {
@@ -81,6 +81,9 @@ WORKLOADS = {
     "global_prefill_8k": PrefillCase(
         "global_prefill T=8192 Hq=64 Hkv=8 D=128 full-causal", [8192], 64, 8,
         128, 0, 0.5, "normal", 3),
+    "global_prefill_8k_rope": PrefillCase(
+        "global_prefill_rope T=8192 Hq=64 Hkv=8 D=128 full-causal rope_base=640000 cache=8192",
+        [8192], 64, 8, 128, 0, 0.5, "normal", 3, rope_base=640000.0, ring_W=8192),
     "varlen_swa_prefill": PrefillCase(
         "varlen_swa_prefill 16 seqs L~U[1024,16384] Hq=64 Hkv=8 D=128 W=128",
         [], 64, 8, 128, 128, 0.5, "normal", 4, varlen_draw=(16, 1024, 16384)),

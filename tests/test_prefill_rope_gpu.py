@@ -3,8 +3,9 @@
 same seeded inputs: the fused ring kernel (G = 8, 4, 2; D = 128 and 64) and
 the workspace path (global layers, wide windows, G = 1), both pairings,
 sequence start positions (pos0) up to the 2^24 limit, ragged and empty
-sequences; the ring it writes (rotated K within one bf16 ulp, V bit exact,
-other slots untouched); and the full SWA layer on sampled rows."""
+sequences; the ring it writes (rotated K equal to the oracle's bf16 values but
+for rare elements next to a rounding boundary, V bit exact, other slots
+untouched); and the full SWA layer on sampled rows."""
 import numpy as np
 import pytest
 import torch
@@ -43,25 +44,42 @@ def run(c, base, pos0=None, interleaved=False, ring_W=0, window=None):
     return o, lse, kr, vr
 
 
-def check_ring(c, kr_gpu, vr_gpu, k_rot_ref, W, pos0):
+def check_ring(c, kr_gpu, vr_gpu, k_rot_ref, W, pos0, interleaved):
     ring0 = np.full((len(c["seqlens"]), W, c["Hkv"], c["D"]), POISON, np.uint16)
     kr_ref, vr_ref = rope.emit_ring(k_rot_ref, c["v"], c["cu_seqlens"], ring0, ring0, W,
                                     pos0=pos0)
+    # the unrotated keys in ring order, for the error bound
+    k_in = rope.emit_ring(c["k"].view(torch.int16).numpy().view(np.uint16), c["v"],
+                          c["cu_seqlens"], ring0, ring0, W, pos0=pos0)[0]
     kg, vg = bits(kr_gpu), bits(vr_gpu)
     assert np.array_equal(vg, vr_ref)
-    # untouched slots keep the poison; written K within one bf16 ulp
-    assert np.array_equal(kg == POISON, kr_ref == POISON)
-    assert ulp_apart(kg, kr_ref).max() <= 1
-    assert (kg != kr_ref).mean() < 1e-3, (kg != kr_ref).mean()
+    # untouched slots keep the poison
+    written = kr_ref != POISON
+    assert np.array_equal(kg == POISON, ~written)
+    check_rotated(kg[written], kr_ref[written], pair_norm(k_in, interleaved)[written])
 
 
-def ulp_apart(a, b):
-    """Distance in bf16 steps between bit patterns (sign-magnitude mapped to
-    a monotone integer line, so -0 and +0 coincide)."""
-    def line(x):
-        x = x.astype(np.int64)
-        return np.where(x & 0x8000, -(x & 0x7FFF), x)
-    return np.abs(line(a) - line(b))
+def pair_norm(k_bits, interleaved):
+    """|(x_a, x_b)| of the pair each element belongs to (rotation keeps it)."""
+    x = rope.bits_to_f64(k_bits)
+    a, b = rope.rope_pairs(x.shape[-1], interleaved)
+    n = np.sqrt(x[..., a] ** 2 + x[..., b] ** 2)
+    out = np.empty_like(x)
+    out[..., a] = n
+    out[..., b] = n
+    return out
+
+
+def check_rotated(got_bits, ref_bits, norm):
+    """A rotated element is the oracle's correctly rounded bf16 value except
+    where fp32 arithmetic (angle error a few 1e-8 rad, products and sums a few
+    float ulps, all relative to the pair's norm) lands on the other side of a
+    rounding boundary: then it is within one bf16 ulp of the value plus
+    2e-6 of the pair's norm. Such elements are rare."""
+    g, r = rope.bits_to_f64(got_bits), rope.bits_to_f64(ref_bits)
+    bound = np.abs(r) * 2.0 ** -7 + 2e-6 * norm
+    assert np.all(np.abs(g - r) <= bound), np.abs(g - r).max()
+    assert (got_bits != ref_bits).mean() < 1e-3, (got_bits != ref_bits).mean()
 
 
 CASES = [  # (name, seqlens, Hq, Hkv, D, W, pos0, interleaved, ring_W)
@@ -90,7 +108,7 @@ def test_rope_prefill_matches_oracle(name, seqlens, Hq, Hkv, D, W, pos0, inter, 
                                          W, base, pos0=pos0, sink=c["sink"],
                                          interleaved=inter)
     check(o, lse, ro, rl, name)
-    check_ring(c, kr, vr, k_rot, ring_W, pos0)
+    check_ring(c, kr, vr, k_rot, ring_W, pos0, inter)
 
 
 def test_rope_equals_plain_prefill_on_rotated_inputs():
@@ -169,4 +187,30 @@ def test_rope_full_swa_layer_sampled():
     k_ref = rope.rope_bf16(c["k"][T - 128:], pos, 1e4)
     kg = bits(kr)[0][pos % 128]
     assert np.array_equal(bits(vr)[0][pos % 128], bits(c["v"][T - 128:]))
-    assert ulp_apart(kg, k_ref).max() <= 1
+    check_rotated(kg, k_ref, pair_norm(bits(c["k"][T - 128:]), False))
+
+
+def test_rope_full_global_layer_sampled():
+    """The benchmark's global layer (T=8192, full causal) with RoPE (base
+    640000) through the workspace path, writing a position-indexed cache of
+    8192 slots; sampled rows vs the oracle, the cache holds every token."""
+    c = wl.make_prefill(wl.WORKLOADS["global_prefill_8k_rope"])
+    base, W = c["rope_base"], c["ring_W"]
+    assert B.swa_sink_attn_fwd_rope_workspace(c["total"], 64, 8, 128, 0) > 0
+    o, lse, kr, vr = run(c, base, ring_W=W)
+    rng = np.random.default_rng(3)
+    toks = np.unique(np.concatenate([rng.integers(0, c["total"], 48), [0, 1, c["total"] - 1]]))
+    G = c["Hq"] // c["Hkv"]
+    heads = rng.integers(0, c["Hkv"], len(toks)) * G
+    rt = np.repeat(toks, G)
+    rh = (np.repeat(heads, G) + np.tile(np.arange(G), len(toks))).astype(np.int32)
+    ro, rl = rope.prefill_rope_rows(c["q"], c["k"], c["v"], c["cu_seqlens"], c["Hq"], c["Hkv"],
+                                    c["D"], 0, base, rt, rh, sink=c["sink"])
+    ti = torch.from_numpy(rt).cuda()
+    hi = torch.from_numpy(rh.astype(np.int64)).cuda()
+    check(o[ti, hi], lse[hi, ti], ro, rl, "global_prefill_8k rope")
+    assert torch.isfinite(o).all().item() and torch.isfinite(lse).all().item()
+    T = c["total"]
+    k_ref = rope.rope_bf16(c["k"], np.arange(T), base)
+    assert np.array_equal(bits(vr)[0], bits(c["v"]))
+    check_rotated(bits(kr)[0], k_ref, pair_norm(bits(c["k"]), False))
