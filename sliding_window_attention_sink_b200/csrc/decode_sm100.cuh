@@ -10,8 +10,8 @@
 // ring) and the new tokens 0..t.
 //
 // Design (sm_100a): one CTA per (sequence, kv head); split-free. 4 warps and
-// one buffer for K then V when the keys fit (KP <= 160: four CTAs share an
-// SM), else 8 warps and separate K and V buffers.
+// one buffer for K then V when the keys fit (KP <= 160: five CTAs share an
+// SM for a 128-slot ring), else 8 warps and separate K and V buffers.
 // * All G query heads of the kv head and all n_q tokens are one set of
 //   R = n_q * G query rows (32 for n_q = 4, G = 8), so each ring byte is read
 //   from HBM exactly once for all of them.
@@ -75,6 +75,21 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
+__device__ __forceinline__ void ldsm_x1_t(uint32_t addr, uint32_t& r0) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x1.trans.shared.b16 {%0}, [%1];"
+               : "=r"(r0)
+               : "r"(addr));
+}
+
+// D += A B on m16n8k8 (bf16 in, f32 accumulate): the last 8 keys of PV.
+__device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                           uint32_t a2, uint32_t a3, uint32_t b0,
                                           uint32_t b1) {
@@ -98,19 +113,25 @@ constexpr int kDecodeSmallWarps = 4;
 constexpr int kDecodeLargeWarps = 8;
 constexpr int kDecodeSmallMaxKP = 160;
 
-// Shared memory (from a 1024-byte aligned base): K and V (or one buffer for
-// both) as D/64 blocks of [KP rows][128 bytes]; Q as D/64 blocks of [32 rows]
-// [128 bytes] (128-byte swizzle: 16-byte unit u of row r at u ^ (r & 7)),
-// later overwritten by P [32][KP+8] bf16; then per-warp row maxima and the two
-// row sums [NWP][32] and per-row l [32] (fp32).
+// Shared memory (the dynamic region, 1024-byte aligned; no static shared
+// memory): K and V (or one buffer for both) as D/64 blocks of [KP rows][128
+// bytes]; Q as D/64 blocks of [32 rows][128 bytes] (128-byte swizzle: 16-byte
+// unit u of row r at u ^ (r & 7)), later overwritten by P [32][LDP] bf16;
+// then per-warp row maxima and the two row sums [NWP][32], per-row l [32]
+// (fp32), and the two mbarriers and the abort flag. KP is a multiple of 8;
+// P rows are KP + 8 apart when KP is a multiple of 16 (a 16-byte shift per
+// row keeps ldmatrix free of bank conflicts), else KP apart (already so).
+// With W = 128 and n_q <= 4 the 4-warp CTA takes 45 216 bytes: five share an SM.
+__host__ __device__ inline int decode_ldp(int KP) { return (KP % 16 == 8) ? KP : KP + 8; }
 __host__ __device__ inline size_t decode_qp_bytes(int D, int KP) {
   const size_t q = static_cast<size_t>(D / 64) * 32 * 128;
-  const size_t pb = static_cast<size_t>(32) * (KP + 8) * 2;
+  const size_t pb = static_cast<size_t>(32) * decode_ldp(KP) * 2;
   return q > pb ? q : pb;
 }
 __host__ __device__ inline size_t decode_smem_bytes(int D, int KP, int nwp) {
   const size_t kv = static_cast<size_t>(D / 64) * KP * 128 * (nwp == kDecodeSmallWarps ? 1 : 2);
-  return 1024 + kv + decode_qp_bytes(D, KP) + (static_cast<size_t>(nwp) * 32 * 3 + 32) * sizeof(float);
+  return kv + decode_qp_bytes(D, KP) + (static_cast<size_t>(nwp) * 32 * 3 + 32) * sizeof(float) +
+         32;
 }
 
 // Byte address of (row, col) in a tile stored as 64-column blocks of `rows`
@@ -121,7 +142,7 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t base, int rows, int row,
 }
 
 template <int D, int MT, int NWP>
-__global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
+__global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 5 : 2)
     decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_kr,
                         const __grid_constant__ CUtensorMap tm_kn,
@@ -135,22 +156,29 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
   constexpr int NTW = 5;           // max n8 key tiles per warp (KP <= 40 * NWP)
   constexpr int DW = D / NWP;      // PV: head-dim columns per warp
   constexpr int NTO = DW / 8;      // n8 tiles per warp in PV (1, 2 or 4)
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_qk, bar_v;
-  __shared__ int abort_sh;
-  volatile int* abort = &abort_sh;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int KP = p.KP;
-  const uint32_t sK = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sK = smem_u32(smem_raw);
   const uint32_t sV = SHARE ? sK : sK + NCH * KP * 128;
   const uint32_t sQ = sV + NCH * KP * 128;
   // P takes Q's place once S is done
-  __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(smem_raw + (sQ - smem_u32(smem_raw)));
-  const int LDP = KP + 8;
-  float* red_max = reinterpret_cast<float*>(smem_raw + (sQ - smem_u32(smem_raw)) +
+  __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(smem_raw + (sQ - sK));
+  const int LDP = decode_ldp(KP);
+  float* red_max = reinterpret_cast<float*>(smem_raw + (sQ - sK) +
                                               decode_qp_bytes(D, KP));  // [NWP][32]
   float* red_lr = red_max + NWP * 32;                         // [NWP][32]
   float* red_lx = red_lr + NWP * 32;                          // [NWP][32]
   float* row_l = red_lx + NWP * 32;                           // [32]
+  uint64_t& bar_qk = *reinterpret_cast<uint64_t*>(row_l + 32);
+  uint64_t& bar_v = *(&bar_qk + 1);
+  int& abort_sh = *reinterpret_cast<int*>(&bar_qk + 2);
+  volatile int* abort = &abort_sh;
+  // the swizzled TMA boxes need a 1024-byte aligned base (the region starts
+  // there when the kernel has no static shared memory)
+  if (sK & 1023u) {
+    if (threadIdx.x == 0) flag_error(2u);
+    return;
+  }
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.x / p.Hkv;
@@ -431,6 +459,7 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
     for (int jn = 0; jn < NTO; ++jn)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mt][jn][e] = 0.f;
+  // keys in steps of 16, then one step of 8 when KP is not a multiple of 16
   for (int kk = 0; kk < KP / 16; ++kk) {
     uint32_t a[MT][4];
 #pragma unroll
@@ -458,6 +487,20 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 4 : 2)
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
         mma_16816(acc[mt][0], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
+    }
+  }
+  if (KP % 16 == 8) {
+    const int k0 = KP - 8;
+    uint32_t a[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+      ldsm_x2(sP + ((mt * 16 + (lane & 15)) * LDP + k0) * 2, a[mt][0], a[mt][1]);
+#pragma unroll
+    for (int jn = 0; jn < NTO; ++jn) {
+      uint32_t b0;
+      ldsm_x1_t(sw128_addr(sV, KP, k0 + (lane & 7), warp * DW + jn * 8), b0);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) mma_1688(acc[mt][jn], a[mt][0], a[mt][1], b0);
     }
   }
 

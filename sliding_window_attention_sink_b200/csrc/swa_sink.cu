@@ -127,6 +127,24 @@ int ensure_smem_attr(K kernel, size_t bytes, size_t (&done)[kMaxDevices]) {
   return SWA_OK;
 }
 
+// Prefer the largest shared-memory carve-out of the unified L1 / shared
+// array for a kernel (once per device).
+template <typename K>
+int ensure_carveout(K kernel, bool (&done)[kMaxDevices]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail("cudaGetDevice", e);
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (!done[dev]) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             static_cast<int>(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(carveout)", e);
+    done[dev] = true;
+  }
+  return SWA_OK;
+}
+bool g_carve_dec[2][2][2][kMaxDevices];
+
 size_t g_attr_prefill64[kMaxDevices], g_attr_prefill128[kMaxDevices];
 size_t g_attr_dec[2][2][2][2][kMaxDevices];
 
@@ -459,6 +477,11 @@ int launch_decode(const swa::DecodeFp8Params& p, cudaStream_t st) {
     auto kern = swa::decode_sm100_kernel<D, MT, NWP>;
     if (ensure_smem_attr(kern, smem, attr) != SWA_OK)
       return SWA_ERR_CUDA;
+    // the whole unified L1 / shared array as shared memory, so that five
+    // 4-warp CTAs fit an SM
+    if (ensure_carveout(kern, g_carve_dec[D == 128][MT - 1][NWP == swa::kDecodeLargeWarps]) !=
+        SWA_OK)
+      return SWA_ERR_CUDA;
     kern<<<grid, NWP * 32, smem, st>>>(tq, tkr, tkn, tvr, tvn, to, p);
   }
   const cudaError_t e = cudaGetLastError();
@@ -519,7 +542,10 @@ int decode_impl(const void* q, const void* k_new, const void* v_new, const void*
   // the new tokens' columns start at a multiple of 8 (16 for an FP8 ring,
   // whose kernel gives them a 16-key block of their own)
   p.W8 = round_up(W, kv_scale ? 16 : 8);
-  p.KP = round_up(p.W8 + n_q, 16);
+  // keys padded to 16 for the FP8 ring's k16 steps; to 8 for the bf16 ring
+  // (its PV ends with a k8 step), which keeps its CTA small enough for five
+  // per SM
+  p.KP = round_up(p.W8 + n_q, kv_scale ? 16 : 8);
   p.sink = sink;
   p.scale_log2 = softmax_scale * swa::kLog2e;
   p.o = static_cast<__nv_bfloat16*>(o);
