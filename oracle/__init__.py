@@ -9,6 +9,8 @@ library never imports it, and it imports nothing from the product package.
 over a ring of E4M3 codes with per-kv-head scales (numpy, fp64).
 ``oracle.rope`` adds the rotary position embedding applied before the
 attention (fp64 rotation, bf16 rounding) and the ring the prefill writes.
+``oracle.backward`` adds the gradients of the prefill (dq, dk, dv and the
+sink's), whole or at sampled rows and keys.
 """
 from .oracle import (  # noqa: F401
     decode,
