@@ -195,6 +195,42 @@ SWA_API int swa_sink_attn_fwd_rope(const void *q, const void *k, const void *v,
                                    size_t workspace_bytes, void *o, float *lse, void *stream);
 
 /*
+ * Backward of swa_sink_attn_fwd: the gradients of q, k, v and of the sink for
+ * an output gradient dout.
+ *
+ * Source: the forward of section 2.2.2 of the report summary above; the
+ * pages give no backward (the ICML 2026 talk write-up's Q&A stresses that the
+ * sink's initialisation and gradient updates must stay stable at scale). With
+ * p_ij = exp(scale q_i.k_j - lse_i) over the visible keys and
+ * p_sink,i = exp(s_h - lse_i):
+ *   Delta_i = dout_i . o_i,   dS_ij = p_ij (dout_i . v_j - Delta_i)
+ *   dq_i = scale sum_j dS_ij k_j,   dk_j = scale sum_i dS_ij q_i,
+ *   dv_j = sum_i p_ij dout_i,       dsink_h = -sum_i p_sink,i Delta_i
+ * with dk, dv of a kv head summed over its Hq/Hkv query heads.
+ *
+ *   q, k, v, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq, Hkv, D,
+ *   window, sink, softmax_scale   as given to swa_sink_attn_fwd
+ *   o, lse      the forward's outputs (bf16 [total, Hq, D], fp32 [Hq, total]);
+ *               lse is required
+ *   dout        bf16 [total, Hq, D]
+ *   dq          bf16 [total, Hq, D] output; dk, dv bf16 [total, Hkv, D] outputs
+ *   dsink       fp32 [Hq] output (zero without a sink), or NULL
+ *   workspace   device memory of swa_sink_attn_bwd_workspace() bytes (Delta,
+ *               fp32 [Hq, total]), 16-byte aligned, owned by the caller; calls
+ *               that overlap in time need separate workspaces.
+ *   Hq/Hkv must divide 64; D 64 or 128.
+ *
+ * Returns SWA_OK or a negative swa_status_t.
+ */
+SWA_API size_t swa_sink_attn_bwd_workspace(int total_tokens, int Hq);
+SWA_API int swa_sink_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                              const void *dout, const float *lse, const int32_t *cu_seqlens,
+                              int num_seqs, int max_seqlen, int total_tokens, int Hq, int Hkv,
+                              int D, int window, const float *sink, float softmax_scale,
+                              void *dq, void *dk, void *dv, float *dsink, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+/*
  * Decode / draft verification over a W-slot KV ring per sequence.
  *
  * Source: section 2.3 "Lightweight MTP" of the report summary above (draft

@@ -52,6 +52,11 @@ def load():
     lib.swa_sink_attn_fwd_rope.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
                                            _f, _f, _i, _vp, _vp, _vp, _i, _vp, ctypes.c_size_t,
                                            _vp, _vp, _vp]
+    lib.swa_sink_attn_bwd_workspace.restype = ctypes.c_size_t
+    lib.swa_sink_attn_bwd_workspace.argtypes = [_i, _i]
+    lib.swa_sink_attn_bwd.restype = _i
+    lib.swa_sink_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                      _i, _vp, _f, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
     lib.swa_sink_attn_decode.restype = _i
     lib.swa_sink_attn_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                          _i, _vp, _f, _vp, _vp, _vp]
@@ -132,6 +137,20 @@ def swa_sink_attn_fwd_rope(q, k, v, cu_seqlens, num_seqs, max_seqlen, total_toke
         float(softmax_scale), float(rope_base), int(rope_interleaved), _ptr(pos0), _ptr(k_ring),
         _ptr(v_ring), int(ring_W), _ptr(workspace), int(workspace_bytes), _ptr(o), _ptr(lse),
         _stream(stream))
+
+
+def swa_sink_attn_bwd_workspace(total_tokens, Hq):
+    return load().swa_sink_attn_bwd_workspace(int(total_tokens), int(Hq))
+
+
+def swa_sink_attn_bwd(q, k, v, o, dout, lse, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq,
+                      Hkv, D, window, sink, softmax_scale, dq, dk, dv, dsink, workspace,
+                      workspace_bytes, stream=None):
+    return load().swa_sink_attn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(cu_seqlens),
+        int(num_seqs), int(max_seqlen), int(total_tokens), int(Hq), int(Hkv), int(D),
+        int(window), _ptr(sink), float(softmax_scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dsink),
+        _ptr(workspace), int(workspace_bytes), _stream(stream))
 
 
 def swa_sink_attn_decode(q, k_new, v_new, k_ring, v_ring, pos, B, n_q, Hq, Hkv, D, W, sink,
@@ -246,6 +265,28 @@ def attn_fwd_rope(q, k, v, cu_seqlens, window, rope_base, sink=None, pos0=None,
     if rc != SWA_OK:
         raise SwaSinkError(rc, "swa_sink_attn_fwd_rope")
     return out, lse
+
+
+def attn_bwd(q, k, v, o, lse, dout, cu_seqlens, window, sink=None, softmax_scale=0.0,
+             max_seqlen=None, want_dsink=True, workspace=None, stream=None):
+    """Gradients of attn_fwd: returns (dq, dk, dv, dsink or None) for the
+    forward's o and lse and the output gradient dout (bf16)."""
+    total, Hq, D = q.shape
+    Hkv = k.shape[1]
+    num_seqs = cu_seqlens.numel() - 1
+    if max_seqlen is None:
+        max_seqlen = total
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dsink = (torch.empty((Hq,), dtype=torch.float32, device=q.device) if want_dsink else None)
+    need = swa_sink_attn_bwd_workspace(total, Hq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = swa_sink_attn_bwd(q, k, v, o, dout, lse, cu_seqlens, num_seqs, max_seqlen, total, Hq,
+                           Hkv, D, window, sink, softmax_scale, dq, dk, dv, dsink, workspace,
+                           workspace.numel(), stream)
+    if rc != SWA_OK:
+        raise SwaSinkError(rc, "swa_sink_attn_bwd")
+    return dq, dk, dv, dsink
 
 
 def attn_decode(q, k_new, v_new, k_ring, v_ring, pos, sink=None, softmax_scale=0.0, out=None,

@@ -1,0 +1,402 @@
+// backward_sm100.cuh -- gradients of the sliding-window / global attention
+// with a per-head sink: dq, dk, dv and the sink's gradient.
+//
+// Operation: the calculus of the forward of "MiMo-V2-Flash Technical Report"
+// summary (mlpod.com), section 2.2.2 (the sink joins the softmax denominator
+// and its max; it has no value). With p_ij = exp(scale q_i.k_j - lse_i) over
+// the visible keys, p_sink,i = exp(s_h - lse_i), o_i = sum_j p_ij v_j and the
+// output gradient dO:
+//   Delta_i = dO_i . o_i
+//   dS_ij   = p_ij (dO_i . v_j - Delta_i)
+//   dq_i    = scale sum_j dS_ij k_j        dk_j = scale sum_i dS_ij q_i
+//   dv_j    = sum_i p_ij dO_i              dsink_h = -sum_i p_sink,i Delta_i
+// (the ICML talk write-up, hzrcw.cc, Q&A: the sink's gradient updates must
+// stay stable at scale). K and V gradients of a kv head sum over its G query
+// heads. P is recomputed from q, k and the forward's lse (fp32), as the
+// forward computed it.
+//
+// Three kernels, mma.sync m16n8k16 (bf16 in, fp32 accumulate) on
+// shared-memory tiles (rows padded by 16 bytes: ldmatrix without bank
+// conflicts):
+//   bwd_prep_kernel  Delta from o and dO (fp32, [Hq, total] in the caller's
+//                    workspace) and dsink (atomic adds into the zeroed output)
+//   bwd_dq_kernel    one CTA of 4 warps per (64 query rows = 64/G tokens x G
+//                    heads, kv head): key blocks of 32 over the rows' window;
+//                    per warp 16 rows: S and dP (16 x 32), dS, dq += dS K
+//   bwd_dkdv_kernel  one CTA of 4 warps per (64 keys, kv head): the query
+//                    rows that see them in chunks of 16 (tokens x G heads);
+//                    per warp 16 keys: S^T and dP^T (16 x 16), dv += P^T dO,
+//                    dk += dS^T q
+// No inter-CTA waits; no traps.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+#include "ptx_sm100.cuh"
+
+namespace swa {
+
+struct BwdParams {
+  const __nv_bfloat16 *q, *k, *v, *o, *dout;
+  const float* lse;  // [Hq, total], natural log
+  const int32_t* cu_seqlens;
+  int num_seqs, total, Hq, Hkv, G, window;
+  const float* sink;  // [Hq] or NULL
+  float scale, scale_log2;
+  float* delta;       // [Hq, total] (workspace)
+  __nv_bfloat16 *dq, *dk, *dv;
+  float* dsink;       // [Hq] or NULL; zero before bwd_prep_kernel
+};
+
+constexpr int kBwdPrepTokens = 8;  // tokens per prep CTA
+constexpr int kBwdQRows = 64;      // query rows per dq CTA
+constexpr int kBwdKeyBlock = 32;   // keys per dq step
+constexpr int kBwdKeys = 64;       // keys per dk/dv CTA
+constexpr int kBwdRowChunk = 16;   // query rows per dk/dv step
+
+__host__ __device__ inline size_t bwd_dq_smem_bytes(int D) {
+  return static_cast<size_t>(2 * kBwdQRows + 2 * kBwdKeyBlock) * (D + 8) * 2;
+}
+__host__ __device__ inline size_t bwd_dkdv_smem_bytes(int D) {
+  return static_cast<size_t>(2 * kBwdKeys + 2 * kBwdRowChunk) * (D + 8) * 2 +
+         4 * kBwdRowChunk * sizeof(float);
+}
+
+// First key visible to token t (same sequence, inside the window), and the
+// end of t's sequence.
+__device__ __forceinline__ void bwd_token_bounds(const BwdParams& p, int t, int& first, int& end) {
+  const int s = seq_of_token(p.cu_seqlens, p.num_seqs, t);
+  const int lo = __ldg(p.cu_seqlens + s);
+  end = __ldg(p.cu_seqlens + s + 1);
+  first = p.window > 0 ? max(lo, t - p.window + 1) : lo;
+}
+
+// Copy `rows` rows of D bf16 (16-byte pieces) into a padded shared tile;
+// src_row(r) gives the source row pointer or nullptr for a zero row.
+template <int D, typename F>
+__device__ __forceinline__ void bwd_load_rows(__nv_bfloat16* dst, int rows, F src_row) {
+  constexpr int U = D / 8;  // 16-byte pieces per row
+  for (int idx = threadIdx.x; idx < rows * U; idx += blockDim.x) {
+    const int r = idx / U, u = idx - r * U;
+    const __nv_bfloat16* s = src_row(r);
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (s != nullptr) val = __ldg(reinterpret_cast<const uint4*>(s) + u);
+    *reinterpret_cast<uint4*>(dst + r * (D + 8) + u * 8) = val;
+  }
+}
+
+__device__ __forceinline__ uint32_t bwd_smem_addr(const __nv_bfloat16* base, int row, int col,
+                                                  int ld) {
+  return smem_u32(base + row * ld + col);
+}
+
+// ---- Delta and dsink ------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * kBwdPrepTokens;
+  constexpr int E = D / 32;  // elements per lane (2 or 4)
+  for (int h = warp; h < p.Hq; h += 8) {
+    const float sk = p.sink != nullptr ? __ldg(p.sink + h) : -INFINITY;
+    float part = 0.f;
+    for (int t = t0; t < min(t0 + kBwdPrepTokens, p.total); ++t) {
+      const size_t off = (static_cast<size_t>(t) * p.Hq + h) * D + lane * E;
+      float acc = 0.f;
+      if constexpr (E == 4) {
+        const uint2 a = __ldg(reinterpret_cast<const uint2*>(p.o + off));
+        const uint2 b = __ldg(reinterpret_cast<const uint2*>(p.dout + off));
+        acc = bf16lo_to_f32(a.x) * bf16lo_to_f32(b.x) + bf16hi_to_f32(a.x) * bf16hi_to_f32(b.x) +
+              bf16lo_to_f32(a.y) * bf16lo_to_f32(b.y) + bf16hi_to_f32(a.y) * bf16hi_to_f32(b.y);
+      } else {
+        const uint32_t a = __ldg(reinterpret_cast<const uint32_t*>(p.o + off));
+        const uint32_t b = __ldg(reinterpret_cast<const uint32_t*>(p.dout + off));
+        acc = bf16lo_to_f32(a) * bf16lo_to_f32(b) + bf16hi_to_f32(a) * bf16hi_to_f32(b);
+      }
+#pragma unroll
+      for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+      const size_t li = static_cast<size_t>(h) * p.total + t;
+      if (lane == 0) p.delta[li] = acc;
+      if (sk != -INFINITY) part -= expf(sk - __ldg(p.lse + li)) * acc;
+    }
+    if (lane == 0 && p.dsink != nullptr && sk != -INFINITY) atomicAdd(p.dsink + h, part);
+  }
+}
+
+// ---- dq -------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
+  constexpr int LD = D + 8;
+  constexpr int NTD = D / 8;  // n8 tiles over the head dim
+  extern __shared__ __align__(16) uint8_t bwd_smem[];
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(bwd_smem);
+  __nv_bfloat16* sdO = sQ + kBwdQRows * LD;
+  __nv_bfloat16* sK = sdO + kBwdQRows * LD;
+  __nv_bfloat16* sV = sK + kBwdKeyBlock * LD;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int TQ = kBwdQRows / p.G;  // tokens per CTA
+  const int n_tiles = (p.total + TQ - 1) / TQ;
+  const int g = blockIdx.x / n_tiles;
+  const int t0 = (blockIdx.x - g * n_tiles) * TQ;
+
+  bwd_load_rows<D>(sQ, kBwdQRows, [&](int r) -> const __nv_bfloat16* {
+    const int t = t0 + r / p.G;
+    return t < p.total ? p.q + (static_cast<size_t>(t) * p.Hq + g * p.G + r % p.G) * D : nullptr;
+  });
+  bwd_load_rows<D>(sdO, kBwdQRows, [&](int r) -> const __nv_bfloat16* {
+    const int t = t0 + r / p.G;
+    return t < p.total ? p.dout + (static_cast<size_t>(t) * p.Hq + g * p.G + r % p.G) * D
+                       : nullptr;
+  });
+  // this thread's two rows (fragment rows lane/4 and lane/4 + 8 of its warp)
+  int tok[2], first[2];
+  float lse2[2], dlt[2];
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    const int r = warp * 16 + (lane >> 2) + hf * 8;
+    const int t = t0 + r / p.G;
+    tok[hf] = t < p.total ? t : -1;
+    first[hf] = 0x7fffffff;
+    lse2[hf] = 0.f;
+    dlt[hf] = 0.f;
+    if (t < p.total) {
+      int end;
+      bwd_token_bounds(p, t, first[hf], end);
+      const size_t li = static_cast<size_t>(g * p.G + r % p.G) * p.total + t;
+      lse2[hf] = __ldg(p.lse + li) * kLog2e;
+      dlt[hf] = p.delta[li];
+    }
+  }
+  // keys: from the first token's first visible key to the last token
+  int kmin, kend;
+  bwd_token_bounds(p, t0, kmin, kend);
+  const int kmax = min(t0 + TQ, p.total) - 1;
+
+  float acc[NTD][4];
+#pragma unroll
+  for (int n = 0; n < NTD; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+
+  for (int j0 = kmin; j0 <= kmax; j0 += kBwdKeyBlock) {
+    __syncthreads();  // the previous block's K and V are no longer read
+    bwd_load_rows<D>(sK, kBwdKeyBlock, [&](int r) -> const __nv_bfloat16* {
+      const int j = j0 + r;
+      return j <= kmax ? p.k + (static_cast<size_t>(j) * p.Hkv + g) * D : nullptr;
+    });
+    bwd_load_rows<D>(sV, kBwdKeyBlock, [&](int r) -> const __nv_bfloat16* {
+      const int j = j0 + r;
+      return j <= kmax ? p.v + (static_cast<size_t>(j) * p.Hkv + g) * D : nullptr;
+    });
+    __syncthreads();
+    // S = Q K^T and dP = dO V^T for this warp's 16 rows x 32 keys
+    float s[4][4], dp[4][4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t a[4], ao[4];
+      const int arow = warp * 16 + (lane & 15), acol = kk * 16 + (lane >> 4) * 8;
+      ldsm_x4(bwd_smem_addr(sQ, arow, acol, LD), a[0], a[1], a[2], a[3]);
+      ldsm_x4(bwd_smem_addr(sdO, arow, acol, LD), ao[0], ao[1], ao[2], ao[3]);
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        const int brow = np * 16 + (lane & 7) + (lane >> 4) * 8;
+        const int bcol = kk * 16 + ((lane >> 3) & 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(bwd_smem_addr(sK, brow, bcol, LD), b0, b1, b2, b3);
+        mma_16816(s[2 * np], a[0], a[1], a[2], a[3], b0, b1);
+        mma_16816(s[2 * np + 1], a[0], a[1], a[2], a[3], b2, b3);
+        ldsm_x4(bwd_smem_addr(sV, brow, bcol, LD), b0, b1, b2, b3);
+        mma_16816(dp[2 * np], ao[0], ao[1], ao[2], ao[3], b0, b1);
+        mma_16816(dp[2 * np + 1], ao[0], ao[1], ao[2], ao[3], b2, b3);
+      }
+    }
+    // dS = P (dP - Delta), P recomputed from the forward's lse; 0 off the mask
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int hf = e >> 1;
+        const int j = j0 + n * 8 + 2 * (lane & 3) + (e & 1);
+        const bool vis = tok[hf] >= 0 && j >= first[hf] && j <= tok[hf];
+        const float pr = vis ? ex2(fmaf(s[n][e], p.scale_log2, -lse2[hf])) : 0.f;
+        s[n][e] = pr * (dp[n][e] - dlt[hf]);
+      }
+    // dq += dS K over the block's 32 keys (two k16 steps)
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      const uint32_t a0 = pack_bf16x2(s[2 * ks][0], s[2 * ks][1]);
+      const uint32_t a1 = pack_bf16x2(s[2 * ks][2], s[2 * ks][3]);
+      const uint32_t a2 = pack_bf16x2(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+      const uint32_t a3 = pack_bf16x2(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+#pragma unroll
+      for (int np = 0; np < NTD / 2; ++np) {
+        const int krow = ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int kcol = np * 16 + (lane >> 4) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(bwd_smem_addr(sK, krow, kcol, LD), b0, b1, b2, b3);
+        mma_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
+        mma_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+  }
+  // dq = scale * acc -> bf16
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    if (tok[hf] < 0) continue;
+    const int r = warp * 16 + (lane >> 2) + hf * 8;
+    __nv_bfloat16* dst = p.dq + (static_cast<size_t>(tok[hf]) * p.Hq + g * p.G + r % p.G) * D;
+#pragma unroll
+    for (int n = 0; n < NTD; ++n)
+      *reinterpret_cast<uint32_t*>(dst + n * 8 + 2 * (lane & 3)) =
+          pack_bf16x2(acc[n][2 * hf] * p.scale, acc[n][2 * hf + 1] * p.scale);
+  }
+}
+
+// ---- dk, dv ---------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) bwd_dkdv_kernel(const BwdParams p) {
+  constexpr int LD = D + 8;
+  constexpr int NTD = D / 8;
+  extern __shared__ __align__(16) uint8_t bwd_smem[];
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(bwd_smem);
+  __nv_bfloat16* sV = sK + kBwdKeys * LD;
+  __nv_bfloat16* sQ = sV + kBwdKeys * LD;
+  __nv_bfloat16* sdO = sQ + kBwdRowChunk * LD;
+  float* rlse2 = reinterpret_cast<float*>(sdO + kBwdRowChunk * LD);
+  float* rdlt = rlse2 + kBwdRowChunk;
+  int* rtok = reinterpret_cast<int*>(rdlt + kBwdRowChunk);
+  int* rfirst = rtok + kBwdRowChunk;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (p.total + kBwdKeys - 1) / kBwdKeys;
+  const int g = blockIdx.x / n_tiles;
+  const int k0 = (blockIdx.x - g * n_tiles) * kBwdKeys;
+  const int klast = min(k0 + kBwdKeys, p.total) - 1;
+
+  bwd_load_rows<D>(sK, kBwdKeys, [&](int r) -> const __nv_bfloat16* {
+    const int j = k0 + r;
+    return j <= klast ? p.k + (static_cast<size_t>(j) * p.Hkv + g) * D : nullptr;
+  });
+  bwd_load_rows<D>(sV, kBwdKeys, [&](int r) -> const __nv_bfloat16* {
+    const int j = k0 + r;
+    return j <= klast ? p.v + (static_cast<size_t>(j) * p.Hkv + g) * D : nullptr;
+  });
+  // rows that see any of these keys: tokens k0 .. the last one that sees klast
+  int f_unused, end_last;
+  bwd_token_bounds(p, klast, f_unused, end_last);
+  const int i_hi = p.window > 0 ? min(klast + p.window - 1, end_last - 1) : end_last - 1;
+  const int n_rows = (i_hi - k0 + 1) * p.G;
+  // this thread's two keys (fragment rows lane/4 and lane/4 + 8 of its warp)
+  int key[2];
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) key[hf] = k0 + warp * 16 + (lane >> 2) + hf * 8;
+
+  float dk[NTD][4], dv[NTD][4];
+#pragma unroll
+  for (int n = 0; n < NTD; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
+
+  for (int r0 = 0; r0 < n_rows; r0 += kBwdRowChunk) {
+    __syncthreads();  // the previous chunk is no longer read
+    auto row_src = [&](const __nv_bfloat16* base, int r) -> const __nv_bfloat16* {
+      const int rr = r0 + r;
+      if (rr >= n_rows) return nullptr;
+      const int t = k0 + rr / p.G;
+      return base + (static_cast<size_t>(t) * p.Hq + g * p.G + rr % p.G) * D;
+    };
+    bwd_load_rows<D>(sQ, kBwdRowChunk, [&](int r) { return row_src(p.q, r); });
+    bwd_load_rows<D>(sdO, kBwdRowChunk, [&](int r) { return row_src(p.dout, r); });
+    if (threadIdx.x < kBwdRowChunk) {
+      const int rr = r0 + threadIdx.x;
+      int t = -1, first = 0x7fffffff;
+      float l2 = 0.f, d = 0.f;
+      if (rr < n_rows) {
+        t = k0 + rr / p.G;
+        int end;
+        bwd_token_bounds(p, t, first, end);
+        const size_t li = static_cast<size_t>(g * p.G + rr % p.G) * p.total + t;
+        l2 = __ldg(p.lse + li) * kLog2e;
+        d = p.delta[li];
+      }
+      rtok[threadIdx.x] = t;
+      rfirst[threadIdx.x] = first;
+      rlse2[threadIdx.x] = l2;
+      rdlt[threadIdx.x] = d;
+    }
+    __syncthreads();
+    // S^T = K Q^T and dP^T = V dO^T for this warp's 16 keys x 16 rows
+    float s[2][4], dp[2][4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t a[4], av[4];
+      const int arow = warp * 16 + (lane & 15), acol = kk * 16 + (lane >> 4) * 8;
+      ldsm_x4(bwd_smem_addr(sK, arow, acol, LD), a[0], a[1], a[2], a[3]);
+      ldsm_x4(bwd_smem_addr(sV, arow, acol, LD), av[0], av[1], av[2], av[3]);
+      const int brow = (lane & 7) + (lane >> 4) * 8;
+      const int bcol = kk * 16 + ((lane >> 3) & 1) * 8;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(bwd_smem_addr(sQ, brow, bcol, LD), b0, b1, b2, b3);
+      mma_16816(s[0], a[0], a[1], a[2], a[3], b0, b1);
+      mma_16816(s[1], a[0], a[1], a[2], a[3], b2, b3);
+      ldsm_x4(bwd_smem_addr(sdO, brow, bcol, LD), b0, b1, b2, b3);
+      mma_16816(dp[0], av[0], av[1], av[2], av[3], b0, b1);
+      mma_16816(dp[1], av[0], av[1], av[2], av[3], b2, b3);
+    }
+    // P^T and dS^T; 0 off the mask
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int rr = n * 8 + 2 * (lane & 3) + (e & 1);
+        const int j = key[e >> 1];
+        const int t = rtok[rr];
+        const bool vis = t >= 0 && j <= klast && j >= rfirst[rr] && j <= t;
+        const float pr = vis ? ex2(fmaf(s[n][e], p.scale_log2, -rlse2[rr])) : 0.f;
+        s[n][e] = pr;
+        dp[n][e] = pr * (dp[n][e] - rdlt[rr]);
+      }
+    // dv += P^T dO and dk += dS^T Q over the chunk's 16 rows (one k16 step)
+    const uint32_t pa0 = pack_bf16x2(s[0][0], s[0][1]), pa1 = pack_bf16x2(s[0][2], s[0][3]);
+    const uint32_t pa2 = pack_bf16x2(s[1][0], s[1][1]), pa3 = pack_bf16x2(s[1][2], s[1][3]);
+    const uint32_t da0 = pack_bf16x2(dp[0][0], dp[0][1]), da1 = pack_bf16x2(dp[0][2], dp[0][3]);
+    const uint32_t da2 = pack_bf16x2(dp[1][0], dp[1][1]), da3 = pack_bf16x2(dp[1][2], dp[1][3]);
+#pragma unroll
+    for (int np = 0; np < NTD / 2; ++np) {
+      const int brow = (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int bcol = np * 16 + (lane >> 4) * 8;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(bwd_smem_addr(sdO, brow, bcol, LD), b0, b1, b2, b3);
+      mma_16816(dv[2 * np], pa0, pa1, pa2, pa3, b0, b1);
+      mma_16816(dv[2 * np + 1], pa0, pa1, pa2, pa3, b2, b3);
+      ldsm_x4_t(bwd_smem_addr(sQ, brow, bcol, LD), b0, b1, b2, b3);
+      mma_16816(dk[2 * np], da0, da1, da2, da3, b0, b1);
+      mma_16816(dk[2 * np + 1], da0, da1, da2, da3, b2, b3);
+    }
+  }
+  // dk = scale * acc, dv -> bf16
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    const int j = key[hf];
+    if (j > klast) continue;
+    __nv_bfloat16* dkr = p.dk + (static_cast<size_t>(j) * p.Hkv + g) * D;
+    __nv_bfloat16* dvr = p.dv + (static_cast<size_t>(j) * p.Hkv + g) * D;
+#pragma unroll
+    for (int n = 0; n < NTD; ++n) {
+      const int c = n * 8 + 2 * (lane & 3);
+      *reinterpret_cast<uint32_t*>(dkr + c) =
+          pack_bf16x2(dk[n][2 * hf] * p.scale, dk[n][2 * hf + 1] * p.scale);
+      *reinterpret_cast<uint32_t*>(dvr + c) = pack_bf16x2(dv[n][2 * hf], dv[n][2 * hf + 1]);
+    }
+  }
+}
+
+}  // namespace swa

@@ -156,7 +156,8 @@ __global__ void __launch_bounds__(NWP * 32, NWP == kDecodeSmallWarps ? 5 : 2)
   constexpr int NTW = 5;           // max n8 key tiles per warp (KP <= 40 * NWP)
   constexpr int DW = D / NWP;      // PV: head-dim columns per warp
   constexpr int NTO = DW / 8;      // n8 tiles per warp in PV (1, 2 or 4)
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t decode_smem[];
+  uint8_t* smem_raw = decode_smem;
   const int KP = p.KP;
   const uint32_t sK = smem_u32(smem_raw);
   const uint32_t sV = SHARE ? sK : sK + NCH * KP * 128;

@@ -18,6 +18,7 @@
 #include <mutex>
 
 #include "../../include/swa_sink.h"
+#include "backward_sm100.cuh"
 #include "decode_fp8_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "decode_splitkv_sm100.cuh"
@@ -711,6 +712,108 @@ int fwd_rope_impl(const void* q, const void* k, const void* v, const int32_t* cu
                              softmax_scale, o, lse, st);
 }
 
+// ---- backward ---------------------------------------------------------------------
+size_t bwd_workspace_bytes(int total, int Hq) {
+  if (total <= 0 || Hq <= 0) return 0;
+  return (static_cast<size_t>(total) * Hq * sizeof(float) + 255) / 256 * 256;
+}
+
+size_t g_attr_bwd_dq[2][kMaxDevices], g_attr_bwd_dkdv[2][kMaxDevices];
+
+template <int D>
+int launch_bwd(const swa::BwdParams& p, cudaStream_t st) {
+  swa::bwd_prep_kernel<D><<<(p.total + swa::kBwdPrepTokens - 1) / swa::kBwdPrepTokens, 256, 0,
+                            st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("backward prep launch", e);
+  {
+    auto kern = swa::bwd_dq_kernel<D>;
+    const size_t smem = swa::bwd_dq_smem_bytes(D);
+    if (ensure_smem_attr(kern, smem, g_attr_bwd_dq[D == 128]) != SWA_OK) return SWA_ERR_CUDA;
+    const int TQ = swa::kBwdQRows / p.G;
+    const long long grid = static_cast<long long>((p.total + TQ - 1) / TQ) * p.Hkv;
+    if (grid > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+    kern<<<static_cast<unsigned>(grid), 128, smem, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("backward dq launch", e);
+  }
+  {
+    auto kern = swa::bwd_dkdv_kernel<D>;
+    const size_t smem = swa::bwd_dkdv_smem_bytes(D);
+    if (ensure_smem_attr(kern, smem, g_attr_bwd_dkdv[D == 128]) != SWA_OK) return SWA_ERR_CUDA;
+    const long long grid =
+        static_cast<long long>((p.total + swa::kBwdKeys - 1) / swa::kBwdKeys) * p.Hkv;
+    if (grid > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+    kern<<<static_cast<unsigned>(grid), 128, smem, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("backward dk/dv launch", e);
+  }
+  return SWA_OK;
+}
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+             int total_tokens, int Hq, int Hkv, int D, int window, const float* sink,
+             float softmax_scale, void* dq, void* dk, void* dv, float* dsink, void* workspace,
+             size_t workspace_bytes, void* stream) {
+  if (num_seqs < 0 || max_seqlen < 0 || total_tokens < 0 || Hq <= 0 || Hkv <= 0)
+    return SWA_ERR_SHAPE;
+  if (Hq % Hkv != 0) return SWA_ERR_SHAPE;
+  if (total_tokens > 0 && num_seqs == 0) return SWA_ERR_SHAPE;
+  if (max_seqlen > total_tokens) return SWA_ERR_SHAPE;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (swa::kBwdQRows % (Hq / Hkv) != 0) return SWA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (total_tokens == 0) {
+    if (dsink != nullptr) {
+      if (!aligned4(dsink)) return SWA_ERR_ALIGN;
+      const cudaError_t e = cudaMemsetAsync(dsink, 0, sizeof(float) * Hq, st);
+      if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync(dsink)", e);
+    }
+    return SWA_OK;
+  }
+  if (!q || !k || !v || !o || !dout || !lse || !cu_seqlens || !dq || !dk || !dv)
+    return SWA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return SWA_ERR_ALIGN;
+  if (!aligned4(cu_seqlens) || !aligned4(lse) || (sink && !aligned4(sink)) ||
+      (dsink && !aligned4(dsink)))
+    return SWA_ERR_ALIGN;
+  if (workspace == nullptr) return SWA_ERR_NULL;
+  if (workspace_bytes < bwd_workspace_bytes(total_tokens, Hq)) return SWA_ERR_SHAPE;
+  if (!aligned16(workspace)) return SWA_ERR_ALIGN;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
+  if (dsink != nullptr) {  // the prep kernel adds into it
+    const cudaError_t e = cudaMemsetAsync(dsink, 0, sizeof(float) * Hq, st);
+    if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync(dsink)", e);
+  }
+  swa::BwdParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.lse = lse;
+  p.cu_seqlens = cu_seqlens;
+  p.num_seqs = num_seqs;
+  p.total = total_tokens;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.window = window;
+  p.sink = sink;
+  p.scale = softmax_scale;
+  p.scale_log2 = softmax_scale * swa::kLog2e;
+  p.delta = static_cast<float*>(workspace);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dsink = dsink;
+  return D == 64 ? launch_bwd<64>(p, st) : launch_bwd<128>(p, st);
+}
+
 // ---- split-KV decode ------------------------------------------------------------
 // Ranges per (sequence, kv head) and their length: enough CTAs for a few waves
 // (a fixed target, so that the workspace size does not depend on the device),
@@ -795,6 +898,20 @@ int swa_sink_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   if (slot < 0 || slot >= kNoAllocSlots) return SWA_ERR_SHAPE;
   return fwd_impl(q, k, v, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq, Hkv, D, window,
                   sink, softmax_scale, o, lse, stream, slot);
+}
+
+size_t swa_sink_attn_bwd_workspace(int total_tokens, int Hq) {
+  return bwd_workspace_bytes(total_tokens, Hq);
+}
+
+int swa_sink_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, const int32_t* cu_seqlens, int num_seqs,
+                      int max_seqlen, int total_tokens, int Hq, int Hkv, int D, int window,
+                      const float* sink, float softmax_scale, void* dq, void* dk, void* dv,
+                      float* dsink, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, dout, lse, cu_seqlens, num_seqs, max_seqlen, total_tokens, Hq, Hkv,
+                  D, window, sink, softmax_scale, dq, dk, dv, dsink, workspace, workspace_bytes,
+                  stream);
 }
 
 size_t swa_sink_attn_fwd_rope_workspace(int total_tokens, int Hq, int Hkv, int D, int window) {

@@ -171,6 +171,12 @@ def make_decode(case: DecodeCase):
     return out
 
 
+def make_dout(shape, sigma=0.5, seed=0):
+    """An output gradient for the backward: N(0,1) * sigma rounded to bf16."""
+    g = torch.Generator().manual_seed(seed)
+    return _bf16(torch.randn(shape, generator=g) * sigma)
+
+
 def prefill_case(seqlens, Hq, Hkv, D, window, sigma=0.5, sink="normal", seed=0):
     """An ad-hoc prefill case (tests use it for edge shapes)."""
     return make_prefill(PrefillCase("adhoc", list(seqlens), Hq, Hkv, D, window,

@@ -200,3 +200,31 @@ def test_fwd_rope_workspace_sizes():
     assert ws(300, 2, 2, 64, 128) == (300 * 2 * 64 * 2 + 255) // 256 * 256 + 300 * 2 * 64 * 2
     assert ws(600, 8, 1, 64, 300) > 0          # window too wide for the ring
     assert ws(0, 64, 8, 128, 0) == 0
+
+
+def bwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, dout=FAKE, lse=FAKE, cu_seqlens=FAKE, num_seqs=1,
+             max_seqlen=8, total_tokens=8, Hq=8, Hkv=2, D=128, window=128, sink=None,
+             softmax_scale=0.0, dq=FAKE, dk=FAKE, dv=FAKE, dsink=None, workspace=FAKE,
+             workspace_bytes=1 << 20, stream=0)
+    a.update(kw)
+    return B.swa_sink_attn_bwd(**a)
+
+
+def test_bwd_argument_errors():
+    assert bwd(Hq=8, Hkv=3) == -2
+    assert bwd(total_tokens=-1) == -2
+    assert bwd(max_seqlen=9) == -2
+    assert bwd(D=96) == -3
+    assert bwd(Hq=96, Hkv=1) == -3          # Hq/Hkv must divide 64
+    assert bwd(lse=None) == -1
+    assert bwd(dout=None) == -1
+    assert bwd(dk=None) == -1
+    assert bwd(workspace=None) == -1
+    assert bwd(workspace_bytes=16) == -2
+    assert bwd(dq=FAKE + 8) == -4
+    assert bwd(lse=FAKE + 2) == -4
+    assert bwd(workspace=FAKE + 4) == -4
+    assert B.swa_sink_attn_bwd_workspace(8, 8) == 256
+    assert B.swa_sink_attn_bwd_workspace(32768, 64) == 32768 * 64 * 4
+    assert B.swa_sink_attn_bwd_workspace(0, 64) == 0

@@ -1,0 +1,153 @@
+"""GPU parity of swa_sink_attn_bwd (through the C ABI) against the backward
+oracle (oracle/backward.py, fp64 gradients of the exact function) on the same
+seeded inputs: whole layers on small shapes (sliding windows, global layers,
+packed sequences with empty and length-1 ones, GQA groups 1..8, head dims 64
+and 128, no sink, extreme sinks), and the full SWA and global layers at
+sampled rows and keys.
+
+Tolerance, from the arithmetic: the kernels take the forward's bf16 o (in
+Delta), round P and dS to bf16 for the tensor cores and round dq, dk, dv to
+bf16: three roundings of at most 2^-9 relative each on every term. The test
+bounds the largest error by 2e-2 of the reference's largest magnitude and the
+mean error by 6e-3 of its mean magnitude (measured: at most 5.2e-3 and 4.0e-3,
+the latter for a window of 1, where dP - Delta cancels most). dsink =
+-sum_i p_sink,i Delta_i cancels too: its error scales with
+S_h = sum_i p_sink,i sum_d |dout_id o_id| (each product of Delta off by up to
+2^-9 of itself through the bf16 o), and the test bounds it by 2^-9 S_h
+(measured: at most 1.7e-4 S_h).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import backward as ob
+from sliding_window_attention_sink_b200 import binding as B
+from sliding_window_attention_sink_b200 import workloads as wl
+
+from _parity import to_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def run_bwd(c, dout, sink="case"):
+    d = to_cuda(c)
+    s = d["sink"] if sink == "case" else sink
+    o, lse = B.attn_fwd(d["q"], d["k"], d["v"], d["cu_seqlens"], c["window"], sink=s,
+                        max_seqlen=c["max_seqlen"])
+    dq, dk, dv, ds = B.attn_bwd(d["q"], d["k"], d["v"], o, lse, dout.cuda(), d["cu_seqlens"],
+                                c["window"], sink=s, max_seqlen=c["max_seqlen"])
+    torch.cuda.synchronize()
+    assert B.swa_sink_device_error() == 0
+    return dq, dk, dv, ds
+
+
+def check_grad(got, ref, what):
+    g = got.float().cpu().numpy().astype(np.float64)
+    assert np.isfinite(g).all(), what
+    err = np.abs(g - ref)
+    scale_max = max(np.abs(ref).max(), 1e-30)
+    scale_mean = max(np.abs(ref).mean(), 1e-30)
+    stats = (float(err.max() / scale_max), float(err.mean() / scale_mean))
+    print("%s: max err / max|ref| %.3g, mean err / mean|ref| %.3g" % (what, *stats))
+    assert stats[0] <= 2e-2 and stats[1] <= 6e-3, (what, stats)
+    return stats
+
+
+def dsink_scale(c, dout, sink):
+    """S_h = sum_i p_sink,i sum_d |dout_id o_id| from the C oracle's forward."""
+    o, lse, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], c["Hq"], c["Hkv"],
+                               c["D"], c["window"], sink=sink)
+    return dsink_scale_from(o, lse, dout, sink)
+
+
+def dsink_scale_from(o, lse, dout, sink):
+    if sink is None:
+        return np.zeros(o.shape[1])
+    s = sink.double().numpy()
+    dO = dout.float().numpy().astype(np.float64)
+    absdot = np.einsum("thd,thd->ht", np.abs(dO), np.abs(o))
+    return (np.exp(s[:, None] - lse) * absdot).sum(axis=1)
+
+
+def check_dsink(got, ref, scale, what):
+    g = got.cpu().numpy().astype(np.float64)
+    err = np.abs(g - ref)
+    ratio = float((err / np.maximum(scale, 1e-30)).max()) if scale.any() else 0.0
+    print("%s: dsink error / S_h max %.3g" % (what, ratio))
+    assert np.all(err <= 2.0 ** -9 * scale + 1e-6), (what, ratio)
+
+
+SMALL = [  # (name, seqlens, Hq, Hkv, D, W, sink)
+    ("swa_g8", [300], 64, 8, 128, 128, "normal"),
+    ("swa_varlen", [100, 0, 257, 1, 33], 16, 2, 128, 128, "normal"),
+    ("global", [400], 16, 2, 128, 0, "normal"),
+    ("global_varlen_d64", [129, 300, 5], 8, 1, 64, 0, "uniform2"),
+    ("g4_w20", [200], 8, 2, 128, 20, "normal"),
+    ("g1_d64", [150], 2, 2, 64, 64, "normal"),
+    ("no_sink", [257], 8, 1, 128, 128, None),
+    ("w1", [70], 8, 1, 64, 1, "normal"),
+]
+
+
+@pytest.mark.parametrize("name,seqlens,Hq,Hkv,D,W,sink", SMALL, ids=[s[0] for s in SMALL])
+def test_backward_matches_oracle(name, seqlens, Hq, Hkv, D, W, sink):
+    c = wl.prefill_case(seqlens, Hq, Hkv, D, W, sigma=0.5, sink=sink, seed=21)
+    dout = wl.make_dout(c["q"].shape, seed=22)
+    dq, dk, dv, ds = run_bwd(c, dout)
+    rq, rk, rv, rs = ob.prefill_backward(c["q"], c["k"], c["v"], dout, c["cu_seqlens"], Hq, Hkv,
+                                         D, W, sink=c["sink"])
+    check_grad(dq, rq, name + " dq")
+    check_grad(dk, rk, name + " dk")
+    check_grad(dv, rv, name + " dv")
+    check_dsink(ds, rs, dsink_scale(c, dout, c["sink"]), name + " dsink")
+
+
+@pytest.mark.parametrize("sval", [6.0, -6.0])
+def test_backward_extreme_sinks(sval):
+    c = wl.prefill_case([200], 8, 1, 128, 128, sigma=0.5, sink=None, seed=23)
+    c["sink"] = torch.full((8,), sval)
+    dout = wl.make_dout(c["q"].shape, seed=24)
+    dq, dk, dv, ds = run_bwd(c, dout)
+    rq, rk, rv, rs = ob.prefill_backward(c["q"], c["k"], c["v"], dout, c["cu_seqlens"], 8, 1, 128,
+                                         128, sink=c["sink"])
+    for got, ref, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        check_grad(got, ref, "sink=%g %s" % (sval, n))
+    check_dsink(ds, rs, dsink_scale(c, dout, c["sink"]), "sink=%g dsink" % sval)
+
+
+@pytest.mark.parametrize("wname", ["swa_prefill_32k", "global_prefill_8k"])
+def test_backward_full_layers_sampled(wname):
+    """The full layers at sampled places: dq at whole query groups of sampled
+    tokens, dk / dv at sampled keys (for the global layer, keys near the end
+    of the sequence, whose rows the oracle can enumerate), dsink for the SWA
+    layer from the C oracle's forward over every row."""
+    c = wl.make_prefill(wl.WORKLOADS[wname])
+    dout = wl.make_dout(c["q"].shape, seed=25)
+    dq, dk, dv, ds = run_bwd(c, dout)
+    T, Hq, Hkv, D, W = c["total"], c["Hq"], c["Hkv"], c["D"], c["window"]
+    G = Hq // Hkv
+    rng = np.random.default_rng(5)
+    toks = np.unique(np.concatenate([rng.integers(0, T, 24), [0, 1, 127, T - 1]]))
+    gq = rng.integers(0, Hkv, len(toks))
+    rt = np.repeat(toks, G)
+    rh = (np.repeat(gq * G, G) + np.tile(np.arange(G), len(toks))).astype(np.int32)
+    if W > 0:
+        kt = np.unique(np.concatenate([rng.integers(0, T, 24), [0, 63, 64, T - 1]]))
+    else:
+        kt = np.unique(np.concatenate([rng.integers(T - 300, T, 8), [T - 1]]))
+    kh = rng.integers(0, Hkv, len(kt))
+    sq, sk, sv = ob.prefill_backward_rows(c["q"], c["k"], c["v"], dout, c["cu_seqlens"], Hq, Hkv,
+                                          D, W, rt, rh, kt, kh, sink=c["sink"])
+    ti, hi = torch.from_numpy(rt).cuda(), torch.from_numpy(rh.astype(np.int64)).cuda()
+    check_grad(dq[ti, hi], sq, wname + " dq")
+    ki, khi = torch.from_numpy(kt).cuda(), torch.from_numpy(kh.astype(np.int64)).cuda()
+    check_grad(dk[ki, khi], sk, wname + " dk")
+    check_grad(dv[ki, khi], sv, wname + " dv")
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t.float()).all().item()
+    if W > 0:
+        o, lse, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], Hq, Hkv, D, W,
+                                   sink=c["sink"])
+        check_dsink(ds, ob.dsink_from_forward(o, lse, dout, c["sink"]),
+                    dsink_scale_from(o, lse, dout, c["sink"]), wname + " dsink")
