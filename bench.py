@@ -55,6 +55,20 @@ def prefill_work(seqlens, Hq, Hkv, D, window):
     return flops, nbytes
 
 
+def backward_work(seqlens, Hq, Hkv, D, window):
+    """Algorithmic FLOPs and bytes of one backward call: FLOPs = 10*D*Hq*pairs
+    (five contractions over the visible pairs: S recomputed, dP = dO V^T,
+    dV = P^T dO, dQ = dS K, dK = dS^T Q); bytes = read q, k, v, o, dO, lse,
+    sink, cu_seqlens once + write dq, dk, dv, dsink once."""
+    f_fwd, _ = prefill_work(seqlens, Hq, Hkv, D, window)
+    total = sum(seqlens)
+    nbytes = (total * Hq * D * 2 * 4          # q, o, dO read; dq written
+              + total * Hkv * D * 2 * 4      # k, v read; dk, dv written
+              + Hq * total * 4               # lse read
+              + Hq * 4 * 2 + (len(seqlens) + 1) * 4)
+    return f_fwd * 5 // 2, nbytes
+
+
 def decode_work(pos, n_q, Hq, Hkv, D, W, kv_bytes=2, Hkv_scales=0):
     """FLOPs over visible pairs; bytes = the cached K/V rows of committed
     tokens (min(pos, W) per sequence, kv_bytes per element: 2 for bf16, 1 for
@@ -99,12 +113,15 @@ KERNEL_SOURCES = {
     "chunked": ["prefill_chunked_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "chunked_rope": ["prefill_chunked_sm100.cuh", "rope_sm100.cuh", "prefill_sm100.cuh",
                      "ptx_sm100.cuh", "swa_sink.cu"],
+    "backward": ["backward_sm100.cuh", "decode_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh",
+                 "swa_sink.cu"],
     "decode": ["decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "decode_fp8": ["decode_fp8_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "splitkv": ["decode_splitkv_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
 }
 WORKLOAD_KERNEL = {"tiny_swa_prefill": "ring", "swa_prefill_32k": "ring",
                    "swa_prefill_32k_rope": "ring_rope", "global_prefill_8k_rope": "chunked_rope",
+                   "swa_backward_32k": "backward", "global_backward_8k": "backward",
                    "varlen_swa_prefill": "ring", "global_prefill_8k": "chunked",
                    "swa_decode_mtp": "decode", "ga_decode_16k": "splitkv",
                    "swa_decode_mtp_fp8": "decode_fp8"}
@@ -198,6 +215,10 @@ class PrefillRunner:
         self.flops, self.bytes = prefill_work(c["seqlens"], c["Hq"], c["Hkv"], c["D"],
                                               c["window"])
         self.rope = c["rope_base"] > 0
+        self.backward = c["backward"]
+        if self.backward:
+            self.flops, self.bytes = backward_work(c["seqlens"], c["Hq"], c["Hkv"], c["D"],
+                                                   c["window"])
         dev = torch.device("cuda")
         self.k_ring = self.v_ring = self.ws = None
         if self.rope:
@@ -226,13 +247,41 @@ class PrefillRunner:
         self.h_out = [torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory(),
                       torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()]
         self.d_out = [self.o, self.lse]
+        if self.backward:
+            # the forward's o and lse (outside the timed region), then the
+            # backward's inputs and outputs
+            B.attn_fwd(self.q, self.k, self.v, self.cu, c["window"], sink=self.sink,
+                       max_seqlen=c["max_seqlen"], out=self.o, lse=self.lse)
+            torch.cuda.synchronize()
+            self.dout = c["dout"].to(dev)
+            self.dq, self.dk, self.dv = (torch.empty_like(self.q), torch.empty_like(self.k),
+                                         torch.empty_like(self.v))
+            self.dsink = torch.empty((c["Hq"],), dtype=torch.float32, device=dev)
+            need = B.swa_sink_attn_bwd_workspace(c["total"], c["Hq"])
+            self.bws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+            self.h_in += [self.o.cpu().pin_memory(), self.lse.cpu().pin_memory(),
+                          c["dout"].pin_memory()]
+            self.d_in += [self.o, self.lse, self.dout]
+            self.h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                          for t in (self.dq, self.dk, self.dv, self.dsink)]
+            self.d_out = [self.dq, self.dk, self.dv, self.dsink]
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
         self.units = c["total"]
         self.launches_per_call = 2 if getattr(self, "rope_pass", False) else 1
+        if self.backward:
+            self.launches_per_call = 3  # Delta / dsink, dq, dk and dv
 
     def call(self, stream):
         c = self.c
+        if self.backward:
+            rc = self.B.swa_sink_attn_bwd(
+                self.q, self.k, self.v, self.o, self.dout, self.lse, self.cu, len(c["seqlens"]),
+                c["max_seqlen"], c["total"], c["Hq"], c["Hkv"], c["D"], c["window"], self.sink,
+                0.0, self.dq, self.dk, self.dv, self.dsink, self.bws, self.bws.numel(), stream)
+            if rc != 0:
+                raise RuntimeError("swa_sink_attn_bwd: %s" % self.B.status_string(rc))
+            return
         if self.rope:
             rc = self.B.swa_sink_attn_fwd_rope(
                 self.q, self.k, self.v, self.cu, len(c["seqlens"]), c["max_seqlen"], c["total"],
@@ -254,6 +303,9 @@ class PrefillRunner:
                "num_seqs": len(c["seqlens"]), "tokens": c["total"]}
         if self.rope:
             out.update(rope_base=c["rope_base"], ring=c["ring_W"])
+        if self.backward:
+            out.update(pass_="backward")
+            out["pass"] = out.pop("pass_")
         return out
 
 
@@ -361,11 +413,23 @@ def oracle_sample(workload, wl, seconds, threads, seed=0):
         F, Bt = prefill_work(c["seqlens"], c["Hq"], c["Hkv"], c["D"], c["window"])
         total_rows = c["total"] * c["Hq"]
 
+        if c["backward"]:
+            F, Bt = backward_work(c["seqlens"], c["Hq"], c["Hkv"], c["D"], c["window"])
+            F, Bt = F * 3 // 5, Bt * 3 // 5  # the dq side the sample runs
+
         def run(n):
             rt = rng.integers(0, c["total"], n)
             rh = rng.integers(0, c["Hq"], n).astype(np.int32)
             t0 = time.perf_counter()
-            if c["rope_base"] > 0:
+            if c["backward"]:
+                # dq at n rows: three of the backward's five contractions
+                # (S, dP, dQ) over those rows' pairs
+                from oracle import backward as obw
+                obw.prefill_backward_rows(c["q"], c["k"], c["v"], c["dout"], c["cu_seqlens"],
+                                          c["Hq"], c["Hkv"], c["D"], c["window"], rt, rh,
+                                          np.zeros(0, np.int64), np.zeros(0, np.int64),
+                                          sink=c["sink"], nthreads=threads)
+            elif c["rope_base"] > 0:
                 from oracle import rope as orope
                 orope.prefill_rope_rows(c["q"], c["k"], c["v"], c["cu_seqlens"], c["Hq"],
                                         c["Hkv"], c["D"], c["window"], c["rope_base"], rt, rh,
@@ -375,7 +439,8 @@ def oracle_sample(workload, wl, seconds, threads, seed=0):
                                     c["D"], c["window"], rt, rh, sink=c["sink"],
                                     nthreads=threads)
             return time.perf_counter() - t0
-        unit = "random (token, head) rows"
+        unit = ("random (token, head) rows of dq (3 of the 5 backward contractions)"
+                if c["backward"] else "random (token, head) rows")
     else:
         d = _cached_inputs(workload, wl)
         fp8 = case.kv == "fp8"

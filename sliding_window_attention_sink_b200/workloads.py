@@ -39,6 +39,9 @@ class PrefillCase:
     # slots per sequence
     rope_base: float = 0.0
     ring_W: int = 0
+    # the backward of this layer (output gradient dout ~ N(0,1) * sigma, bf16,
+    # drawn with seed + 1; o and lse from the forward)
+    backward: bool = False
 
 
 @dataclass
@@ -65,7 +68,7 @@ class DecodeCase:
 
 # The workloads: a tiny parity case, one SWA layer and one global layer (each
 # also with the rotary embedding applied inside the call and the decode ring /
-# position-indexed cache written), a packed
+# position-indexed cache written, and each also backward), a packed
 # varlen SWA batch, a decode / draft-verification batch of the SWA layers and
 # one of a global layer over long contexts.
 WORKLOADS = {
@@ -84,6 +87,12 @@ WORKLOADS = {
     "global_prefill_8k_rope": PrefillCase(
         "global_prefill_rope T=8192 Hq=64 Hkv=8 D=128 full-causal rope_base=640000 cache=8192",
         [8192], 64, 8, 128, 0, 0.5, "normal", 3, rope_base=640000.0, ring_W=8192),
+    "swa_backward_32k": PrefillCase(
+        "swa_backward T=32768 Hq=64 Hkv=8 D=128 W=128", [32768], 64, 8, 128, 128, 0.5,
+        "normal", 2, backward=True),
+    "global_backward_8k": PrefillCase(
+        "global_backward T=8192 Hq=64 Hkv=8 D=128 full-causal", [8192], 64, 8, 128, 0, 0.5,
+        "normal", 3, backward=True),
     "varlen_swa_prefill": PrefillCase(
         "varlen_swa_prefill 16 seqs L~U[1024,16384] Hq=64 Hkv=8 D=128 W=128",
         [], 64, 8, 128, 128, 0.5, "normal", 4, varlen_draw=(16, 1024, 16384)),
@@ -144,7 +153,8 @@ def make_prefill(case: PrefillCase):
     return dict(q=q, k=k, v=v, cu_seqlens=cu, sink=sink, seqlens=seqlens,
                 total=total, Hq=case.Hq, Hkv=case.Hkv, D=case.D,
                 window=case.window, max_seqlen=max(seqlens) if seqlens else 0,
-                rope_base=case.rope_base, ring_W=case.ring_W)
+                rope_base=case.rope_base, ring_W=case.ring_W, backward=case.backward,
+                dout=(make_dout(q.shape, case.sigma, case.seed + 1) if case.backward else None))
 
 
 def make_decode(case: DecodeCase):
