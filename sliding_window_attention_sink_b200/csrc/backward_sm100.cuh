@@ -23,10 +23,10 @@
 //   bwd_dq_kernel    one CTA of 4 warps per (64 query rows = 64/G tokens x G
 //                    heads, kv head): key blocks of 32 over the rows' window;
 //                    per warp 16 rows: S and dP (16 x 32), dS, dq += dS K
-//   bwd_dkdv_kernel  one CTA of 4 warps per (64 keys, kv head): the query
-//                    rows that see them in chunks of 16 (tokens x G heads);
-//                    per warp 16 keys: S^T and dP^T (16 x 16), dv += P^T dO,
-//                    dk += dS^T q
+//   bwd_dkdv_kernel  one CTA of 8 warps per (128 keys, kv head): the query
+//                    rows that see them in chunks of 32 (tokens x G heads),
+//                    double-buffered with cp.async; per warp 16 keys: S^T
+//                    and dP^T (16 x 32), dv += P^T dO, dk += dS^T q
 // No inter-CTA waits; no traps.
 #pragma once
 #include <cuda_bf16.h>
@@ -53,15 +53,15 @@ struct BwdParams {
 constexpr int kBwdPrepTokens = 8;  // tokens per prep CTA
 constexpr int kBwdQRows = 64;      // query rows per dq CTA
 constexpr int kBwdKeyBlock = 32;   // keys per dq step
-constexpr int kBwdKeys = 64;       // keys per dk/dv CTA
-constexpr int kBwdRowChunk = 16;   // query rows per dk/dv step
+constexpr int kBwdKeys = 128;      // keys per dk/dv CTA (8 warps x 16)
+constexpr int kBwdRowChunk = 32;   // query rows per dk/dv step
 
 __host__ __device__ inline size_t bwd_dq_smem_bytes(int D) {
   return static_cast<size_t>(2 * kBwdQRows + 2 * kBwdKeyBlock) * (D + 8) * 2;
 }
 __host__ __device__ inline size_t bwd_dkdv_smem_bytes(int D) {
-  return static_cast<size_t>(2 * kBwdKeys + 2 * kBwdRowChunk) * (D + 8) * 2 +
-         4 * kBwdRowChunk * sizeof(float);
+  return static_cast<size_t>(2 * kBwdKeys + 4 * kBwdRowChunk) * (D + 8) * 2 +
+         2 * 4 * kBwdRowChunk * sizeof(float);
 }
 
 // First key visible to token t (same sequence, inside the window), and the
@@ -258,61 +258,70 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
 }
 
 // ---- dk, dv ---------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// One CTA of 8 warps per (128 keys, kv head); warp w owns keys 16w .. 16w+15
+// and accumulates their dk and dv (16 x D each) in registers. The rows that
+// see the keys come in chunks of 32 (tokens x G heads), double-buffered with
+// cp.async: the next chunk's q and dO rows land while this one is computed.
 template <int D>
-__global__ void __launch_bounds__(128) bwd_dkdv_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
   constexpr int LD = D + 8;
   constexpr int NTD = D / 8;
+  constexpr int KT = kBwdKeys, RC = kBwdRowChunk;
+  constexpr int U = D / 8;  // 16-byte pieces per row
   extern __shared__ __align__(16) uint8_t bwd_smem[];
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(bwd_smem);
-  __nv_bfloat16* sV = sK + kBwdKeys * LD;
-  __nv_bfloat16* sQ = sV + kBwdKeys * LD;
-  __nv_bfloat16* sdO = sQ + kBwdRowChunk * LD;
-  float* rlse2 = reinterpret_cast<float*>(sdO + kBwdRowChunk * LD);
-  float* rdlt = rlse2 + kBwdRowChunk;
-  int* rtok = reinterpret_cast<int*>(rdlt + kBwdRowChunk);
-  int* rfirst = rtok + kBwdRowChunk;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = (p.total + kBwdKeys - 1) / kBwdKeys;
+  __nv_bfloat16* sV = sK + KT * LD;
+  __nv_bfloat16* sQb = sV + KT * LD;     // [2][RC][LD]
+  __nv_bfloat16* sdOb = sQb + 2 * RC * LD;  // [2][RC][LD]
+  float* rlse2b = reinterpret_cast<float*>(sdOb + 2 * RC * LD);  // [2][RC]
+  float* rdltb = rlse2b + 2 * RC;
+  int* rtokb = reinterpret_cast<int*>(rdltb + 2 * RC);
+  int* rfirstb = rtokb + 2 * RC;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_tiles = (p.total + KT - 1) / KT;
   const int g = blockIdx.x / n_tiles;
-  const int k0 = (blockIdx.x - g * n_tiles) * kBwdKeys;
-  const int klast = min(k0 + kBwdKeys, p.total) - 1;
+  const int k0 = (blockIdx.x - g * n_tiles) * KT;
+  const int klast = min(k0 + KT, p.total) - 1;
 
-  bwd_load_rows<D>(sK, kBwdKeys, [&](int r) -> const __nv_bfloat16* {
-    const int j = k0 + r;
-    return j <= klast ? p.k + (static_cast<size_t>(j) * p.Hkv + g) * D : nullptr;
-  });
-  bwd_load_rows<D>(sV, kBwdKeys, [&](int r) -> const __nv_bfloat16* {
-    const int j = k0 + r;
-    return j <= klast ? p.v + (static_cast<size_t>(j) * p.Hkv + g) * D : nullptr;
-  });
   // rows that see any of these keys: tokens k0 .. the last one that sees klast
   int f_unused, end_last;
   bwd_token_bounds(p, klast, f_unused, end_last);
   const int i_hi = p.window > 0 ? min(klast + p.window - 1, end_last - 1) : end_last - 1;
   const int n_rows = (i_hi - k0 + 1) * p.G;
-  // this thread's two keys (fragment rows lane/4 and lane/4 + 8 of its warp)
-  int key[2];
-#pragma unroll
-  for (int hf = 0; hf < 2; ++hf) key[hf] = k0 + warp * 16 + (lane >> 2) + hf * 8;
+  const int n_chunks = (n_rows + RC - 1) / RC;
 
-  float dk[NTD][4], dv[NTD][4];
-#pragma unroll
-  for (int n = 0; n < NTD; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
-
-  for (int r0 = 0; r0 < n_rows; r0 += kBwdRowChunk) {
-    __syncthreads();  // the previous chunk is no longer read
-    auto row_src = [&](const __nv_bfloat16* base, int r) -> const __nv_bfloat16* {
-      const int rr = r0 + r;
-      if (rr >= n_rows) return nullptr;
-      const int t = k0 + rr / p.G;
-      return base + (static_cast<size_t>(t) * p.Hq + g * p.G + rr % p.G) * D;
-    };
-    bwd_load_rows<D>(sQ, kBwdRowChunk, [&](int r) { return row_src(p.q, r); });
-    bwd_load_rows<D>(sdO, kBwdRowChunk, [&](int r) { return row_src(p.dout, r); });
-    if (threadIdx.x < kBwdRowChunk) {
-      const int rr = r0 + threadIdx.x;
+  // chunk c of the rows into buffer c & 1 (q, dO by cp.async; row data by
+  // plain stores)
+  auto prefetch = [&](int c) {
+    const int bf = c & 1;
+    for (int idx = tid; idx < RC * U * 2; idx += blockDim.x) {
+      const int which = idx / (RC * U);  // 0: q, 1: dO
+      const int rem = idx - which * RC * U;
+      const int r = rem / U, u = rem - r * U;
+      const int rr = c * RC + r;
+      const bool ok = rr < n_rows;
+      const int t = k0 + (ok ? rr / p.G : 0);
+      const __nv_bfloat16* src = (which == 0 ? p.q : p.dout) +
+                                 (static_cast<size_t>(t) * p.Hq + g * p.G + (ok ? rr % p.G : 0)) * D +
+                                 u * 8;
+      __nv_bfloat16* dst = (which == 0 ? sQb : sdOb) + (bf * RC + r) * LD + u * 8;
+      cp_async16(smem_u32(dst), src, ok);
+    }
+    if (tid < RC) {
+      const int rr = c * RC + tid;
       int t = -1, first = 0x7fffffff;
       float l2 = 0.f, d = 0.f;
       if (rr < n_rows) {
@@ -323,16 +332,57 @@ __global__ void __launch_bounds__(128) bwd_dkdv_kernel(const BwdParams p) {
         l2 = __ldg(p.lse + li) * kLog2e;
         d = p.delta[li];
       }
-      rtok[threadIdx.x] = t;
-      rfirst[threadIdx.x] = first;
-      rlse2[threadIdx.x] = l2;
-      rdlt[threadIdx.x] = d;
+      rtokb[bf * RC + tid] = t;
+      rfirstb[bf * RC + tid] = first;
+      rlse2b[bf * RC + tid] = l2;
+      rdltb[bf * RC + tid] = d;
     }
-    __syncthreads();
-    // S^T = K Q^T and dP^T = V dO^T for this warp's 16 keys x 16 rows
-    float s[2][4], dp[2][4];
+  };
+
+  // K and V of the tile (part of the first group)
+  for (int idx = tid; idx < KT * U * 2; idx += blockDim.x) {
+    const int which = idx / (KT * U);
+    const int rem = idx - which * KT * U;
+    const int r = rem / U, u = rem - r * U;
+    const int j = k0 + r;
+    const bool ok = j <= klast;
+    const __nv_bfloat16* src =
+        (which == 0 ? p.k : p.v) + (static_cast<size_t>(ok ? j : k0) * p.Hkv + g) * D + u * 8;
+    cp_async16(smem_u32((which == 0 ? sK : sV) + r * LD + u * 8), src, ok);
+  }
+  prefetch(0);
+  cp_async_commit();
+
+  int key[2];
 #pragma unroll
-    for (int n = 0; n < 2; ++n)
+  for (int hf = 0; hf < 2; ++hf) key[hf] = k0 + warp * 16 + (lane >> 2) + hf * 8;
+
+  float dk[NTD][4], dv[NTD][4];
+#pragma unroll
+  for (int n = 0; n < NTD; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
+
+  for (int c = 0; c < n_chunks; ++c) {
+    if (c + 1 < n_chunks) {
+      prefetch(c + 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();  // chunk c (and K, V) landed; its row data are visible
+    const int bf = c & 1;
+    const __nv_bfloat16* sQ = sQb + bf * RC * LD;
+    const __nv_bfloat16* sdO = sdOb + bf * RC * LD;
+    const float* rlse2 = rlse2b + bf * RC;
+    const float* rdlt = rdltb + bf * RC;
+    const int* rtok = rtokb + bf * RC;
+    const int* rfirst = rfirstb + bf * RC;
+    // S^T = K Q^T and dP^T = V dO^T for this warp's 16 keys x 32 rows
+    float s[4][4], dp[4][4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.f;
 #pragma unroll
@@ -341,19 +391,22 @@ __global__ void __launch_bounds__(128) bwd_dkdv_kernel(const BwdParams p) {
       const int arow = warp * 16 + (lane & 15), acol = kk * 16 + (lane >> 4) * 8;
       ldsm_x4(bwd_smem_addr(sK, arow, acol, LD), a[0], a[1], a[2], a[3]);
       ldsm_x4(bwd_smem_addr(sV, arow, acol, LD), av[0], av[1], av[2], av[3]);
-      const int brow = (lane & 7) + (lane >> 4) * 8;
-      const int bcol = kk * 16 + ((lane >> 3) & 1) * 8;
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(bwd_smem_addr(sQ, brow, bcol, LD), b0, b1, b2, b3);
-      mma_16816(s[0], a[0], a[1], a[2], a[3], b0, b1);
-      mma_16816(s[1], a[0], a[1], a[2], a[3], b2, b3);
-      ldsm_x4(bwd_smem_addr(sdO, brow, bcol, LD), b0, b1, b2, b3);
-      mma_16816(dp[0], av[0], av[1], av[2], av[3], b0, b1);
-      mma_16816(dp[1], av[0], av[1], av[2], av[3], b2, b3);
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        const int brow = np * 16 + (lane & 7) + (lane >> 4) * 8;
+        const int bcol = kk * 16 + ((lane >> 3) & 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(bwd_smem_addr(sQ, brow, bcol, LD), b0, b1, b2, b3);
+        mma_16816(s[2 * np], a[0], a[1], a[2], a[3], b0, b1);
+        mma_16816(s[2 * np + 1], a[0], a[1], a[2], a[3], b2, b3);
+        ldsm_x4(bwd_smem_addr(sdO, brow, bcol, LD), b0, b1, b2, b3);
+        mma_16816(dp[2 * np], av[0], av[1], av[2], av[3], b0, b1);
+        mma_16816(dp[2 * np + 1], av[0], av[1], av[2], av[3], b2, b3);
+      }
     }
     // P^T and dS^T; 0 off the mask
 #pragma unroll
-    for (int n = 0; n < 2; ++n)
+    for (int n = 0; n < 4; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int rr = n * 8 + 2 * (lane & 3) + (e & 1);
@@ -364,24 +417,33 @@ __global__ void __launch_bounds__(128) bwd_dkdv_kernel(const BwdParams p) {
         s[n][e] = pr;
         dp[n][e] = pr * (dp[n][e] - rdlt[rr]);
       }
-    // dv += P^T dO and dk += dS^T Q over the chunk's 16 rows (one k16 step)
-    const uint32_t pa0 = pack_bf16x2(s[0][0], s[0][1]), pa1 = pack_bf16x2(s[0][2], s[0][3]);
-    const uint32_t pa2 = pack_bf16x2(s[1][0], s[1][1]), pa3 = pack_bf16x2(s[1][2], s[1][3]);
-    const uint32_t da0 = pack_bf16x2(dp[0][0], dp[0][1]), da1 = pack_bf16x2(dp[0][2], dp[0][3]);
-    const uint32_t da2 = pack_bf16x2(dp[1][0], dp[1][1]), da3 = pack_bf16x2(dp[1][2], dp[1][3]);
+    // dv += P^T dO and dk += dS^T Q over the chunk's 32 rows (two k16 steps)
 #pragma unroll
-    for (int np = 0; np < NTD / 2; ++np) {
-      const int brow = (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int bcol = np * 16 + (lane >> 4) * 8;
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(bwd_smem_addr(sdO, brow, bcol, LD), b0, b1, b2, b3);
-      mma_16816(dv[2 * np], pa0, pa1, pa2, pa3, b0, b1);
-      mma_16816(dv[2 * np + 1], pa0, pa1, pa2, pa3, b2, b3);
-      ldsm_x4_t(bwd_smem_addr(sQ, brow, bcol, LD), b0, b1, b2, b3);
-      mma_16816(dk[2 * np], da0, da1, da2, da3, b0, b1);
-      mma_16816(dk[2 * np + 1], da0, da1, da2, da3, b2, b3);
+    for (int ks = 0; ks < 2; ++ks) {
+      const uint32_t pa0 = pack_bf16x2(s[2 * ks][0], s[2 * ks][1]);
+      const uint32_t pa1 = pack_bf16x2(s[2 * ks][2], s[2 * ks][3]);
+      const uint32_t pa2 = pack_bf16x2(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+      const uint32_t pa3 = pack_bf16x2(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+      const uint32_t da0 = pack_bf16x2(dp[2 * ks][0], dp[2 * ks][1]);
+      const uint32_t da1 = pack_bf16x2(dp[2 * ks][2], dp[2 * ks][3]);
+      const uint32_t da2 = pack_bf16x2(dp[2 * ks + 1][0], dp[2 * ks + 1][1]);
+      const uint32_t da3 = pack_bf16x2(dp[2 * ks + 1][2], dp[2 * ks + 1][3]);
+#pragma unroll
+      for (int np = 0; np < NTD / 2; ++np) {
+        const int brow = ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int bcol = np * 16 + (lane >> 4) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(bwd_smem_addr(sdO, brow, bcol, LD), b0, b1, b2, b3);
+        mma_16816(dv[2 * np], pa0, pa1, pa2, pa3, b0, b1);
+        mma_16816(dv[2 * np + 1], pa0, pa1, pa2, pa3, b2, b3);
+        ldsm_x4_t(bwd_smem_addr(sQ, brow, bcol, LD), b0, b1, b2, b3);
+        mma_16816(dk[2 * np], da0, da1, da2, da3, b0, b1);
+        mma_16816(dk[2 * np + 1], da0, da1, da2, da3, b2, b3);
+      }
     }
+    __syncthreads();  // buffer bf is read: the prefetch two chunks on may overwrite it
   }
+  cp_async_wait<0>();
   // dk = scale * acc, dv -> bf16
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {

@@ -744,7 +744,7 @@ int launch_bwd(const swa::BwdParams& p, cudaStream_t st) {
     const long long grid =
         static_cast<long long>((p.total + swa::kBwdKeys - 1) / swa::kBwdKeys) * p.Hkv;
     if (grid > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
-    kern<<<static_cast<unsigned>(grid), 128, smem, st>>>(p);
+    kern<<<static_cast<unsigned>(grid), 256, smem, st>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("backward dk/dv launch", e);
   }
