@@ -97,28 +97,43 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kBwdPrepTokens;
+  const int nt = min(kBwdPrepTokens, p.total - t0);
   constexpr int E = D / 32;  // elements per lane (2 or 4)
   for (int h = warp; h < p.Hq; h += 8) {
     const float sk = p.sink != nullptr ? __ldg(p.sink + h) : -INFINITY;
-    float part = 0.f;
-    for (int t = t0; t < min(t0 + kBwdPrepTokens, p.total); ++t) {
-      const size_t off = (static_cast<size_t>(t) * p.Hq + h) * D + lane * E;
-      float acc = 0.f;
-      if constexpr (E == 4) {
-        const uint2 a = __ldg(reinterpret_cast<const uint2*>(p.o + off));
-        const uint2 b = __ldg(reinterpret_cast<const uint2*>(p.dout + off));
-        acc = bf16lo_to_f32(a.x) * bf16lo_to_f32(b.x) + bf16hi_to_f32(a.x) * bf16hi_to_f32(b.x) +
-              bf16lo_to_f32(a.y) * bf16lo_to_f32(b.y) + bf16hi_to_f32(a.y) * bf16hi_to_f32(b.y);
-      } else {
-        const uint32_t a = __ldg(reinterpret_cast<const uint32_t*>(p.o + off));
-        const uint32_t b = __ldg(reinterpret_cast<const uint32_t*>(p.dout + off));
-        acc = bf16lo_to_f32(a) * bf16lo_to_f32(b) + bf16hi_to_f32(a) * bf16hi_to_f32(b);
-      }
+    // every token's loads first, then the dot products and their reductions
+    float acc[kBwdPrepTokens];
 #pragma unroll
-      for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-      const size_t li = static_cast<size_t>(h) * p.total + t;
-      if (lane == 0) p.delta[li] = acc;
-      if (sk != -INFINITY) part -= expf(sk - __ldg(p.lse + li)) * acc;
+    for (int u = 0; u < kBwdPrepTokens; ++u) {
+      acc[u] = 0.f;
+      if (u < nt) {
+        const size_t off = (static_cast<size_t>(t0 + u) * p.Hq + h) * D + lane * E;
+        if constexpr (E == 4) {
+          const uint2 a = __ldg(reinterpret_cast<const uint2*>(p.o + off));
+          const uint2 b = __ldg(reinterpret_cast<const uint2*>(p.dout + off));
+          acc[u] = bf16lo_to_f32(a.x) * bf16lo_to_f32(b.x) +
+                   bf16hi_to_f32(a.x) * bf16hi_to_f32(b.x) +
+                   bf16lo_to_f32(a.y) * bf16lo_to_f32(b.y) +
+                   bf16hi_to_f32(a.y) * bf16hi_to_f32(b.y);
+        } else {
+          const uint32_t a = __ldg(reinterpret_cast<const uint32_t*>(p.o + off));
+          const uint32_t b = __ldg(reinterpret_cast<const uint32_t*>(p.dout + off));
+          acc[u] = bf16lo_to_f32(a) * bf16lo_to_f32(b) + bf16hi_to_f32(a) * bf16hi_to_f32(b);
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1)
+#pragma unroll
+      for (int u = 0; u < kBwdPrepTokens; ++u) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], m);
+    float part = 0.f;
+#pragma unroll
+    for (int u = 0; u < kBwdPrepTokens; ++u) {
+      if (u < nt) {
+        const size_t li = static_cast<size_t>(h) * p.total + t0 + u;
+        if (lane == 0) p.delta[li] = acc[u];
+        if (sk != -INFINITY) part -= expf(sk - __ldg(p.lse + li)) * acc[u];
+      }
     }
     if (lane == 0 && p.dsink != nullptr && sk != -INFINITY) atomicAdd(p.dsink + h, part);
   }
@@ -190,6 +205,17 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
       return j <= kmax ? p.v + (static_cast<size_t>(j) * p.Hkv + g) * D : nullptr;
     });
     __syncthreads();
+    // a block none of this warp's 16 rows sees adds nothing: skip its MMAs
+    // (warp-uniform: from the rows' first keys and tokens)
+    {
+      int fmin = min(first[0], first[1]), tmax = max(tok[0], tok[1]);
+#pragma unroll
+      for (int m = 4; m < 32; m <<= 1) {
+        fmin = min(fmin, __shfl_xor_sync(0xffffffffu, fmin, m));
+        tmax = max(tmax, __shfl_xor_sync(0xffffffffu, tmax, m));
+      }
+      if (tmax < j0 || fmin > j0 + kBwdKeyBlock - 1) continue;
+    }
     // S = Q K^T and dP = dO V^T for this warp's 16 rows x 32 keys
     float s[4][4], dp[4][4];
 #pragma unroll
@@ -379,6 +405,21 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
     const float* rdlt = rdltb + bf * RC;
     const int* rtok = rtokb + bf * RC;
     const int* rfirst = rfirstb + bf * RC;
+    // a block wholly off the band (every row of the chunk sees none of this
+    // warp's keys) adds nothing: the warp skips its MMAs (the decision is the
+    // same for the whole warp: it depends on the chunk's tokens and the
+    // warp's keys only)
+    {
+      const int t_first = rtok[0];
+      const int t_last = rtok[RC - 1] >= 0 ? rtok[RC - 1] : p.total - 1;
+      const int kw0 = k0 + warp * 16, kw1 = min(kw0 + 15, klast);
+      const bool none = kw0 > klast || t_last < kw0 ||
+                        (p.window > 0 && t_first > kw1 + p.window - 1);
+      if (none) {
+        __syncthreads();
+        continue;
+      }
+    }
     // S^T = K Q^T and dP^T = V dO^T for this warp's 16 keys x 32 rows
     float s[4][4], dp[4][4];
 #pragma unroll
