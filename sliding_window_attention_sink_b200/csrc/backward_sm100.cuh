@@ -21,8 +21,9 @@
 //   bwd_prep_kernel  Delta from o and dO (fp32, [Hq, total] in the caller's
 //                    workspace) and dsink (atomic adds into the zeroed output)
 //   bwd_dq_kernel    one CTA of 4 warps per (64 query rows = 64/G tokens x G
-//                    heads, kv head): key blocks of 32 over the rows' window;
-//                    per warp 16 rows: S and dP (16 x 32), dS, dq += dS K
+//                    heads, kv head): key blocks of 32 over the rows' window,
+//                    double-buffered with cp.async; per warp 16 rows: S and
+//                    dP (16 x 32), dS, dq += dS K
 //   bwd_dkdv_kernel  one CTA of 8 warps per (128 keys, kv head): the query
 //                    rows that see them in chunks of 32 (tokens x G heads),
 //                    double-buffered with cp.async; per warp 16 keys: S^T
@@ -57,7 +58,7 @@ constexpr int kBwdKeys = 128;      // keys per dk/dv CTA (8 warps x 16)
 constexpr int kBwdRowChunk = 32;   // query rows per dk/dv step
 
 __host__ __device__ inline size_t bwd_dq_smem_bytes(int D) {
-  return static_cast<size_t>(2 * kBwdQRows + 2 * kBwdKeyBlock) * (D + 8) * 2;
+  return static_cast<size_t>(2 * kBwdQRows + 4 * kBwdKeyBlock) * (D + 8) * 2;
 }
 __host__ __device__ inline size_t bwd_dkdv_smem_bytes(int D) {
   return static_cast<size_t>(2 * kBwdKeys + 4 * kBwdRowChunk) * (D + 8) * 2 +
@@ -90,6 +91,24 @@ __device__ __forceinline__ void bwd_load_rows(__nv_bfloat16* dst, int rows, F sr
 __device__ __forceinline__ uint32_t bwd_smem_addr(const __nv_bfloat16* base, int row, int col,
                                                   int ld) {
   return smem_u32(base + row * ld + col);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ---- Delta and dsink ------------------------------------------------------------
@@ -144,26 +163,52 @@ template <int D>
 __global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
   constexpr int LD = D + 8;
   constexpr int NTD = D / 8;  // n8 tiles over the head dim
+  constexpr int U = D / 8;    // 16-byte pieces per row
+  constexpr int KB = kBwdKeyBlock;
   extern __shared__ __align__(16) uint8_t bwd_smem[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(bwd_smem);
   __nv_bfloat16* sdO = sQ + kBwdQRows * LD;
-  __nv_bfloat16* sK = sdO + kBwdQRows * LD;
-  __nv_bfloat16* sV = sK + kBwdKeyBlock * LD;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __nv_bfloat16* sKb = sdO + kBwdQRows * LD;  // [2][KB][LD]
+  __nv_bfloat16* sVb = sKb + 2 * KB * LD;     // [2][KB][LD]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int TQ = kBwdQRows / p.G;  // tokens per CTA
   const int n_tiles = (p.total + TQ - 1) / TQ;
   const int g = blockIdx.x / n_tiles;
   const int t0 = (blockIdx.x - g * n_tiles) * TQ;
 
-  bwd_load_rows<D>(sQ, kBwdQRows, [&](int r) -> const __nv_bfloat16* {
+  // the Q and dO rows of the tile (first cp.async group, with key block 0)
+  for (int idx = tid; idx < kBwdQRows * U * 2; idx += blockDim.x) {
+    const int which = idx / (kBwdQRows * U);
+    const int rem = idx - which * kBwdQRows * U;
+    const int r = rem / U, u = rem - r * U;
     const int t = t0 + r / p.G;
-    return t < p.total ? p.q + (static_cast<size_t>(t) * p.Hq + g * p.G + r % p.G) * D : nullptr;
-  });
-  bwd_load_rows<D>(sdO, kBwdQRows, [&](int r) -> const __nv_bfloat16* {
-    const int t = t0 + r / p.G;
-    return t < p.total ? p.dout + (static_cast<size_t>(t) * p.Hq + g * p.G + r % p.G) * D
-                       : nullptr;
-  });
+    const bool ok = t < p.total;
+    const __nv_bfloat16* src = (which == 0 ? p.q : p.dout) +
+                               (static_cast<size_t>(ok ? t : t0) * p.Hq + g * p.G + r % p.G) * D +
+                               u * 8;
+    cp_async16(smem_u32((which == 0 ? sQ : sdO) + r * LD + u * 8), src, ok);
+  }
+  // keys: from the first token's first visible key to the last token
+  int kmin, kend;
+  bwd_token_bounds(p, t0, kmin, kend);
+  const int kmax = min(t0 + TQ, p.total) - 1;
+  const int n_blocks = (kmax - kmin) / KB + 1;
+  auto load_block = [&](int bl) {
+    const int j0 = kmin + bl * KB, bf = bl & 1;
+    for (int idx = tid; idx < KB * U * 2; idx += blockDim.x) {
+      const int which = idx / (KB * U);
+      const int rem = idx - which * KB * U;
+      const int r = rem / U, u = rem - r * U;
+      const int j = j0 + r;
+      const bool ok = j <= kmax;
+      const __nv_bfloat16* src =
+          (which == 0 ? p.k : p.v) + (static_cast<size_t>(ok ? j : kmin) * p.Hkv + g) * D + u * 8;
+      cp_async16(smem_u32((which == 0 ? sKb : sVb) + (bf * KB + r) * LD + u * 8), src, ok);
+    }
+  };
+  load_block(0);
+  cp_async_commit();
+
   // this thread's two rows (fragment rows lane/4 and lane/4 + 8 of its warp)
   int tok[2], first[2];
   float lse2[2], dlt[2];
@@ -183,10 +228,14 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
       dlt[hf] = p.delta[li];
     }
   }
-  // keys: from the first token's first visible key to the last token
-  int kmin, kend;
-  bwd_token_bounds(p, t0, kmin, kend);
-  const int kmax = min(t0 + TQ, p.total) - 1;
+  // the key range of this warp's rows (warp-uniform): blocks outside it are
+  // skipped
+  int fmin = min(first[0], first[1]), tmax = max(tok[0], tok[1]);
+#pragma unroll
+  for (int m = 4; m < 32; m <<= 1) {
+    fmin = min(fmin, __shfl_xor_sync(0xffffffffu, fmin, m));
+    tmax = max(tmax, __shfl_xor_sync(0xffffffffu, tmax, m));
+  }
 
   float acc[NTD][4];
 #pragma unroll
@@ -194,81 +243,74 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
 
-  for (int j0 = kmin; j0 <= kmax; j0 += kBwdKeyBlock) {
-    __syncthreads();  // the previous block's K and V are no longer read
-    bwd_load_rows<D>(sK, kBwdKeyBlock, [&](int r) -> const __nv_bfloat16* {
-      const int j = j0 + r;
-      return j <= kmax ? p.k + (static_cast<size_t>(j) * p.Hkv + g) * D : nullptr;
-    });
-    bwd_load_rows<D>(sV, kBwdKeyBlock, [&](int r) -> const __nv_bfloat16* {
-      const int j = j0 + r;
-      return j <= kmax ? p.v + (static_cast<size_t>(j) * p.Hkv + g) * D : nullptr;
-    });
-    __syncthreads();
-    // a block none of this warp's 16 rows sees adds nothing: skip its MMAs
-    // (warp-uniform: from the rows' first keys and tokens)
-    {
-      int fmin = min(first[0], first[1]), tmax = max(tok[0], tok[1]);
-#pragma unroll
-      for (int m = 4; m < 32; m <<= 1) {
-        fmin = min(fmin, __shfl_xor_sync(0xffffffffu, fmin, m));
-        tmax = max(tmax, __shfl_xor_sync(0xffffffffu, tmax, m));
-      }
-      if (tmax < j0 || fmin > j0 + kBwdKeyBlock - 1) continue;
+  for (int bl = 0; bl < n_blocks; ++bl) {
+    if (bl + 1 < n_blocks) {
+      load_block(bl + 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    // S = Q K^T and dP = dO V^T for this warp's 16 rows x 32 keys
-    float s[4][4], dp[4][4];
+    __syncthreads();  // block bl (and, first time, the Q / dO rows) landed
+    const int j0 = kmin + bl * KB;
+    const __nv_bfloat16* sK = sKb + (bl & 1) * KB * LD;
+    const __nv_bfloat16* sV = sVb + (bl & 1) * KB * LD;
+    if (!(tmax < j0 || fmin > j0 + KB - 1)) {
+      // S = Q K^T and dP = dO V^T for this warp's 16 rows x 32 keys
+      float s[4][4], dp[4][4];
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+      for (int n = 0; n < 4; ++n)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.f;
+        for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t a[4], ao[4];
-      const int arow = warp * 16 + (lane & 15), acol = kk * 16 + (lane >> 4) * 8;
-      ldsm_x4(bwd_smem_addr(sQ, arow, acol, LD), a[0], a[1], a[2], a[3]);
-      ldsm_x4(bwd_smem_addr(sdO, arow, acol, LD), ao[0], ao[1], ao[2], ao[3]);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t a[4], ao[4];
+        const int arow = warp * 16 + (lane & 15), acol = kk * 16 + (lane >> 4) * 8;
+        ldsm_x4(bwd_smem_addr(sQ, arow, acol, LD), a[0], a[1], a[2], a[3]);
+        ldsm_x4(bwd_smem_addr(sdO, arow, acol, LD), ao[0], ao[1], ao[2], ao[3]);
 #pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        const int brow = np * 16 + (lane & 7) + (lane >> 4) * 8;
-        const int bcol = kk * 16 + ((lane >> 3) & 1) * 8;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(bwd_smem_addr(sK, brow, bcol, LD), b0, b1, b2, b3);
-        mma_16816(s[2 * np], a[0], a[1], a[2], a[3], b0, b1);
-        mma_16816(s[2 * np + 1], a[0], a[1], a[2], a[3], b2, b3);
-        ldsm_x4(bwd_smem_addr(sV, brow, bcol, LD), b0, b1, b2, b3);
-        mma_16816(dp[2 * np], ao[0], ao[1], ao[2], ao[3], b0, b1);
-        mma_16816(dp[2 * np + 1], ao[0], ao[1], ao[2], ao[3], b2, b3);
+        for (int np = 0; np < 2; ++np) {
+          const int brow = np * 16 + (lane & 7) + (lane >> 4) * 8;
+          const int bcol = kk * 16 + ((lane >> 3) & 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(bwd_smem_addr(sK, brow, bcol, LD), b0, b1, b2, b3);
+          mma_16816(s[2 * np], a[0], a[1], a[2], a[3], b0, b1);
+          mma_16816(s[2 * np + 1], a[0], a[1], a[2], a[3], b2, b3);
+          ldsm_x4(bwd_smem_addr(sV, brow, bcol, LD), b0, b1, b2, b3);
+          mma_16816(dp[2 * np], ao[0], ao[1], ao[2], ao[3], b0, b1);
+          mma_16816(dp[2 * np + 1], ao[0], ao[1], ao[2], ao[3], b2, b3);
+        }
       }
-    }
-    // dS = P (dP - Delta), P recomputed from the forward's lse; 0 off the mask
+      // dS = P (dP - Delta), P recomputed from the forward's lse; 0 off the mask
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+      for (int n = 0; n < 4; ++n)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int hf = e >> 1;
-        const int j = j0 + n * 8 + 2 * (lane & 3) + (e & 1);
-        const bool vis = tok[hf] >= 0 && j >= first[hf] && j <= tok[hf];
-        const float pr = vis ? ex2(fmaf(s[n][e], p.scale_log2, -lse2[hf])) : 0.f;
-        s[n][e] = pr * (dp[n][e] - dlt[hf]);
-      }
-    // dq += dS K over the block's 32 keys (two k16 steps)
+        for (int e = 0; e < 4; ++e) {
+          const int hf = e >> 1;
+          const int j = j0 + n * 8 + 2 * (lane & 3) + (e & 1);
+          const bool vis = tok[hf] >= 0 && j >= first[hf] && j <= tok[hf];
+          const float pr = vis ? ex2(fmaf(s[n][e], p.scale_log2, -lse2[hf])) : 0.f;
+          s[n][e] = pr * (dp[n][e] - dlt[hf]);
+        }
+      // dq += dS K over the block's 32 keys (two k16 steps)
 #pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      const uint32_t a0 = pack_bf16x2(s[2 * ks][0], s[2 * ks][1]);
-      const uint32_t a1 = pack_bf16x2(s[2 * ks][2], s[2 * ks][3]);
-      const uint32_t a2 = pack_bf16x2(s[2 * ks + 1][0], s[2 * ks + 1][1]);
-      const uint32_t a3 = pack_bf16x2(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+      for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t a0 = pack_bf16x2(s[2 * ks][0], s[2 * ks][1]);
+        const uint32_t a1 = pack_bf16x2(s[2 * ks][2], s[2 * ks][3]);
+        const uint32_t a2 = pack_bf16x2(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+        const uint32_t a3 = pack_bf16x2(s[2 * ks + 1][2], s[2 * ks + 1][3]);
 #pragma unroll
-      for (int np = 0; np < NTD / 2; ++np) {
-        const int krow = ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int kcol = np * 16 + (lane >> 4) * 8;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(bwd_smem_addr(sK, krow, kcol, LD), b0, b1, b2, b3);
-        mma_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
-        mma_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+        for (int np = 0; np < NTD / 2; ++np) {
+          const int krow = ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int kcol = np * 16 + (lane >> 4) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(bwd_smem_addr(sK, krow, kcol, LD), b0, b1, b2, b3);
+          mma_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
+          mma_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+        }
       }
     }
+    __syncthreads();  // buffer bl & 1 is read: the load two blocks on may overwrite it
   }
   // dq = scale * acc -> bf16
 #pragma unroll
@@ -284,19 +326,6 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
 }
 
 // ---- dk, dv ---------------------------------------------------------------------
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // One CTA of 8 warps per (128 keys, kv head); warp w owns keys 16w .. 16w+15
 // and accumulates their dk and dv (16 x D each) in registers. The rows that
 // see the keys come in chunks of 32 (tokens x G heads), double-buffered with
@@ -312,7 +341,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
   __nv_bfloat16* sV = sK + KT * LD;
   __nv_bfloat16* sQb = sV + KT * LD;     // [2][RC][LD]
   __nv_bfloat16* sdOb = sQb + 2 * RC * LD;  // [2][RC][LD]
-  float* rlse2b = reinterpret_cast<float*>(sdOb + 2 * RC * LD);  // [2][RC]
+  float* rlse2b = reinterpret_cast<float*>(sdOb + 2 * RC * LD);  // [2][RC] lse (natural log)
   float* rdltb = rlse2b + 2 * RC;
   int* rtokb = reinterpret_cast<int*>(rdltb + 2 * RC);
   int* rfirstb = rtokb + 2 * RC;
@@ -328,6 +357,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
   const int i_hi = p.window > 0 ? min(klast + p.window - 1, end_last - 1) : end_last - 1;
   const int n_rows = (i_hi - k0 + 1) * p.G;
   const int n_chunks = (n_rows + RC - 1) / RC;
+  int c_lo = 0, c_hi = -1;  // sequence of the last row token looked up
 
   // chunk c of the rows into buffer c & 1 (q, dO by cp.async; row data by
   // plain stores)
@@ -347,21 +377,26 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
       cp_async16(smem_u32(dst), src, ok);
     }
     if (tid < RC) {
+      // the row's token and first key (sequence bounds cached across chunks:
+      // tokens only grow), its lse and Delta by cp.async like the rows
       const int rr = c * RC + tid;
+      const bool ok = rr < n_rows;
       int t = -1, first = 0x7fffffff;
-      float l2 = 0.f, d = 0.f;
-      if (rr < n_rows) {
+      size_t li = 0;
+      if (ok) {
         t = k0 + rr / p.G;
-        int end;
-        bwd_token_bounds(p, t, first, end);
-        const size_t li = static_cast<size_t>(g * p.G + rr % p.G) * p.total + t;
-        l2 = __ldg(p.lse + li) * kLog2e;
-        d = p.delta[li];
+        if (t >= c_hi) {
+          const int sq = seq_of_token(p.cu_seqlens, p.num_seqs, t);
+          c_lo = __ldg(p.cu_seqlens + sq);
+          c_hi = __ldg(p.cu_seqlens + sq + 1);
+        }
+        first = p.window > 0 ? max(c_lo, t - p.window + 1) : c_lo;
+        li = static_cast<size_t>(g * p.G + rr % p.G) * p.total + t;
       }
       rtokb[bf * RC + tid] = t;
       rfirstb[bf * RC + tid] = first;
-      rlse2b[bf * RC + tid] = l2;
-      rdltb[bf * RC + tid] = d;
+      cp_async4(smem_u32(rlse2b + bf * RC + tid), p.lse + li, ok);
+      cp_async4(smem_u32(rdltb + bf * RC + tid), p.delta + li, ok);
     }
   };
 
@@ -454,7 +489,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
         const int j = key[e >> 1];
         const int t = rtok[rr];
         const bool vis = t >= 0 && j <= klast && j >= rfirst[rr] && j <= t;
-        const float pr = vis ? ex2(fmaf(s[n][e], p.scale_log2, -rlse2[rr])) : 0.f;
+        const float pr = vis ? ex2(fmaf(s[n][e], p.scale_log2, -rlse2[rr] * kLog2e)) : 0.f;
         s[n][e] = pr;
         dp[n][e] = pr * (dp[n][e] - rdlt[rr]);
       }
