@@ -173,8 +173,10 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int TQ = kBwdQRows / p.G;  // tokens per CTA
   const int n_tiles = (p.total + TQ - 1) / TQ;
-  const int g = blockIdx.x / n_tiles;
-  const int t0 = (blockIdx.x - g * n_tiles) * TQ;
+  // the last query tiles (the most keys, in a global layer) first, all kv
+  // heads of a tile together
+  const int g = blockIdx.x % p.Hkv;
+  const int t0 = (n_tiles - 1 - static_cast<int>(blockIdx.x) / p.Hkv) * TQ;
 
   // the Q and dO rows of the tile (first cp.async group, with key block 0)
   for (int idx = tid; idx < kBwdQRows * U * 2; idx += blockDim.x) {
@@ -346,9 +348,10 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
   int* rtokb = reinterpret_cast<int*>(rdltb + 2 * RC);
   int* rfirstb = rtokb + 2 * RC;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_tiles = (p.total + KT - 1) / KT;
-  const int g = blockIdx.x / n_tiles;
-  const int k0 = (blockIdx.x - g * n_tiles) * KT;
+  // the first key tiles (the most rows, in a global layer) first, all kv
+  // heads of a tile together
+  const int g = blockIdx.x % p.Hkv;
+  const int k0 = (static_cast<int>(blockIdx.x) / p.Hkv) * KT;
   const int klast = min(k0 + KT, p.total) - 1;
 
   // rows that see any of these keys: tokens k0 .. the last one that sees klast
