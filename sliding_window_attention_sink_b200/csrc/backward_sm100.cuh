@@ -19,7 +19,9 @@
 // shared-memory tiles (rows padded by 16 bytes: ldmatrix without bank
 // conflicts):
 //   bwd_prep_kernel  Delta from o and dO (fp32, [Hq, total] in the caller's
-//                    workspace) and dsink (atomic adds into the zeroed output)
+//                    workspace; coalesced 16-byte loads of whole rows) and
+//                    dsink (per-CTA sums in shared memory, then atomic adds
+//                    into the zeroed output)
 //   bwd_dq_kernel    one CTA of 4 warps per (64 query rows = 64/G tokens x G
 //                    heads, kv head): key blocks of 32 over the rows' window,
 //                    double-buffered with cp.async; per warp 16 rows: S and
@@ -51,7 +53,7 @@ struct BwdParams {
   float* dsink;       // [Hq] or NULL; zero before bwd_prep_kernel
 };
 
-constexpr int kBwdPrepTokens = 8;  // tokens per prep CTA
+constexpr int kBwdPrepTokens = 16;  // tokens per prep CTA
 constexpr int kBwdQRows = 64;      // query rows per dq CTA
 constexpr int kBwdKeyBlock = 32;   // keys per dq step
 constexpr int kBwdKeys = 128;      // keys per dk/dv CTA (8 warps x 16)
@@ -112,50 +114,60 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // ---- Delta and dsink ------------------------------------------------------------
+// Rows (token, head) are contiguous in o and dO: D/8 lanes take one row in
+// 16-byte pieces (coalesced), four rows per group in flight; dsink partials
+// gather per head in shared memory, one atomic add per head per CTA.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * kBwdPrepTokens;
-  const int nt = min(kBwdPrepTokens, p.total - t0);
-  constexpr int E = D / 32;  // elements per lane (2 or 4)
-  for (int h = warp; h < p.Hq; h += 8) {
-    const float sk = p.sink != nullptr ? __ldg(p.sink + h) : -INFINITY;
-    // every token's loads first, then the dot products and their reductions
-    float acc[kBwdPrepTokens];
+  constexpr int LPR = D / 8;          // lanes per row
+  constexpr int RPW = 32 / LPR;       // rows per warp per step
+  constexpr int RPS = 8 * RPW;        // rows per CTA per step
+  constexpr int UNR = 4;              // steps in flight
+  extern __shared__ float prep_sink[];  // [Hq]
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int sub = lane / LPR, pl = lane - sub * LPR;
+  const long long row0 = static_cast<long long>(blockIdx.x) * kBwdPrepTokens * p.Hq;
+  const long long row_end =
+      min(row0 + static_cast<long long>(kBwdPrepTokens) * p.Hq,
+          static_cast<long long>(p.total) * p.Hq);
+  for (int h = tid; h < p.Hq; h += blockDim.x) prep_sink[h] = 0.f;
+  __syncthreads();
+  const long long my0 = row0 + (tid >> 5) * RPW + sub;
+  for (long long base = my0; base < row_end; base += static_cast<long long>(RPS) * UNR) {
+    uint4 a[UNR], b[UNR];
 #pragma unroll
-    for (int u = 0; u < kBwdPrepTokens; ++u) {
-      acc[u] = 0.f;
-      if (u < nt) {
-        const size_t off = (static_cast<size_t>(t0 + u) * p.Hq + h) * D + lane * E;
-        if constexpr (E == 4) {
-          const uint2 a = __ldg(reinterpret_cast<const uint2*>(p.o + off));
-          const uint2 b = __ldg(reinterpret_cast<const uint2*>(p.dout + off));
-          acc[u] = bf16lo_to_f32(a.x) * bf16lo_to_f32(b.x) +
-                   bf16hi_to_f32(a.x) * bf16hi_to_f32(b.x) +
-                   bf16lo_to_f32(a.y) * bf16lo_to_f32(b.y) +
-                   bf16hi_to_f32(a.y) * bf16hi_to_f32(b.y);
-        } else {
-          const uint32_t a = __ldg(reinterpret_cast<const uint32_t*>(p.o + off));
-          const uint32_t b = __ldg(reinterpret_cast<const uint32_t*>(p.dout + off));
-          acc[u] = bf16lo_to_f32(a) * bf16lo_to_f32(b) + bf16hi_to_f32(a) * bf16hi_to_f32(b);
-        }
+    for (int u = 0; u < UNR; ++u) {
+      const long long row = base + static_cast<long long>(u) * RPS;
+      a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (row < row_end) {
+        a[u] = __ldg(reinterpret_cast<const uint4*>(p.o + row * D) + pl);
+        b[u] = __ldg(reinterpret_cast<const uint4*>(p.dout + row * D) + pl);
       }
     }
 #pragma unroll
-    for (int m = 16; m > 0; m >>= 1)
+    for (int u = 0; u < UNR; ++u) {
+      const uint32_t av[4] = {a[u].x, a[u].y, a[u].z, a[u].w};
+      const uint32_t bv[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
+      float acc = 0.f;
 #pragma unroll
-      for (int u = 0; u < kBwdPrepTokens; ++u) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], m);
-    float part = 0.f;
+      for (int e = 0; e < 4; ++e)
+        acc += bf16lo_to_f32(av[e]) * bf16lo_to_f32(bv[e]) +
+               bf16hi_to_f32(av[e]) * bf16hi_to_f32(bv[e]);
 #pragma unroll
-    for (int u = 0; u < kBwdPrepTokens; ++u) {
-      if (u < nt) {
-        const size_t li = static_cast<size_t>(h) * p.total + t0 + u;
-        if (lane == 0) p.delta[li] = acc[u];
-        if (sk != -INFINITY) part -= expf(sk - __ldg(p.lse + li)) * acc[u];
+      for (int m = LPR / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+      const long long row = base + static_cast<long long>(u) * RPS;
+      if (pl == 0 && row < row_end) {
+        const int t = static_cast<int>(row / p.Hq), h = static_cast<int>(row - t * p.Hq);
+        const size_t li = static_cast<size_t>(h) * p.total + t;
+        p.delta[li] = acc;
+        if (p.sink != nullptr)
+          atomicAdd(&prep_sink[h], -expf(__ldg(p.sink + h) - __ldg(p.lse + li)) * acc);
       }
     }
-    if (lane == 0 && p.dsink != nullptr && sk != -INFINITY) atomicAdd(p.dsink + h, part);
   }
+  __syncthreads();
+  if (p.dsink != nullptr && p.sink != nullptr)
+    for (int h = tid; h < p.Hq; h += blockDim.x) atomicAdd(p.dsink + h, prep_sink[h]);
 }
 
 // ---- dq -------------------------------------------------------------------------

@@ -722,8 +722,8 @@ size_t g_attr_bwd_dq[2][kMaxDevices], g_attr_bwd_dkdv[2][kMaxDevices];
 
 template <int D>
 int launch_bwd(const swa::BwdParams& p, cudaStream_t st) {
-  swa::bwd_prep_kernel<D><<<(p.total + swa::kBwdPrepTokens - 1) / swa::kBwdPrepTokens, 256, 0,
-                            st>>>(p);
+  swa::bwd_prep_kernel<D><<<(p.total + swa::kBwdPrepTokens - 1) / swa::kBwdPrepTokens, 256,
+                            sizeof(float) * p.Hq, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("backward prep launch", e);
   {
@@ -763,6 +763,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   if (max_seqlen > total_tokens) return SWA_ERR_SHAPE;
   if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
   if (swa::kBwdQRows % (Hq / Hkv) != 0) return SWA_ERR_UNSUPPORTED;
+  if (Hq > 4096) return SWA_ERR_UNSUPPORTED;  // the prep kernel's per-head sums
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (total_tokens == 0) {
     if (dsink != nullptr) {
