@@ -1,5 +1,5 @@
 // ptx_sm100.cuh -- thin inline-PTX wrappers for sm_100a: mbarrier, TMA
-// (cp.async.bulk.tensor, no multicast), tcgen05 (TMEM alloc, MMA, commit,
+// (cp.async.bulk.tensor into this CTA's own shared memory only), tcgen05 (TMEM alloc, MMA, commit,
 // ld/st, fences), and the shared-memory matrix / instruction descriptors.
 //
 // Descriptor formats (tcgen05 "shared memory descriptor" and "instruction
