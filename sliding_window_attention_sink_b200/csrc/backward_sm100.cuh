@@ -28,7 +28,8 @@
 //                    dP (16 x 32), dS, dq += dS K
 //   bwd_dkdv_kernel  one CTA of 8 warps per (128 keys, kv head): the query
 //                    rows that see them in chunks of 32 (tokens x G heads),
-//                    double-buffered with cp.async; per warp 16 keys: S^T
+//                    three buffers filled by cp.async (one barrier per
+//                    chunk); per warp 16 keys: S^T
 //                    and dP^T (16 x 32), dv += P^T dO, dk += dS^T q
 // No inter-CTA waits; no traps.
 #pragma once
@@ -63,8 +64,8 @@ __host__ __device__ inline size_t bwd_dq_smem_bytes(int D) {
   return static_cast<size_t>(2 * kBwdQRows + 4 * kBwdKeyBlock) * (D + 8) * 2;
 }
 __host__ __device__ inline size_t bwd_dkdv_smem_bytes(int D) {
-  return static_cast<size_t>(2 * kBwdKeys + 4 * kBwdRowChunk) * (D + 8) * 2 +
-         2 * 4 * kBwdRowChunk * sizeof(float);
+  return static_cast<size_t>(2 * kBwdKeys + 6 * kBwdRowChunk) * (D + 8) * 2 +
+         3 * 4 * kBwdRowChunk * sizeof(float);
 }
 
 // First key visible to token t (same sequence, inside the window), and the
@@ -353,12 +354,12 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
   extern __shared__ __align__(16) uint8_t bwd_smem[];
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(bwd_smem);
   __nv_bfloat16* sV = sK + KT * LD;
-  __nv_bfloat16* sQb = sV + KT * LD;     // [2][RC][LD]
-  __nv_bfloat16* sdOb = sQb + 2 * RC * LD;  // [2][RC][LD]
-  float* rlse2b = reinterpret_cast<float*>(sdOb + 2 * RC * LD);  // [2][RC] lse (natural log)
-  float* rdltb = rlse2b + 2 * RC;
-  int* rtokb = reinterpret_cast<int*>(rdltb + 2 * RC);
-  int* rfirstb = rtokb + 2 * RC;
+  __nv_bfloat16* sQb = sV + KT * LD;     // [3][RC][LD]
+  __nv_bfloat16* sdOb = sQb + 3 * RC * LD;  // [3][RC][LD]
+  float* rlse2b = reinterpret_cast<float*>(sdOb + 3 * RC * LD);  // [3][RC] lse (natural log)
+  float* rdltb = rlse2b + 3 * RC;
+  int* rtokb = reinterpret_cast<int*>(rdltb + 3 * RC);
+  int* rfirstb = rtokb + 3 * RC;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // the first key tiles (the most rows, in a global layer) first, all kv
   // heads of a tile together
@@ -374,10 +375,10 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
   const int n_chunks = (n_rows + RC - 1) / RC;
   int c_lo = 0, c_hi = -1;  // sequence of the last row token looked up
 
-  // chunk c of the rows into buffer c & 1 (q, dO by cp.async; row data by
-  // plain stores)
+  // chunk c of the rows into buffer c % 3 (q, dO, lse and Delta by cp.async;
+  // token and first key by plain stores)
   auto prefetch = [&](int c) {
-    const int bf = c & 1;
+    const int bf = c % 3;
     for (int idx = tid; idx < RC * U * 2; idx += blockDim.x) {
       const int which = idx / (RC * U);  // 0: q, 1: dO
       const int rem = idx - which * RC * U;
@@ -447,8 +448,11 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
     } else {
       cp_async_wait<0>();
     }
-    __syncthreads();  // chunk c (and K, V) landed; its row data are visible
-    const int bf = c & 1;
+    // chunk c (and K, V) landed and its row data are visible; and every
+    // thread is past chunk c - 1, so the prefetch of chunk c + 2 (next
+    // iteration) may overwrite buffer (c - 1) % 3 -- one barrier per chunk
+    __syncthreads();
+    const int bf = c % 3;
     const __nv_bfloat16* sQ = sQb + bf * RC * LD;
     const __nv_bfloat16* sdO = sdOb + bf * RC * LD;
     const float* rlse2 = rlse2b + bf * RC;
@@ -465,10 +469,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
       const int kw0 = k0 + warp * 16, kw1 = min(kw0 + 15, klast);
       const bool none = kw0 > klast || t_last < kw0 ||
                         (p.window > 0 && t_first > kw1 + p.window - 1);
-      if (none) {
-        __syncthreads();
-        continue;
-      }
+      if (none) continue;
     }
     // S^T = K Q^T and dP^T = V dO^T for this warp's 16 keys x 32 rows
     float s[4][4], dp[4][4];
@@ -532,7 +533,6 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const BwdParams p) {
         mma_16816(dk[2 * np + 1], da0, da1, da2, da3, b2, b3);
       }
     }
-    __syncthreads();  // buffer bf is read: the prefetch two chunks on may overwrite it
   }
   cp_async_wait<0>();
   // dk = scale * acc, dv -> bf16
