@@ -79,7 +79,7 @@ def decode_work(pos, n_q, Hq, Hkv, D, W, kv_bytes=2, Hkv_scales=0):
     for P in pos:
         cached += min(P, W)
         for t in range(n_q):
-            pairs += min(P, W - 1 - t) + (t + 1)   # ring keys + new keys 0..t
+            pairs += min(P, max(0, W - 1 - t)) + (t + 1)   # ring keys + new keys 0..t
     B = len(pos)
     flops = 4 * D * Hq * pairs
     nbytes = (cached * Hkv * D * kv_bytes * 2 + B * n_q * Hkv * D * 2 * 2
