@@ -218,7 +218,9 @@ SWA_API int swa_sink_attn_fwd_rope(const void *q, const void *k, const void *v,
  *   workspace   device memory of swa_sink_attn_bwd_workspace() bytes (Delta,
  *               fp32 [Hq, total]), 16-byte aligned, owned by the caller; calls
  *               that overlap in time need separate workspaces.
- *   Hq/Hkv must divide 64; D 64 or 128.
+ *   Hq/Hkv must divide 64; Hq <= 4096; D 64 or 128 (else SWA_ERR_UNSUPPORTED).
+ *   dsink is zeroed and then accumulated on the stream (atomic adds: the
+ *   order of its fp32 sums, and so its last bits, can differ between calls).
  *
  * Returns SWA_OK or a negative swa_status_t.
  */
