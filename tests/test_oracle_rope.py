@@ -234,3 +234,17 @@ def test_global_cache_is_position_indexed():
     vb = c["v"].view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(k_c[0, 3:9], kr[0:6]) and np.array_equal(v_c[1, 0:9], vb[6:15])
     assert not k_c[0, :3].any() and not k_c[0, 9:].any()
+
+
+@pytest.mark.parametrize("W", [9, 0])
+def test_sampled_rows_equal_whole_prefill(W):
+    c = wl.prefill_case([40, 3, 25], 8, 2, 16, W, sigma=0.7, sink="normal", seed=12)
+    pos0 = [17, 0, 300]
+    o, lse, _, _ = rope.prefill_rope(c["q"], c["k"], c["v"], c["cu_seqlens"], 8, 2, 16, W, 1e4,
+                                     pos0=pos0, sink=c["sink"], interleaved=True)
+    rng = np.random.default_rng(6)
+    rt = np.concatenate([rng.integers(0, 68, 30), [0, 39, 40, 42, 43, 67]])
+    rh = rng.integers(0, 8, len(rt)).astype(np.int32)
+    so, sl = rope.prefill_rope_rows(c["q"], c["k"], c["v"], c["cu_seqlens"], 8, 2, 16, W, 1e4,
+                                    rt, rh, pos0=pos0, sink=c["sink"], interleaved=True)
+    assert np.array_equal(so, o[rt, rh]) and np.array_equal(sl, lse[rh, rt])
