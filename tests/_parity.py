@@ -1,6 +1,7 @@
 """Shared helpers for the GPU parity tests: device transfer and the error
-bounds stated for bf16 I/O with fp32 accumulation (max |dO| <= 1e-2,
-mean |dO| <= 1e-3, max |dLSE| <= 1e-3) against the fp64 oracle."""
+bounds stated for bf16 I/O with fp32 accumulation (output error: max
+|O - O_ref| <= 1e-2, mean <= 1e-3; max |LSE - LSE_ref| <= 1e-3) against the
+fp64 oracle."""
 import numpy as np
 import torch
 
