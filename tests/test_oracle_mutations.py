@@ -14,6 +14,10 @@ fail at least one pin, so the pins would catch it in the oracle itself.
 * RoPE oracle (oracle/rope.py): the frequency exponent halved, the rotation's
   sign flipped, the rotate-half pairing replaced by the interleaved one. Pins:
   the complex-multiplication form, the closed forms, the invariants.
+* FP8 oracle (oracle/fp8.py): the exponent bias, the tie rule, the K / V
+  scale index, the encoder's sign, the commit slot. Pins: torch's E4M3
+  decoding and cast, the midpoint ties, the C oracle on exactly representable
+  rings, the per-head scales, the commit's slots and codes.
 The unmutated oracles pass the same pin sets (checked first), so a failure
 comes from the planted mistake.
 """
@@ -27,6 +31,7 @@ import oracle
 import oracle.oracle as core
 import test_oracle as TO
 import test_oracle_backward as TB
+import test_oracle_fp8 as TF
 import test_oracle_rope as TR
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -168,6 +173,36 @@ def test_rope_pins_pass_unmutated(tmp_path, monkeypatch):
 def test_rope_mistake_fails_a_pin(mistake, tmp_path, monkeypatch):
     monkeypatch.setattr(TR, "rope", load_mutant("rope", ROPE_MUTATIONS[mistake], tmp_path))
     assert run_pins(ROPE_PINS), mistake
+
+
+FP8_PINS = [
+    ("table = torch", TF.test_table_matches_torch),
+    ("encode = torch cast", TF.test_encode_matches_torch_random),
+    ("midpoints to even", TF.test_encode_midpoints_ties_to_even),
+    ("exact rings = C oracle", lambda: TF.test_decode_fp8_equals_c_oracle_on_exact_rings(16, 0, 40)),
+    ("per-head scales", TF.test_dequantize_applies_per_head_scales),
+    ("commit slots and codes", TF.test_kv_commit_fp8_slots_and_codes),
+]
+
+FP8_MUTATIONS = {
+    "exponent bias": [("(1.0 + m / 8.0) * 2.0 ** (e - 7)", "(1.0 + m / 8.0) * 2.0 ** (e - 8)")],
+    "tie rule": [("(lo if lo % 2 == 0 else hi)", "(hi if lo % 2 == 0 else lo)")],
+    "K and V scales swapped": [("[which * Hkv:(which + 1) * Hkv]",
+                                "[(1 - which) * Hkv:(2 - which) * Hkv]")],
+    "encoder drops the sign": [("res[n] = c | (0x80 if", "res[n] = c | (0x00 if")],
+    "commit slot off by one": [("slot = (int(pos[b]) + u) % W", "slot = (int(pos[b]) + u + 1) % W")],
+}
+
+
+def test_fp8_pins_pass_unmutated(tmp_path, monkeypatch):
+    monkeypatch.setattr(TF, "fp8", load_mutant("fp8", [], tmp_path))
+    assert run_pins(FP8_PINS) == []
+
+
+@pytest.mark.parametrize("mistake", sorted(FP8_MUTATIONS))
+def test_fp8_mistake_fails_a_pin(mistake, tmp_path, monkeypatch):
+    monkeypatch.setattr(TF, "fp8", load_mutant("fp8", FP8_MUTATIONS[mistake], tmp_path))
+    assert run_pins(FP8_PINS), mistake
 
 
 def test_the_real_oracle_is_back(tmp_path):
