@@ -718,33 +718,72 @@ size_t bwd_workspace_bytes(int total, int Hq) {
   return (static_cast<size_t>(total) * Hq * sizeof(float) + 255) / 256 * 256;
 }
 
-size_t g_attr_bwd_dq[2][kMaxDevices], g_attr_bwd_dkdv[2][kMaxDevices];
+size_t g_attr_bt_dq[2][kMaxDevices], g_attr_bt_dkdv[2][kMaxDevices];
 
+// Backward on tcgen05: prep (Delta, dsink), then the dq and dk/dv pipelines
+// (persistent, one CTA per SM).
 template <int D>
-int launch_bwd(const swa::BwdParams& p, cudaStream_t st) {
-  swa::bwd_prep_kernel<D><<<(p.total + swa::kBwdPrepTokens - 1) / swa::kBwdPrepTokens, 256,
-                            sizeof(float) * p.Hq, st>>>(p);
+int launch_bwd(const swa::BwdParams& b, cudaStream_t st) {
+  swa::bwd_prep_kernel<D><<<(b.total + swa::kBwdPrepTokens - 1) / swa::kBwdPrepTokens, 256,
+                            sizeof(float) * b.Hq, st>>>(b);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("backward prep launch", e);
+  const int nsm = sm_count();
+  if (nsm <= 0) return SWA_ERR_CUDA;
+  swa::BtParams p;
+  p.cu_seqlens = b.cu_seqlens;
+  p.num_seqs = b.num_seqs;
+  p.total = b.total;
+  p.Hq = b.Hq;
+  p.Hkv = b.Hkv;
+  p.G = b.G;
+  p.lg = 0;
+  while ((1 << p.lg) < b.G) ++p.lg;  // G divides 64: a power of two
+  p.window = b.window;
+  p.TM = swa::kBtQRows / b.G;
+  p.TOK = swa::kBtRows / b.G;
+  p.lse = b.lse;
+  p.delta = b.delta;
+  p.scale = b.scale;
+  p.scale_log2 = b.scale_log2;
+  p.dq = b.dq;
+  p.dk = b.dk;
+  p.dv = b.dv;
+  p.q_box_bytes = 64u * 2u * swa::kBtQRows;
+  const uint32_t G = static_cast<uint32_t>(b.G);
   {
-    auto kern = swa::bwd_dq_kernel<D>;
-    const size_t smem = swa::bwd_dq_smem_bytes(D);
-    if (ensure_smem_attr(kern, smem, g_attr_bwd_dq[D == 128]) != SWA_OK) return SWA_ERR_CUDA;
-    const int TQ = swa::kBwdQRows / p.G;
-    const long long grid = static_cast<long long>((p.total + TQ - 1) / TQ) * p.Hkv;
-    if (grid > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
-    kern<<<static_cast<unsigned>(grid), 128, smem, st>>>(p);
+    CUtensorMap tq, tdo, tk, tv;
+    if (encode_3d(&tq, b.q, D, b.Hq, b.total, 64, G, p.TM) != SWA_OK ||
+        encode_3d(&tdo, b.dout, D, b.Hq, b.total, 64, G, p.TM) != SWA_OK ||
+        encode_3d(&tk, b.k, D, b.Hkv, b.total, 64, 1, swa::kBtChunk) != SWA_OK ||
+        encode_3d(&tv, b.v, D, b.Hkv, b.total, 64, 1, swa::kBtChunk) != SWA_OK)
+      return SWA_ERR_CUDA;
+    p.n_units = (b.total + p.TM - 1) / p.TM;
+    const long long tiles = static_cast<long long>(p.n_units) * b.Hkv;
+    if (tiles > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+    p.n_tiles = static_cast<int>(tiles);
+    auto kern = swa::bwd_dq_tc_kernel<D>;
+    const size_t smem = swa::bt_dq_smem_bytes<D>();
+    if (ensure_smem_attr(kern, smem, g_attr_bt_dq[D == 128]) != SWA_OK) return SWA_ERR_CUDA;
+    kern<<<std::min(p.n_tiles, nsm), swa::kBtThreads, smem, st>>>(tq, tdo, tk, tv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("backward dq launch", e);
   }
   {
-    auto kern = swa::bwd_dkdv_kernel<D>;
-    const size_t smem = swa::bwd_dkdv_smem_bytes(D);
-    if (ensure_smem_attr(kern, smem, g_attr_bwd_dkdv[D == 128]) != SWA_OK) return SWA_ERR_CUDA;
-    const long long grid =
-        static_cast<long long>((p.total + swa::kBwdKeys - 1) / swa::kBwdKeys) * p.Hkv;
-    if (grid > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
-    kern<<<static_cast<unsigned>(grid), 256, smem, st>>>(p);
+    CUtensorMap tk, tv, tq, tdo;
+    if (encode_3d(&tk, b.k, D, b.Hkv, b.total, 64, 1, swa::kBtKeys) != SWA_OK ||
+        encode_3d(&tv, b.v, D, b.Hkv, b.total, 64, 1, swa::kBtKeys) != SWA_OK ||
+        encode_3d(&tq, b.q, D, b.Hq, b.total, 64, G, p.TOK) != SWA_OK ||
+        encode_3d(&tdo, b.dout, D, b.Hq, b.total, 64, G, p.TOK) != SWA_OK)
+      return SWA_ERR_CUDA;
+    p.n_units = (b.total + swa::kBtKeys - 1) / swa::kBtKeys;
+    const long long tiles = static_cast<long long>(p.n_units) * b.Hkv;
+    if (tiles > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+    p.n_tiles = static_cast<int>(tiles);
+    auto kern = swa::bwd_dkdv_tc_kernel<D>;
+    const size_t smem = swa::bt_dkdv_smem_bytes<D>();
+    if (ensure_smem_attr(kern, smem, g_attr_bt_dkdv[D == 128]) != SWA_OK) return SWA_ERR_CUDA;
+    kern<<<std::min(p.n_tiles, nsm), swa::kBtThreads, smem, st>>>(tk, tv, tq, tdo, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("backward dk/dv launch", e);
   }
@@ -762,7 +801,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   if (total_tokens > 0 && num_seqs == 0) return SWA_ERR_SHAPE;
   if (max_seqlen > total_tokens) return SWA_ERR_SHAPE;
   if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
-  if (swa::kBwdQRows % (Hq / Hkv) != 0) return SWA_ERR_UNSUPPORTED;
+  if (swa::kBtRows % (Hq / Hkv) != 0) return SWA_ERR_UNSUPPORTED;  // G divides 64
   if (Hq > 4096) return SWA_ERR_UNSUPPORTED;  // the prep kernel's per-head sums
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (total_tokens == 0) {
