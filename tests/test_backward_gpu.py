@@ -9,12 +9,14 @@ Tolerance, from the arithmetic: the kernels take the forward's bf16 o (in
 Delta), round P and dS to bf16 for the tensor cores and round dq, dk, dv to
 bf16: three roundings of at most 2^-9 relative each on every term. The test
 bounds the largest error by 2e-2 of the reference's largest magnitude and the
-mean error by 6e-3 of its mean magnitude (measured: at most 5.2e-3 and 4.0e-3,
-the latter for a window of 1, where dP - Delta cancels most). dsink =
+mean error by 6e-3 of its mean magnitude (measured on the earlier mma.sync
+kernels, which round at the same points: at most 5.2e-3 and 4.0e-3, the
+latter for a window of 1, where dP - Delta cancels most). dsink =
 -sum_i p_sink,i Delta_i cancels too: its error scales with
 S_h = sum_i p_sink,i sum_d |dout_id o_id| (each product of Delta off by up to
 2^-9 of itself through the bf16 o), and the test bounds it by 2^-9 S_h
-(measured: at most 1.7e-4 S_h).
+(measured on the earlier kernels: at most 1.7e-4 S_h; the prep kernel that
+computes dsink is unchanged).
 """
 import numpy as np
 import pytest
