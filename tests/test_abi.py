@@ -217,6 +217,8 @@ def test_bwd_argument_errors():
     assert bwd(max_seqlen=9) == -2
     assert bwd(D=96) == -3
     assert bwd(Hq=96, Hkv=1) == -3          # Hq/Hkv must divide 64
+    assert bwd(Hq=128, Hkv=1) == -3         # G = 128 does not divide 64
+    assert bwd(Hq=8192, Hkv=128) == -3      # G = 64 divides 64, but Hq > 4096
     assert bwd(lse=None) == -1
     assert bwd(dout=None) == -1
     assert bwd(dk=None) == -1
