@@ -16,7 +16,9 @@ from the kernels and kept in step with them by hand.
   arrives once the thread's earlier MMAs have. Under random schedules no role
   deadlocks and every read (MMA operand, TMEM load, shared-memory statistics)
   sees the version it expects over its whole issue-to-completion window. A
-  removed wait, a flipped parity and a wrong arrival count each fail it.
+  removed wait, a flipped parity and a wrong arrival count each fail it, and
+  index mistakes (a chunk too few, a mask or row range off by one, rows ending
+  with the tile's first key) each fail the coverage check.
 """
 import bisect
 import random
@@ -465,3 +467,34 @@ def test_protocol_model_catches_mistakes(mistake, monkeypatch):
         except AssertionError:
             failed += 1
     assert failed > 0
+
+
+COVER_MISTAKES = {
+    "dq: one chunk too few": ("nchunk = (t_last - lo + 64) // 64", "nchunk = (t_last - lo + 1) // 64"),
+    "dq: mask off by one": ("cmin = row_lo - cb; cmax = row_hi - cb",
+                            "cmin = row_lo - cb; cmax = row_hi - cb - 1"),
+    "dkdv: rows end with the first key's": ("t_hi = vis_end(cu, W, min(k0 + 128, total) - 1)",
+                                            "t_hi = vis_end(cu, W, k0)"),
+    "dkdv: row range off by one": ("cmax = (min(max(j_end - t0, 0), TOK) << lg) - 1 - 32 * hw",
+                                   "cmax = (min(max(j_end - t0, 0), TOK) << lg) - 2 - 32 * hw"),
+}
+
+
+@pytest.mark.parametrize("mistake", sorted(COVER_MISTAKES))
+def test_coverage_model_catches_mistakes(mistake):
+    """Each index mistake, put into a copy of the coverage model, fails it on
+    some of the shapes above."""
+    import inspect
+    old, new = COVER_MISTAKES[mistake]
+    src = "\n".join(inspect.getsource(f) for f in (emulate_dq, emulate_dkdv, check))
+    assert src.count(old) == 1, old
+    ns = dict(seq_of=seq_of, first_key=first_key, vis_end=vis_end, brute=brute)
+    exec(src.replace(old, new), ns)
+    failed = False
+    for cu, Hq, Hkv, W in COVER_CASES[:6]:
+        try:
+            ns["check"](cu, Hq, Hkv, W)
+        except AssertionError:
+            failed = True
+            break
+    assert failed
