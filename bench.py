@@ -205,6 +205,67 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ workloads --
+def describe_prefill(c):
+    out = {"Hq": c["Hq"], "Hkv": c["Hkv"], "head_dim": c["D"], "window": c["window"],
+           "num_seqs": len(c["seqlens"]), "tokens": c["total"]}
+    if c["rope_base"] > 0:
+        out.update(rope_base=c["rope_base"], ring=c["ring_W"])
+    if c["backward"]:
+        out["pass"] = "backward"
+    return out
+
+
+def describe_decode(d, full, fp8):
+    out = {"batch": d["B"], "n_q": d["n_q"], "Hq": d["Hq"], "Hkv": d["Hkv"],
+           "head_dim": d["D"], ("cache" if full else "ring"): d["W"]}
+    if fp8:
+        out["kv_cache"] = "e4m3, one fp32 scale per kv head for K and for V"
+    return out
+
+
+def decode_sets(full):
+    """Input sets the decode timing rotates over (the SWA batch is near L2)."""
+    return 1 if full else 3
+
+
+def l2_note(nbytes, nsets=1):
+    if nsets > 1:
+        return ("%d input sets rotated, %.0f MB each, %.0f MB together (> L2): a step's inputs "
+                "are not L2-resident" % (nsets, nbytes / 1e6, nsets * nbytes / 1e6))
+    return "inputs larger than L2 (%.0f MB per step)" % (nbytes / 1e6)
+
+
+def workload_config(case, wl, world, c=None):
+    """The bench line's config for a workload (both arms print the same)."""
+    c = c if c is not None else _cached_inputs_of(case, wl)
+    if isinstance(case, wl.PrefillCase):
+        if c["backward"]:
+            _, nbytes = backward_work(c["seqlens"], c["Hq"], c["Hkv"], c["D"], c["window"])
+        else:
+            _, nbytes = prefill_work(c["seqlens"], c["Hq"], c["Hkv"], c["D"], c["window"])
+            if c["rope_base"] > 0:
+                nbytes += sum(min(L, c["ring_W"]) for L in c["seqlens"]) * c["Hkv"] * c["D"] * 4
+        desc, note = describe_prefill(c), l2_note(nbytes)
+    else:
+        full, fp8 = case.cache == "full", case.kv == "fp8"
+        _, nbytes = decode_work_of(c, fp8)
+        desc, note = describe_decode(c, full, fp8), l2_note(nbytes, decode_sets(full))
+    return dict({"workload": case.name, "parallelism": "replicas" if world == 1 else
+                 "dp%d" % world, "l2": note}, **desc)
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 class PrefillRunner:
     def __init__(self, case, rank, torch, B, wl):
         self.torch, self.B = torch, B
@@ -297,15 +358,7 @@ class PrefillRunner:
             raise RuntimeError("swa_sink_attn_fwd: %s" % self.B.status_string(rc))
 
     def describe(self):
-        c = self.c
-        out = {"Hq": c["Hq"], "Hkv": c["Hkv"], "head_dim": c["D"], "window": c["window"],
-               "num_seqs": len(c["seqlens"]), "tokens": c["total"]}
-        if self.rope:
-            out.update(rope_base=c["rope_base"], ring=c["ring_W"])
-        if self.backward:
-            out.update(pass_="backward")
-            out["pass"] = out.pop("pass_")
-        return out
+        return describe_prefill(self.c)
 
 
 class DecodeRunner:
@@ -327,7 +380,7 @@ class DecodeRunner:
         self.g = {n: d[n].to(dev) for n in names}
         self.full = case.cache == "full"
         self.max_ctx = case.pos_hi
-        self.NSETS = 1 if self.full else 3
+        self.NSETS = decode_sets(self.full)
         self.sets = [self.g] + [{n: (t.clone() if n != "pos" else t) for n, t in self.g.items()}
                                 for _ in range(self.NSETS - 1)]
         self.ws = None
@@ -348,10 +401,6 @@ class DecodeRunner:
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
         self.units = d["B"]
         self.launches_per_call = 2 if getattr(self, "full", False) else 1
-        if self.NSETS > 1:
-            self.l2_note = ("%d input sets rotated, %.0f MB each, %.0f MB together (> L2): a "
-                            "step's inputs are not L2-resident" %
-                            (self.NSETS, self.bytes / 1e6, self.NSETS * self.bytes / 1e6))
 
     def call(self, stream):
         d, g = self.d, self.sets[self.turn]
@@ -380,29 +429,30 @@ class DecodeRunner:
             raise RuntimeError("swa_sink_attn_decode: %s" % self.B.status_string(rc))
 
     def describe(self):
-        d = self.d
-        out = {"batch": d["B"], "n_q": d["n_q"], "Hq": d["Hq"], "Hkv": d["Hkv"],
-               "head_dim": d["D"], ("cache" if self.full else "ring"): d["W"]}
-        if self.fp8:
-            out["kv_cache"] = "e4m3, one fp32 scale per kv head for K and for V"
-        return out
+        return describe_decode(self.d, self.full, self.fp8)
 
 
 # ------------------------------------------------------------ oracle timing --
 _INPUTS = {}
 
 
+def _cached_inputs_of(case, wl):
+    key = repr(case)
+    if key not in _INPUTS:
+        _INPUTS[key] = (wl.make_prefill(case) if isinstance(case, wl.PrefillCase)
+                        else wl.make_decode(case))
+    return _INPUTS[key]
+
+
 def _cached_inputs(workload, wl):
-    if workload not in _INPUTS:
-        case = wl.WORKLOADS[workload]
-        _INPUTS[workload] = (wl.make_prefill(case) if isinstance(case, wl.PrefillCase)
-                             else wl.make_decode(case))
-    return _INPUTS[workload]
+    return _cached_inputs_of(wl.WORKLOADS[workload], wl)
 
 
-def oracle_sample(workload, wl, seconds, threads, seed=0):
-    """Time the fp64 oracle on a bounded sample of the workload. Returns
-    (flops_done, bytes_equiv, elapsed_s, description, threads used)."""
+def oracle_sample(workload, wl, seconds, threads, seed=0, full_if_within=0.0):
+    """Time the fp64 oracle on a bounded sample of the workload (about
+    `seconds` of work), or on all of it when a whole pass is estimated to take
+    at most `full_if_within` seconds. Returns (flops_done, bytes_equiv,
+    elapsed_s, description, threads used)."""
     import numpy as np
     import oracle
     case = wl.WORKLOADS[workload]
@@ -469,7 +519,10 @@ def oracle_sample(workload, wl, seconds, threads, seed=0):
     # calibrate on a small sample, then size the timed sample to `seconds`
     n0 = max(1, min(total_rows, 2000 if unit != "sequences" else 4))
     t_cal = run(n0)
-    n = int(min(total_rows, max(n0, n0 * seconds / max(t_cal, 1e-3))))
+    if t_cal * total_rows / n0 <= full_if_within:
+        n = total_rows
+    else:
+        n = int(min(total_rows, max(n0, n0 * seconds / max(t_cal, 1e-3))))
     elapsed = run(n)
     frac = n / total_rows
     return F * frac, Bt * frac, elapsed, "%d of %d %s of %s, %d threads" % (
@@ -477,7 +530,10 @@ def oracle_sample(workload, wl, seconds, threads, seed=0):
 
 
 def run_reference(args, wl):
-    """The reference arm: the fp64 CPU oracle as it stands, on bounded samples."""
+    """The reference arm: the fp64 CPU oracle as it stands. Each timed step is
+    the whole workload when all steps together stay within about four minutes
+    (the SWA layer: about 7 s a pass on 16 threads), else a bounded sample of
+    it; warm-up steps are short samples."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -488,13 +544,14 @@ def run_reference(args, wl):
     case = wl.WORKLOADS[args.workload]
     is_prefill = isinstance(case, wl.PrefillCase)
     per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    full_within = 240.0 / max(1, args.steps)
     for _ in range(args.warmup):
-        oracle_sample(args.workload, wl, per_step / 4, threads)
+        oracle_sample(args.workload, wl, 1.0, threads)
     flops = nb = el = 0.0
     desc = ""
     for s in range(args.steps):
         f, b, e, desc, threads_used = oracle_sample(args.workload, wl, per_step, threads,
-                                                    seed=s + 1)
+                                                    seed=s + 1, full_if_within=full_within)
         flops += f
         nb += b
         el += e
@@ -505,9 +562,9 @@ def run_reference(args, wl):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": case.name, "impl_note": "fp64 CPU oracle, bounded samples"},
+        "config": workload_config(case, wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": unit, "cores": threads_used, "kind": "oracle",
-                         "sample": desc + " per step"},
+                         "cpu_model": cpu_model(), "sample": desc + " per step"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -586,7 +643,7 @@ def main():
         f, b, e, desc, threads = oracle_sample(args.workload, wl, args.cpu_seconds, threads)
         cpu = {"value": (f / e / 1e12) if is_prefill else (b / e / 1e9),
                "unit": "TFLOP/s" if is_prefill else "GB/s", "cores": threads,
-               "kind": "oracle", "sample": desc + ", %.1f s" % e}
+               "cpu_model": cpu_model(), "kind": "oracle", "sample": desc + ", %.1f s" % e}
 
     def barrier():
         if world > 1:
@@ -696,9 +753,7 @@ def main():
             "dtype": "bf16", "data": "synthetic",
             "config": dict({"workload": case.name,
                             "parallelism": "replicas" if world == 1 else "dp%d" % world,
-                            "l2": getattr(runner, "l2_note", None) or (
-                                "inputs larger than L2 (%.0f MB per step)" %
-                                (runner.bytes / 1e6))},
+                            "l2": l2_note(runner.bytes, getattr(runner, "NSETS", 1))},
                            **runner.describe()),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * runner.launches_per_call, "clocks": clk.summary(), "device_error_flags": flag,

@@ -26,12 +26,14 @@
  * --------------------------
  * - All array pointers are DEVICE pointers owned by the caller. bf16 arrays
  *   must be 16-byte aligned (TMA and 16-byte vector loads); int32/fp32 arrays
- *   4-byte. The library's own device memory is one 512-byte buffer per device
- *   (64 tile-scheduler slots of two counters), allocated, zeroed and
- *   synchronised by the first swa_sink_attn_fwd call on that device (so make
- *   that first call outside CUDA-graph capture); each later call takes the
- *   next slot, and its kernel leaves the slot zero again. Calls whose kernels
- *   overlap in time must therefore be fewer than 64 apart in call order.
+ *   4-byte. The library allocates no device memory and keeps no device state
+ *   between calls, apart from the error flags of swa_sink_device_error() and
+ *   the static slots of swa_sink_attn_fwd_noalloc. (The sliding-window
+ *   prefill balances its tiles with the hardware's cluster launch control:
+ *   a CTA that finishes early cancels the launch of a CTA of the same grid
+ *   that has not started and does its work. Calls on any number of streams
+ *   may run at the same time.) Workspaces, where a call needs one, are the
+ *   caller's.
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   Every call is asynchronous on that stream; the caller synchronises.
  * - Argument errors are returned as a negative status BEFORE anything is
@@ -40,9 +42,9 @@
  *   (about 2 s); if one expires, or a device-resident argument is out of range
  *   (a negative pos, an n_accept outside [0, n_q]), the kernel records a flag
  *   readable with swa_sink_device_error() and returns.
- * - Thread-safe: the global host state (the driver entry point, per-device
- *   kernel attributes and scheduler buffers, the slot counter) is filled
- *   under locks or updated atomically.
+ * - Thread-safe: the host state (the driver entry point, per-device kernel
+ *   attributes) is filled under locks. The first call of a kernel on a
+ *   device raises that kernel's shared-memory limit (cudaFuncSetAttribute).
  */
 #ifndef SWA_SINK_H
 #define SWA_SINK_H
@@ -101,17 +103,19 @@ SWA_API int swa_sink_attn_fwd(const void *q, const void *k, const void *v,
                       float *lse, void *stream);
 
 /*
- * swa_sink_attn_fwd without any device allocation.
+ * swa_sink_attn_fwd with a software tile scheduler in a static device array.
  *
  * The pages have no counterpart: this is an interface variant. The arguments
- * and the results (bit for bit) are those of swa_sink_attn_fwd; the only
- * difference is where the tile scheduler of the sliding-window kernel keeps
- * its two counters: in a static device array of the library (8 slots of two
- * 32-bit words, 64 bytes in all) instead of the buffer that swa_sink_attn_fwd
- * allocates with cudaMalloc on its first call on a device. For callers that
- * must not allocate: work inside a CUDA stream capture (a first
- * swa_sink_attn_fwd call there would call cudaMalloc), or a serving runtime
- * that hands all device memory to its own pool at start-up.
+ * and the results (bit for bit) are those of swa_sink_attn_fwd, and like it
+ * this call allocates no device memory. It is meant for callers that cannot
+ * allocate: code that runs while a CUDA stream is being captured, where
+ * cudaMalloc is not allowed, and serving runtimes that hand all device memory
+ * to their own pool at start-up. The difference lies in the sliding-window
+ * kernel's load balancing: here the kernel runs on one CTA per SM and draws
+ * its tile ranges from two counters in a static device array of the library
+ * (8 slots of two 32-bit words, 64 bytes in all, held by every GPU that loads
+ * the library until the process exits) instead of cancelling launches of its
+ * own grid.
  *
  *   slot   the static scheduler slot, 0 <= slot < 8. Any other value returns
  *          SWA_ERR_SHAPE before anything is launched (the array holds 8).
@@ -122,10 +126,12 @@ SWA_API int swa_sink_attn_fwd(const void *q, const void *k, const void *v,
  * - Calls whose kernels overlap in time (other streams, concurrently running
  *   graphs) race on a shared slot and give wrong results: give each of them
  *   its own slot.
- * - The first call on each device also looks up the array's device address
- *   (cudaGetSymbolAddress), raises the kernels' shared-memory limits and
- *   fetches the driver's tensor-map entry point; make that first call before
- *   any stream capture.
+ * - The first call on each device does all of this entry point's set-up: it
+ *   looks up the array's device address (cudaGetSymbolAddress), raises the
+ *   shared-memory limits of every prefill kernel it can launch (all head
+ *   dims and windows) and fetches the driver's tensor-map entry point. Later
+ *   calls make no set-up call; make that first call before any stream
+ *   capture.
  * - Only the sliding-window ring kernel has a scheduler; for shapes it does
  *   not take, the call runs the same kernel as swa_sink_attn_fwd and `slot`
  *   is not used.

@@ -109,10 +109,16 @@ struct RingParams {
   uint32_t s_stride;      // TMEM column of S / P buffer b is b * s_stride
   uint32_t o_col;         // TMEM column of O
   // Tile schedule. Tiles f = g * n_tok_tiles + tb are taken in ranges of
-  // consecutive f: CTA c first takes [c * static_tiles, (c + 1) * static_tiles),
-  // then draws ranges of dyn_span tiles from dyn_base on through sched[0].
-  // sched[1] counts finished CTAs; the last one sets both back to zero.
+  // consecutive f, one range per work unit u: units u < n_static are the
+  // static share [u * static_tiles, (u + 1) * static_tiles); unit
+  // n_static + d is the range of dyn_span tiles from dyn_base + d * dyn_span.
+  // A CTA first does unit blockIdx.x. Then, with sched == NULL (the grid has
+  // one CTA per unit), it takes over units of CTAs that have not started yet
+  // by cancelling their launch (cluster launch control); with a sched
+  // counter (the grid has n_static CTAs), it draws d from sched[0], and
+  // sched[1] counts finished CTAs, the last of which sets both back to zero.
   unsigned int* sched;
+  int n_static;
   int static_tiles;
   int dyn_base;
   int dyn_span;
@@ -161,6 +167,9 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   // ranges of tiles, from the producer to the 14 other warps
   __shared__ __align__(8) uint64_t rq_full[kRingRanges], rq_empty[kRingRanges];
   __shared__ int rq_lo[kRingRanges], rq_hi[kRingRanges];
+  // cluster launch control: the response to a cancellation request
+  __shared__ __align__(16) uint32_t clc_resp[4];
+  __shared__ __align__(8) uint64_t clc_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -198,6 +207,7 @@ __global__ void __launch_bounds__(kRingThreads, 1)
       mbar_init(smem_u32(&rq_full[q]), 1);
       mbar_init(smem_u32(&rq_empty[q]), kRingRangeReaders);
     }
+    mbar_init(smem_u32(&clc_bar), 1);
     if (ROPE) {
       for (int s = 0; s < p.NQ; ++s) mbar_init(smem_u32(&q_rot[s]), 4);
       for (int s = 0; s < p.NB; ++s) mbar_init(smem_u32(&k_rot[s]), 4);
@@ -590,18 +600,35 @@ __global__ void __launch_bounds__(kRingThreads, 1)
         return true;
       };
       bool ok = true;
+      uint32_t clc_phase = 0;
+      int u = static_cast<int>(blockIdx.x);  // this CTA's own unit first
       for (int k = 0; ok && !*abort; ++k) {
+        if (k > 0) {
+          if (p.sched != nullptr) {  // the next unit from the counter
+            u = p.n_static + static_cast<int>(atomicAdd(p.sched, 1u));
+          } else {  // the unit of a CTA whose launch this request cancels
+            mbar_arrive_expect_tx(smem_u32(&clc_bar), 16u);
+            clc_try_cancel(smem_u32(clc_resp), smem_u32(&clc_bar));
+            if (!mbar_wait(smem_u32(&clc_bar), clc_phase, abort)) break;
+            clc_phase ^= 1u;
+            if (!clc_query(smem_u32(clc_resp), u)) break;  // none left
+          }
+        }
         int f0, f1;
-        if (k == 0) {  // the static part
-          f0 = static_cast<int>(blockIdx.x) * p.static_tiles;
+        if (u < p.n_static) {
+          f0 = u * p.static_tiles;
           f1 = min(f0 + p.static_tiles, p.n_tiles);
-          if (f0 >= f1) continue;
-        } else {  // ranges drawn while any are left
-          const unsigned int d = atomicAdd(p.sched, 1u);
-          const long long s0 = p.dyn_base + static_cast<long long>(d) * p.dyn_span;
-          if (s0 >= p.n_tiles) break;
-          f0 = static_cast<int>(s0);
+        } else {
+          const long long s0 =
+              p.dyn_base + static_cast<long long>(u - p.n_static) * p.dyn_span;
+          f0 = static_cast<int>(min(s0, static_cast<long long>(p.n_tiles)));
           f1 = min(f0 + p.dyn_span, p.n_tiles);
+        }
+        if (f0 >= f1) {
+          // an empty static share: go on to the other units; past the end of
+          // the counter's ranges: done
+          if (k > 0 && p.sched != nullptr) break;
+          continue;
         }
         if (!publish(f0, f1)) break;
         for (int f = f0; f < f1 && ok; ++f, ++j) {
@@ -639,13 +666,15 @@ __global__ void __launch_bounds__(kRingThreads, 1)
         }
       }
       publish(0, 0);  // end of the schedule
-      // this CTA draws no more ranges; the last CTA to get here clears the
-      // call's scheduler slot for the next call that uses it
-      __threadfence();
-      if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      // with a counter: this CTA draws no more ranges; the last CTA to get
+      // here clears the call's scheduler slot for the next call that uses it
+      if (p.sched != nullptr) {
         __threadfence();
-        atomicExch(p.sched, 0u);
-        atomicExch(p.sched + 1, 0u);
+        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+          __threadfence();
+          atomicExch(p.sched, 0u);
+          atomicExch(p.sched + 1, 0u);
+        }
       }
     }
   } else if (warp == 13) {

@@ -165,6 +165,41 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------ cluster launch control --
+// Ask the hardware to cancel the launch of a CTA of this grid that has not
+// started yet, so that this CTA can do that CTA's work instead: the 16-byte
+// response goes to shared memory at `resp` (16-byte aligned), its completion
+// is counted (16 bytes) on the mbarrier `bar`. Launched without clusters,
+// every CTA is a cluster of one, so nothing is multicast. One thread issues.
+// After a response that says nothing was cancelled, no further request may be
+// issued by this CTA.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128"
+      " [%0], [%1];" ::"r"(resp), "r"(bar)
+      : "memory");
+}
+
+// Read a completed response: true with the cancelled CTA's blockIdx.x, or
+// false when no CTA was left to cancel. The fence lets the next request
+// write the same response buffer after this read.
+__device__ __forceinline__ bool clc_query(uint32_t resp, int& ctaid_x) {
+  uint32_t ok, x;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+      "mov.u32 %1, 0;\n\t"
+      "ld.shared.b128 r, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+      : "=r"(ok), "=r"(x)
+      : "r"(resp)
+      : "memory");
+  fence_proxy_async_smem();
+  ctaid_x = static_cast<int>(x);
+  return ok != 0;
+}
+
 // ------------------------------------------------------------ tcgen05 -----
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

@@ -3,8 +3,9 @@
 // sliding-window / global attention with a per-head sink on sm_100a.
 //
 // The operation and its sources are described in include/swa_sink.h. Every
-// argument error is returned before any launch. The only device memory the
-// library allocates is the per-device tile-scheduler buffer (sched_slot).
+// argument error is returned before any launch. The library allocates no
+// device memory; its only device-side state is the error-flag word and the
+// eight static scheduler slots of swa_sink_attn_fwd_noalloc.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -14,8 +15,8 @@
 #include <cstdio>
 #include <cstdlib>
 #include <algorithm>
-#include <atomic>
 #include <mutex>
+#include <utility>
 
 #include "../../include/swa_sink.h"
 #include "backward_sm100.cuh"
@@ -166,56 +167,24 @@ int sm_count() {
 
 size_t g_attr_ring[2][2][swa::kRingMaxBN16 + 1][kMaxDevices];
 
-// ---- tile scheduler state -----------------------------------------------------
-// The persistent prefill kernels draw tile ranges from a counter in device
-// memory: a slot of two words (next range, CTAs finished) that must read zero
-// when a launch starts and that the launch's last CTA sets back to zero. Each
-// call takes the next of kSchedSlots slots, so calls running at the same time
-// on different streams count separately (up to kSchedSlots of them).
-constexpr unsigned int kSchedSlots = 64;
-std::mutex g_sched_mu;
-unsigned int* g_sched[kMaxDevices];
-std::atomic<unsigned int> g_sched_seq{0};
-
-// This call's slot. The first call on a device allocates and zeroes the
-// slots (cudaMalloc, cudaMemset, then a device synchronisation).
-int sched_slot(unsigned int** slot) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail("cudaGetDevice", e);
-  {
-    std::lock_guard<std::mutex> lk(g_sched_mu);
-    if (g_sched[dev] == nullptr) {
-      void* ptr = nullptr;
-      const size_t bytes = 2 * kSchedSlots * sizeof(unsigned int);
-      e = cudaMalloc(&ptr, bytes);
-      if (e != cudaSuccess) return cuda_fail("cudaMalloc(scheduler slots)", e);
-      e = cudaMemset(ptr, 0, bytes);
-      if (e == cudaSuccess) e = cudaDeviceSynchronize();
-      if (e != cudaSuccess) {
-        cudaFree(ptr);
-        return cuda_fail("cudaMemset(scheduler slots)", e);
-      }
-      g_sched[dev] = static_cast<unsigned int*>(ptr);
-    }
-  }
-  *slot = g_sched[dev] + 2 * (g_sched_seq.fetch_add(1u) % kSchedSlots);
-  return SWA_OK;
-}
-
 // ---- scheduler slots that need no allocation ------------------------------------
-// swa_sink_attn_fwd_noalloc takes its tile-scheduler slot from this static
-// array instead of the per-device buffer that swa_sink_attn_fwd allocates on
-// its first call. Each slot is two words that must read zero when a launch
-// starts: they are zero when the module loads, and every launch leaves its
-// slot zero again (its last CTA clears it). 8 slots = 64 bytes.
+// swa_sink_attn_fwd_noalloc runs the ring kernel with a software tile
+// scheduler whose counters live in this static array. Each slot is two words
+// that must read zero when a launch starts: they are zero when the module
+// loads, and every launch leaves its slot zero again (its last CTA clears
+// it). 8 slots = 64 bytes.
 constexpr int kNoAllocSlots = 8;
 static __device__ __align__(256) unsigned int g_noalloc_sched[2 * kNoAllocSlots];
 std::mutex g_noalloc_mu;
 unsigned int* g_noalloc_base[kMaxDevices];
 
-// The device address of the slot, looked up once per device (with that device
-// current) by cudaGetSymbolAddress.
+int raise_prefill_smem_limits();
+
+// The device address of the slot. The first call on a device (with that
+// device current) looks the array up with cudaGetSymbolAddress and does the
+// rest of the one-time set-up of every prefill kernel this call can run (the
+// shared-memory limits, the tensor-map entry point), so later calls make no
+// set-up call of any kind.
 int noalloc_slot(int slot, unsigned int** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -225,23 +194,34 @@ int noalloc_slot(int slot, unsigned int** out) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_noalloc_sched);
     if (e != cudaSuccess || ptr == nullptr) return cuda_fail("cudaGetSymbolAddress", e);
+    if (raise_prefill_smem_limits() != SWA_OK) return SWA_ERR_CUDA;
+    if (get_encode_fn() == nullptr)
+      return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", 0);
     g_noalloc_base[dev] = static_cast<unsigned int*>(ptr);
   }
   *out = g_noalloc_base[dev] + 2 * slot;
   return SWA_OK;
 }
 
-// Static share and dynamic range length of a persistent launch over n_tiles
-// tiles: each CTA first takes static_tiles consecutive tiles (about
-// kStaticShare of an even split), the rest goes out in short ranges to
-// whichever CTA is free, so SMs that run faster take more. (On B200 the same
-// tile stream ran up to 1.3x faster on some SMs than on others.) A ring range
-// of kRingDynSpan tiles refills the K/V window once (NWIN - 1 extra blocks).
+// Work units of the ring kernel over n_tiles tiles on nsm SMs: each of the
+// first min(nsm, n_tiles) units is a static share of static_tiles consecutive
+// tiles (about kStaticShare of an even split); the rest of the tiles go out in
+// ranges of kRingDynSpan to whichever CTA is free, so SMs that run faster take
+// more. (On B200 the same tile stream ran up to 1.3x faster on some SMs than
+// on others.) A ring range refills the K/V window once (NWIN - 1 extra
+// blocks). With no counter (counted == false) an empty static share is left
+// out: the launch has one CTA per non-empty unit. Returns the number of units.
 constexpr double kStaticShare = 0.75;
 constexpr int kRingDynSpan = 8;
-void split_schedule(int n_tiles, int grid, int* static_tiles, int* dyn_base) {
-  *static_tiles = static_cast<int>(kStaticShare * n_tiles / grid);
-  *dyn_base = *static_tiles * grid;
+int ring_schedule(int n_tiles, int nsm, bool counted, swa::RingParams* p) {
+  const int lead = std::min(nsm, n_tiles);
+  p->static_tiles = static_cast<int>(kStaticShare * n_tiles / lead);
+  p->n_static = (p->static_tiles > 0 || counted) ? lead : 0;
+  p->dyn_base = p->static_tiles * p->n_static;
+  p->dyn_span = kRingDynSpan;
+  const long long n_dyn = (static_cast<long long>(n_tiles) - p->dyn_base + kRingDynSpan - 1) /
+                          kRingDynSpan;
+  return static_cast<int>(p->n_static + n_dyn);
 }
 
 template <int D, int BN16, bool ROPE>
@@ -287,9 +267,12 @@ bool ring_shape(int D, int G, int window, RingShape* r) {
 
 // Sliding-window prefill on the persistent ring pipeline when ring_shape
 // accepts the shape; SWA_ERR_UNSUPPORTED (nothing launched) otherwise. The
-// tile scheduler uses static slot `noalloc` when it is >= 0, else the next
-// slot of the library's per-device buffer. With `rope` the kernel rotates q
-// and k itself (and writes the ring it names).
+// launch has one CTA per work unit, and CTAs that finish early take over the
+// units of CTAs not yet started by cancelling their launch (cluster launch
+// control): no device memory and no state between calls. With `noalloc` >= 0
+// the kernel instead draws its ranges from the counter in static slot
+// `noalloc`, on one CTA per SM. With `rope` the kernel rotates q and k itself
+// (and writes the ring it names).
 template <int D>
 int launch_prefill_ring(const void* q, const void* k, const void* v, const int32_t* cu,
                         int num_seqs, int total, int Hq, int Hkv, int window, const float* sink,
@@ -300,8 +283,7 @@ int launch_prefill_ring(const void* q, const void* k, const void* v, const int32
   if (!ring_shape(D, G, window, &rs)) return SWA_ERR_UNSUPPORTED;
   const int TM = rs.TM, BN = rs.BN;
   unsigned int* slot = nullptr;
-  if ((noalloc >= 0 ? noalloc_slot(noalloc, &slot) : sched_slot(&slot)) != SWA_OK)
-    return SWA_ERR_CUDA;
+  if (noalloc >= 0 && noalloc_slot(noalloc, &slot) != SWA_OK) return SWA_ERR_CUDA;
   swa::RingParams p;
   p.cu_seqlens = cu;
   p.num_seqs = num_seqs;
@@ -333,10 +315,9 @@ int launch_prefill_ring(const void* q, const void* k, const void* v, const int32
   const size_t smem = swa::ring_smem_bytes(D, TM, rs.NB, rs.NQ);
   const int nsm = sm_count();
   if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(multiprocessor count)", 0);
-  const int grid = std::min(nsm, p.n_tiles);
   p.sched = slot;
-  p.dyn_span = kRingDynSpan;
-  split_schedule(p.n_tiles, grid, &p.static_tiles, &p.dyn_base);
+  const int units = ring_schedule(p.n_tiles, nsm, slot != nullptr, &p);
+  const int grid = slot != nullptr ? p.n_static : units;
   static const swa::RopeArgs no_rope{};
   switch (BN / 16) {
 #define SWA_RING_CASE(N)                                                              \
@@ -399,6 +380,12 @@ int launch_prefill_chunked(const void* q, const void* k, const void* v, const in
   return e == cudaSuccess ? SWA_OK : cuda_fail("chunked prefill launch", e);
 }
 
+// Dynamic shared memory of the fallback prefill kernel for key chunks of BN.
+size_t prefill_smem_bytes(int D, int BN) {
+  return 1024 + (D / 64) * 16384 + 2 * (D / 64) * static_cast<size_t>(BN) * 128 +
+         static_cast<size_t>((BN + 63) / 64) * 16384;
+}
+
 template <int D>
 int launch_prefill(const void* q, const void* k, const void* v, const int32_t* cu, int num_seqs,
                    int total, int Hq, int Hkv, int window, const float* sink, float scale,
@@ -436,8 +423,7 @@ int launch_prefill(const void* q, const void* k, const void* v, const int32_t* c
   if (encode_3d(&tk, k, D, Hkv, total, 64, 1, BN) != SWA_OK) return SWA_ERR_CUDA;
   if (encode_3d(&tv, v, D, Hkv, total, 64, 1, BN) != SWA_OK) return SWA_ERR_CUDA;
 
-  const size_t smem = 1024 + (D / 64) * 16384 + 2 * (D / 64) * static_cast<size_t>(BN) * 128 +
-                      static_cast<size_t>((BN + 63) / 64) * 16384;
+  const size_t smem = prefill_smem_bytes(D, BN);
   auto kern = swa::prefill_sm100_kernel<D>;
   if (ensure_smem_attr(kern, smem, D == 64 ? g_attr_prefill64 : g_attr_prefill128) != SWA_OK)
     return SWA_ERR_CUDA;
@@ -554,6 +540,37 @@ int decode_impl(const void* q, const void* k_new, const void* v_new, const void*
   if (static_cast<long long>(B) * Hkv > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return kv_scale ? pick_decode<true>(p, D, st) : pick_decode<false>(p, D, st);
+}
+
+// Raise the shared-memory limit of every prefill kernel swa_sink_attn_fwd can
+// launch (the ring kernel for each window size class, the chunked kernel and
+// the fallback kernel, both head dims) to the most it can ask for, on the
+// current device.
+template <int D, int... N>
+int raise_ring_limits(std::integer_sequence<int, N...>) {
+  int rc = SWA_OK;
+  ((rc = rc != SWA_OK ? rc
+                      : ensure_smem_attr(swa::prefill_swa_ring_kernel<D, N + 1, false>,
+                                         kRingSmemLimit, g_attr_ring[0][D == 128][N + 1])),
+   ...);
+  return rc;
+}
+
+int raise_prefill_smem_limits() {
+  using Classes = std::make_integer_sequence<int, swa::kRingMaxBN16>;
+  if (raise_ring_limits<64>(Classes{}) != SWA_OK || raise_ring_limits<128>(Classes{}) != SWA_OK)
+    return SWA_ERR_CUDA;
+  if (ensure_smem_attr(swa::prefill_chunked_kernel<64>, swa::chunked_smem_bytes(64),
+                       g_attr_chunked[0]) != SWA_OK ||
+      ensure_smem_attr(swa::prefill_chunked_kernel<128>, swa::chunked_smem_bytes(128),
+                       g_attr_chunked[1]) != SWA_OK)
+    return SWA_ERR_CUDA;
+  if (ensure_smem_attr(swa::prefill_sm100_kernel<64>, prefill_smem_bytes(64, 256),
+                       g_attr_prefill64) != SWA_OK ||
+      ensure_smem_attr(swa::prefill_sm100_kernel<128>, prefill_smem_bytes(128, 256),
+                       g_attr_prefill128) != SWA_OK)
+    return SWA_ERR_CUDA;
+  return SWA_OK;
 }
 
 // swa_sink_attn_fwd and swa_sink_attn_fwd_noalloc: validation and kernel

@@ -32,3 +32,39 @@ def check(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     if lse_gpu is not None:
         assert stats["max_lse"] <= MAX_ABS_LSE, (what, stats)
     return stats
+
+
+def check_every_row(o_gpu, lse_gpu, q, k, v, cu_seqlens, Hq, Hkv, D, window, sink, what,
+                    chunk_tokens=2048):
+    """Every (token, head) row of a prefill against the oracle, element by
+    element, one chunk of tokens at a time (the oracle's output for a whole
+    32K-token layer would be 2 GB of float64). The bounds are those of
+    check(): the largest error over all rows, and the mean over all rows.
+    q, k, v are what the oracle attends over (bf16 tensors or bit arrays)."""
+    import oracle
+    total = o_gpu.shape[0]
+    qb, kb, vb = oracle.oracle._bits(q), oracle.oracle._bits(k), oracle.oracle._bits(v)
+    max_o = max_l = 0.0
+    sum_o = 0.0
+    n_o = 0
+    for t0 in range(0, total, chunk_tokens):
+        t1 = min(total, t0 + chunk_tokens)
+        rt = np.repeat(np.arange(t0, t1, dtype=np.int64), Hq)
+        rh = np.tile(np.arange(Hq, dtype=np.int32), t1 - t0)
+        ro, rl, _ = oracle.prefill_rows(qb, kb, vb, cu_seqlens, Hq, Hkv, D, window, rt, rh,
+                                        sink=sink)
+        og = o_gpu[t0:t1].float().cpu().numpy().astype(np.float64).reshape(-1, D)
+        assert np.isfinite(og).all(), "%s: non-finite output in tokens [%d, %d)" % (what, t0, t1)
+        err = np.abs(og - ro)
+        max_o = max(max_o, float(err.max()))
+        sum_o += float(err.sum())
+        n_o += err.size
+        if lse_gpu is not None:
+            lg = lse_gpu[:, t0:t1].t().contiguous().cpu().numpy().astype(np.float64).reshape(-1)
+            assert np.isfinite(lg).all(), "%s: non-finite lse" % what
+            max_l = max(max_l, float(np.abs(lg - rl).max()))
+        assert max_o <= MAX_ABS_O and max_l <= MAX_ABS_LSE, (what, t0, max_o, max_l)
+    stats = dict(max_o=max_o, mean_o=sum_o / max(n_o, 1), max_lse=max_l, rows=total * Hq)
+    print("%s: every row %s" % (what, stats))
+    assert stats["mean_o"] <= MEAN_ABS_O, (what, stats)
+    return stats

@@ -7,16 +7,20 @@ sampled rows and keys.
 
 Tolerance, from the arithmetic: the kernels take the forward's bf16 o (in
 Delta), round P and dS to bf16 for the tensor cores and round dq, dk, dv to
-bf16: three roundings of at most 2^-9 relative each on every term. The test
-bounds the largest error by 2e-2 of the reference's largest magnitude and the
-mean error by 6e-3 of its mean magnitude (measured on the earlier mma.sync
-kernels, which round at the same points: at most 5.2e-3 and 4.0e-3, the
-latter for a window of 1, where dP - Delta cancels most). dsink =
--sum_i p_sink,i Delta_i cancels too: its error scales with
-S_h = sum_i p_sink,i sum_d |dout_id o_id| (each product of Delta off by up to
-2^-9 of itself through the bf16 o), and the test bounds it by 2^-9 S_h
-(measured on the earlier kernels: at most 1.7e-4 S_h; the prep kernel that
-computes dsink is unchanged).
+bf16. Each rounding is at most 2^-9 relative (bf16 has 8 significant bits);
+the last one alone puts up to 2^-9 of max|ref| on the largest element, and
+the two earlier ones reach a gradient through sums whose terms have both
+signs, so their share of an element's error is of the same order but can be
+a few times larger where the sum cancels (dP - Delta for a window of 1). The
+tcgen05 kernels measured, over the cases below (the full layers included):
+largest error up to 5.2e-3 of max|ref| (2.7 x 2^-9; global layer, D = 64,
+dq) and mean error up to 2.3e-3 of mean|ref|, 4.0e-3 for the window of 1.
+The bounds are at most twice the largest of these: max error <= 1e-2
+max|ref|, mean error <= 6e-3 mean|ref| (1.5x). dsink = -sum_i p_sink,i
+Delta_i cancels too: its error scales with S_h = sum_i p_sink,i
+sum_d |dout_id o_id| (each product of Delta off by about 2^-9 of itself
+through the bf16 o, with both signs); measured at most 1.7e-4 S_h, bounded
+by 3.4e-4 S_h.
 """
 import numpy as np
 import pytest
@@ -30,6 +34,10 @@ from sliding_window_attention_sink_b200 import workloads as wl
 from _parity import to_cuda
 
 pytestmark = pytest.mark.gpu
+
+MAX_REL = 1e-2      # largest error / largest reference magnitude
+MEAN_REL = 6e-3     # mean error / mean reference magnitude
+DSINK_REL = 3.4e-4  # dsink error / S_h
 
 
 def run_bwd(c, dout, sink="case"):
@@ -52,7 +60,7 @@ def check_grad(got, ref, what):
     scale_mean = max(np.abs(ref).mean(), 1e-30)
     stats = (float(err.max() / scale_max), float(err.mean() / scale_mean))
     print("%s: max err / max|ref| %.3g, mean err / mean|ref| %.3g" % (what, *stats))
-    assert stats[0] <= 2e-2 and stats[1] <= 6e-3, (what, stats)
+    assert stats[0] <= MAX_REL and stats[1] <= MEAN_REL, (what, stats)
     return stats
 
 
@@ -77,7 +85,7 @@ def check_dsink(got, ref, scale, what):
     err = np.abs(g - ref)
     ratio = float((err / np.maximum(scale, 1e-30)).max()) if scale.any() else 0.0
     print("%s: dsink error / S_h max %.3g" % (what, ratio))
-    assert np.all(err <= 2.0 ** -9 * scale + 1e-6), (what, ratio)
+    assert np.all(err <= DSINK_REL * scale + 1e-6), (what, ratio)
 
 
 SMALL = [  # (name, seqlens, Hq, Hkv, D, W, sink)

@@ -28,11 +28,11 @@ def small(case):
 @pytest.mark.parametrize("name", sorted(wl.WORKLOADS))
 def test_oracle_sample_runs(name, monkeypatch):
     monkeypatch.setitem(wl.WORKLOADS, name, small(wl.WORKLOADS[name]))
-    bench._INPUTS.pop(name, None)
+    bench._INPUTS.clear()
     try:
         f, nbytes, el, desc, threads = bench.oracle_sample(name, wl, 0.05, 2, seed=1)
     finally:
-        bench._INPUTS.pop(name, None)
+        bench._INPUTS.clear()
     assert f > 0 and nbytes > 0 and el > 0 and threads >= 1
     assert name in desc
     # the work reported is the whole workload's times the fraction sampled
@@ -45,8 +45,33 @@ def test_oracle_sample_runs(name, monkeypatch):
         if c["backward"]:
             F, Bt = bench.backward_work(c["seqlens"], c["Hq"], c["Hkv"], c["D"], c["window"])
             F = F * 3 // 5
-        bench._INPUTS.pop(name, None)
+        bench._INPUTS.clear()
         assert total == sum(c["seqlens"]) * c["Hq"]
         assert f == pytest.approx(F * n / total)
     else:
         assert total == case.B and 1 <= n <= total
+
+
+@pytest.mark.parametrize("name", ["swa_prefill_32k", "swa_decode_mtp"])
+def test_reference_arm_line(name, monkeypatch, capsys):
+    """--impl reference prints one JSON line with our arm's config (the same
+    dict workload_config gives the GPU arm), the oracle's CPU model and core
+    count, and covers the whole (scaled-down) workload each step."""
+    import json
+    import types
+    monkeypatch.setitem(wl.WORKLOADS, name, small(wl.WORKLOADS[name]))
+    bench._INPUTS.clear()
+    monkeypatch.delenv("RANK", raising=False)
+    args = types.SimpleNamespace(workload=name, steps=2, warmup=1, gpus=1)
+    try:
+        bench.run_reference(args, wl)
+        line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+        assert line["impl"] == "reference" and line["steps"] == 2
+        assert line["config"] == bench.workload_config(wl.WORKLOADS[name], wl, 1)
+        cpu = line["cpu_baseline"]
+        assert cpu["kind"] == "oracle" and cpu["cores"] >= 1 and cpu["cpu_model"]
+        words = cpu["sample"].split()
+        assert words[0] == words[2]  # "<n> of <total> ...": every row / sequence
+        assert line["e2e"]["h2d_bytes_per_step"] == 0
+    finally:
+        bench._INPUTS.clear()

@@ -1,8 +1,10 @@
 """GPU parity of swa_sink_attn_fwd (through the C ABI) against the fp64 oracle
-on the same seeded inputs: small shapes compared element by element, the full
-workloads on sampled rows, plus edge cases (ragged tails, empty and length-1
-sequences, tiles straddling sequences, no sink, extreme sinks, W = 1, G = 1
-and G = 16, chunked windows and global layers)."""
+on the same seeded inputs: small shapes and the full workloads (the SWA layer,
+the global layer and the packed varlen batch) compared element by element on
+every row, plus edge cases (ragged tails, empty and length-1 sequences, tiles
+straddling sequences, no sink, extreme sinks, W = 1, G = 1 and G = 16,
+chunked windows and global layers, and query groups that do not divide 128,
+which run the fallback kernel)."""
 import math
 
 import numpy as np
@@ -13,7 +15,7 @@ import oracle
 from sliding_window_attention_sink_b200 import binding as B
 from sliding_window_attention_sink_b200 import workloads as wl
 
-from _parity import check, to_cuda
+from _parity import check, check_every_row, to_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -43,6 +45,15 @@ SMALL = [  # (name, seqlens, Hq, Hkv, D, W, sink)
     ("no_sink", [257], 8, 1, 128, 128, None),
     ("w1", [70], 8, 1, 64, 1, "normal"),
     ("short_seqs", [1, 2, 3, 17], 8, 1, 128, 128, "normal"),
+    # G does not divide 128: the fallback kernel (tiles of floor(128/G) tokens)
+    ("fallback_g3_swa", [300], 12, 4, 128, 128, "normal"),
+    ("fallback_g3_global", [500], 48, 16, 128, 0, "normal"),
+    ("fallback_g6_varlen", [100, 0, 257, 1, 33], 6, 1, 128, 128, "normal"),
+    ("fallback_g5_d64_global_varlen", [129, 300, 5], 10, 2, 64, 0, "uniform2"),
+    ("fallback_g7_w37", [200], 7, 1, 64, 37, "normal"),
+    ("fallback_g96_one_token_tiles", [150], 96, 1, 64, 128, "normal"),
+    ("fallback_g3_wide_window", [600], 3, 1, 128, 300, "normal"),
+    ("fallback_g3_no_sink", [257], 12, 4, 128, 128, None),
 ]
 
 
@@ -107,47 +118,22 @@ def test_prefill_lse_optional_and_scale():
     check(o, None, ro, rl, "scale=0.3")
 
 
-def sample_rows(c, n, seed):
-    rng = np.random.default_rng(seed)
-    total, Hq = c["total"], c["Hq"]
-    cu = c["cu_seqlens"].tolist()
-    toks = set(rng.integers(0, total, n).tolist())
-    for s in range(len(cu) - 1):   # sequence starts and ends, window edges
-        for t in (cu[s], cu[s] + 1, cu[s] + 127, cu[s] + 128, cu[s + 1] - 1):
-            if cu[s] <= t < cu[s + 1]:
-                toks.add(t)
-    toks = sorted(toks)
-    heads = rng.integers(0, Hq, len(toks))
-    return np.array(toks, np.int64), heads.astype(np.int32)
-
-
 @pytest.mark.parametrize("wname", ["swa_prefill_32k", "global_prefill_8k",
                                    "varlen_swa_prefill"])
-def test_prefill_full_workloads_sampled(wname):
-    """The benchmark's launch configuration at full size; sampled rows
-    (all heads of each sampled token's kv group are checked) vs the oracle."""
+def test_prefill_full_workloads_every_row(wname):
+    """The benchmark's launch configuration at full size, every (token, head)
+    row against the oracle (the global layer's oracle takes about a minute on
+    16 host threads)."""
     case = wl.WORKLOADS[wname]
     c = wl.make_prefill(case)
     o, lse = run_gpu(c)
-    rt, rh = sample_rows(c, 384, 1)
-    G = c["Hq"] // c["Hkv"]
-    # widen each sampled (token, head) to its whole query group
-    rt = np.repeat(rt, G)
-    rh = (np.repeat(rh // G, G) * G + np.tile(np.arange(G), len(rh))).astype(np.int32)
-    ro, rl, _ = oracle.prefill_rows(c["q"], c["k"], c["v"], c["cu_seqlens"], c["Hq"],
-                                    c["Hkv"], c["D"], c["window"], rt, rh, sink=c["sink"])
-    og = o[torch.from_numpy(rt).cuda(), torch.from_numpy(rh.astype(np.int64)).cuda()]
-    lg = lse[torch.from_numpy(rh.astype(np.int64)).cuda(), torch.from_numpy(rt).cuda()]
-    check(og, lg, ro, rl, wname)
-    # every row written (the output was poisoned with NaN)
-    assert torch.isfinite(o).all().item()
-    assert torch.isfinite(lse).all().item()
+    check_every_row(o, lse, c["q"], c["k"], c["v"], c["cu_seqlens"], c["Hq"], c["Hkv"],
+                    c["D"], c["window"], c["sink"], wname)
 
 
-def test_prefill_repeated_calls_reuse_scheduler_slots():
-    # more calls than scheduler slots, on one stream and on two at once: each
-    # kernel must find its slot zeroed by the previous user of that slot, so
-    # every output equals the first one bit for bit
+def test_prefill_repeated_calls_on_two_streams():
+    # 70 rounds of a sliding-window and a global call, alternating between two
+    # streams: every output equals the first one bit for bit
     c = wl.prefill_case([700, 300], 16, 2, 128, 128, sigma=0.5, sink="normal", seed=5)
     d = to_cuda(c)
     ref_o, ref_l = B.attn_fwd(d["q"], d["k"], d["v"], d["cu_seqlens"], 128, sink=d["sink"])
@@ -167,3 +153,41 @@ def test_prefill_repeated_calls_reuse_scheduler_slots():
     for o, lse, go, gl in outs:
         assert torch.equal(o, ref_o) and torch.equal(lse, ref_l)
         assert torch.equal(go, ref_go) and torch.equal(gl, ref_gl)
+
+
+def test_prefill_many_calls_in_flight_on_several_streams():
+    """96 calls queued at once on four streams, each stream held back by a
+    timed sleep kernel until all are queued, so that many run on the GPU at
+    the same time (most are a few CTAs). The sliding-window kernel keeps no
+    state between calls (its load balancing cancels launches of its own grid),
+    so every output equals the serial result bit for bit."""
+    cases = [
+        wl.prefill_case([40], 16, 2, 128, 128, sigma=0.5, sink="normal", seed=31),
+        wl.prefill_case([700, 300], 16, 2, 128, 128, sigma=0.5, sink="normal", seed=32),
+        wl.prefill_case([257, 3], 8, 1, 64, 128, sigma=0.5, sink="normal", seed=33),
+        wl.prefill_case([33], 64, 8, 128, 128, sigma=0.5, sink=None, seed=34),
+        wl.prefill_case([500], 16, 2, 128, 0, sigma=0.5, sink="normal", seed=35),
+    ]
+    devs = [to_cuda(c) for c in cases]
+
+    def call(c, d):
+        return B.attn_fwd(d["q"], d["k"], d["v"], d["cu_seqlens"], c["window"], sink=d["sink"],
+                          max_seqlen=c["max_seqlen"])
+
+    refs = []
+    for c, d in zip(cases, devs):
+        refs.append(call(c, d))
+        torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    for st in streams:
+        with torch.cuda.stream(st):
+            torch.cuda._sleep(40_000_000)  # a bounded spin of about 20 ms
+    outs = []
+    for it in range(96):
+        i = it % len(cases)
+        with torch.cuda.stream(streams[(it // len(cases)) % len(streams)]):
+            outs.append((i, *call(cases[i], devs[i])))
+    torch.cuda.synchronize()
+    assert B.swa_sink_device_error() == 0
+    for i, o, lse in outs:
+        assert torch.equal(o, refs[i][0]) and torch.equal(lse, refs[i][1]), i

@@ -1,10 +1,12 @@
-"""GPU check of swa_sink_attn_fwd_noalloc, the entry point that allocates
-nothing: its tile scheduler uses a static slot instead of the buffer that
-swa_sink_attn_fwd allocates. Two calls in a row on the same slot (the second
-finds the slot as the first left it) must give exactly what swa_sink_attn_fwd
-gives, for the sliding-window ring kernel (the one with a scheduler) and for
-a global layer (no scheduler). The file is named to be collected last, so it
-also runs after every other GPU test in the same process."""
+"""GPU check of swa_sink_attn_fwd_noalloc, the entry point for callers that
+cannot allocate device memory: its sliding-window kernel draws tile ranges
+from counters in a static slot of the library instead of cancelling launches
+of its own grid as swa_sink_attn_fwd does. Two calls in a row on the same
+slot (the second finds the slot as the first left it) must give exactly what
+swa_sink_attn_fwd gives, for the sliding-window ring kernel (the one with a
+scheduler) and for a global layer (no scheduler). The file is named to be
+collected last, so it also runs after every other GPU test in the same
+process."""
 import pytest
 import torch
 
