@@ -328,9 +328,10 @@ class PrefillRunner:
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
         self.units = c["total"]
+        self.rope_fused = False  # RoPE: rotate inside the ring kernel, no workspace
         self.launches_per_call = 2 if getattr(self, "rope_pass", False) else 1
         if self.backward:
-            self.launches_per_call = 3  # Delta / dsink, dq, dk and dv
+            self.launches_per_call = 2  # dq (with Delta and dsink), dk and dv
 
     def call(self, stream):
         c = self.c
@@ -343,11 +344,12 @@ class PrefillRunner:
                 raise RuntimeError("swa_sink_attn_bwd: %s" % self.B.status_string(rc))
             return
         if self.rope:
+            ws = None if self.rope_fused else self.ws
             rc = self.B.swa_sink_attn_fwd_rope(
                 self.q, self.k, self.v, self.cu, len(c["seqlens"]), c["max_seqlen"], c["total"],
                 c["Hq"], c["Hkv"], c["D"], c["window"], self.sink, 0.0, c["rope_base"], 0, None,
-                self.k_ring, self.v_ring, c["ring_W"], self.ws, self.ws.numel(), self.o,
-                self.lse, stream)
+                self.k_ring, self.v_ring, c["ring_W"], ws, 0 if ws is None else ws.numel(),
+                self.o, self.lse, stream)
             if rc != 0:
                 raise RuntimeError("swa_sink_attn_fwd_rope: %s" % self.B.status_string(rc))
             return
@@ -583,6 +585,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--rope-fused", action="store_true",
+                    help="RoPE workloads of the ring kernel's shapes: pass no workspace, so "
+                         "the ring kernel rotates q and k itself (default: the rotation pass "
+                         "into the workspace, then the plain prefill)")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="prefill workloads: replace the sequence lengths by one "
                          "sequence of this length (small cases for profiling)")
@@ -618,6 +624,9 @@ def main():
                                    name="%s (T=%d)" % (case.name, args.seqlen))
         args.no_cpu_baseline = True
     runner = (PrefillRunner if is_prefill else DecodeRunner)(case, rank, torch, B, wl)
+    if args.rope_fused and getattr(runner, "rope", False):
+        runner.rope_fused = True
+        runner.launches_per_call = 1
     stream = torch.cuda.Stream()
     sptr = stream.cuda_stream
     if args.steps <= 0:
@@ -728,8 +737,13 @@ def main():
     else:
         value = runner.bytes * world / (ms_per_step * 1e-3) / 1e9
         unit = "GB/s"
-    # roofline of the (only) kernel in the step: the slower of tensor and HBM time
-    t_tensor = runner.flops / (peaks["bf16_tflops"] * 1e12)
+    # roofline of the (only) kernel in the step: the slower of tensor and HBM time.
+    # The tensor peak is the burst figure for a short timed region and the
+    # sustained one (the power cap's steady state) for one of half a second
+    # or more.
+    sustained = total_ms >= 500.0 and "bf16_tflops_sustained" in peaks
+    tensor_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    t_tensor = runner.flops / (tensor_peak * 1e12)
     t_hbm = runner.bytes / (peaks["hbm_gbs"] * 1e9)
     if t_hbm >= t_tensor:
         achieved = runner.bytes / (kern_avg * 1e-3) / 1e9
@@ -737,8 +751,9 @@ def main():
                 "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"]}
     else:
         achieved = runner.flops / (kern_avg * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak,
+                "unit": "TFLOP/s", "frac": achieved / tensor_peak,
+                "peak_kind": "sustained" if sustained else "burst"}
     roof["peak_source"] = src
     roof["algorithmic_bytes"] = runner.bytes
     roof["algorithmic_flops"] = runner.flops
@@ -754,7 +769,9 @@ def main():
             "config": dict({"workload": case.name,
                             "parallelism": "replicas" if world == 1 else "dp%d" % world,
                             "l2": l2_note(runner.bytes, getattr(runner, "NSETS", 1))},
-                           **runner.describe()),
+                           **runner.describe(),
+                           **({"rope_route": "fused"} if getattr(runner, "rope_fused", False)
+                              else {})),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * runner.launches_per_call, "clocks": clk.summary(), "device_error_flags": flag,
         }

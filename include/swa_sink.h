@@ -178,14 +178,17 @@ SWA_API int swa_sink_attn_fwd_noalloc(const void *q, const void *k, const void *
  *               the other slots are not touched. ring_W >= pos0[s] + L_s gives
  *               a plain position-indexed cache (the global layers' layout for
  *               swa_sink_attn_decode_splitkv).
- *   workspace   device memory of swa_sink_attn_fwd_rope_workspace() bytes,
- *               16-byte aligned, owned by the caller (NULL allowed when that
- *               is 0). Zero for sliding windows on the fused ring kernel
- *               (Hq/Hkv in {2, 4, 8}, window + 128/(Hq/Hkv) - 1 <= 192 keys):
- *               it rotates each Q tile and K block in shared memory. For the
- *               other shapes (global layers among them) a separate pass first
- *               writes rotated copies of q and k there, then the prefill runs
- *               on them. Calls that overlap in time need separate workspaces.
+ *   workspace   device memory of swa_sink_attn_fwd_rope_workspace() bytes
+ *               (the size of q plus k), 16-byte aligned, owned by the caller.
+ *               With it, a separate pass writes rotated copies of q and k
+ *               there, then the prefill runs on them: the faster route. NULL
+ *               (workspace_bytes ignored) is allowed for sliding windows on
+ *               the ring kernel (Hq/Hkv in {2, 4, 8}, window + 128/(Hq/Hkv) - 1
+ *               <= 192 keys): that kernel then rotates each Q tile and K block
+ *               in shared memory, needing no memory beyond the call's inputs
+ *               and outputs. Other shapes (global layers among them) need the
+ *               workspace. Calls that overlap in time need separate
+ *               workspaces.
  *
  * Returns SWA_OK or a negative swa_status_t (SWA_ERR_SHAPE for a bad base,
  * pairing flag, ring_W or a workspace that is too small).
@@ -224,7 +227,7 @@ SWA_API int swa_sink_attn_fwd_rope(const void *q, const void *k, const void *v,
  *   workspace   device memory of swa_sink_attn_bwd_workspace() bytes (Delta,
  *               fp32 [Hq, total]), 16-byte aligned, owned by the caller; calls
  *               that overlap in time need separate workspaces.
- *   Hq/Hkv must divide 64; Hq <= 4096; D 64 or 128 (else SWA_ERR_UNSUPPORTED).
+ *   Hq/Hkv must divide 64; D 64 or 128 (else SWA_ERR_UNSUPPORTED).
  *   dsink is zeroed and then accumulated on the stream (atomic adds: the
  *   order of its fp32 sums, and so its last bits, can differ between calls).
  *

@@ -239,12 +239,13 @@ def attn_fwd(q, k, v, cu_seqlens, window, sink=None, softmax_scale=0.0, max_seql
 def attn_fwd_rope(q, k, v, cu_seqlens, window, rope_base, sink=None, pos0=None,
                   interleaved=False, k_ring=None, v_ring=None, softmax_scale=0.0,
                   max_seqlen=None, out=None, lse=None, want_lse=True, workspace=None,
-                  stream=None):
+                  fused=False, stream=None):
     """attn_fwd with RoPE applied to q and k inside the call (q, k are read
     only). pos0: int32 CUDA [num_seqs] first position of each sequence (None:
     0). k_ring / v_ring: bf16 [num_seqs, ring_W, Hkv, D] written with the last
     ring_W tokens of each sequence (rotated K, V), or None. The workspace (a
-    uint8 CUDA tensor) is allocated here when the shape needs one."""
+    uint8 CUDA tensor) is allocated here unless given; fused=True passes none,
+    so that shapes of the ring kernel rotate in its shared memory."""
     total, Hq, D = q.shape
     Hkv = k.shape[1]
     num_seqs = cu_seqlens.numel() - 1
@@ -255,7 +256,7 @@ def attn_fwd_rope(q, k, v, cu_seqlens, window, rope_base, sink=None, pos0=None,
     if lse is None and want_lse:
         lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device)
     need = swa_sink_attn_fwd_rope_workspace(total, Hq, Hkv, D, window)
-    if workspace is None and need > 0:
+    if workspace is None and need > 0 and not fused:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ring_W = 0 if k_ring is None else k_ring.shape[1]
     rc = swa_sink_attn_fwd_rope(q, k, v, cu_seqlens, num_seqs, max_seqlen, total, Hq, Hkv, D,

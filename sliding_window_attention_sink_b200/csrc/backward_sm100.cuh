@@ -15,14 +15,14 @@
 // heads. P is recomputed from q, k and the forward's lse (fp32), as the
 // forward computed it.
 //
-// Three launches:
-//   bwd_prep_kernel     Delta from o and dO (fp32, [Hq, total] in the caller's
-//                       workspace; coalesced 16-byte loads of whole rows) and
-//                       dsink (per-CTA sums in shared memory, then atomic adds
-//                       into the zeroed output);
+// Two launches:
 //   bwd_dq_tc_kernel    persistent, warp-specialised, tcgen05: a tile is 128
 //                       query rows (128/G tokens x the G heads of one kv head,
 //                       as the forward packs them), resident with its dO rows;
+//                       its epilogue warps first find Delta = dO . o for the
+//                       next tile's rows (fp32, into the caller's workspace
+//                       [Hq, total] for dk/dv) and add -exp(s - lse) Delta into
+//                       dsink (zeroed by the call);
 //                       the tile's keys [first key of its first token, its last
 //                       token] stream in chunks of 64. Per chunk: S = Q K^T and
 //                       dP = dO V^T (K-major operands, into TMEM), dS = P (dP -
@@ -47,7 +47,8 @@
 //               [32 hw, 32 hw + 32) of the 64 and writes its 16 columns of
 //               bf16 pairs over its own first 16 score columns, so the groups
 //               never wait on each other;
-//   warps 8-11  epilogue (TMEM accumulators -> bf16 -> global, one row each);
+//   warps 8-11  epilogue (TMEM accumulators -> bf16 -> global, one row each;
+//               in dq also Delta and dsink, one tile ahead);
 //   warp 12     producer (TMA; lse / Delta by cp.async for dk/dv);
 //   warp 13     TMEM allocation; issues the two score MMAs;
 //   warp 14     issues the accumulating MMAs.
@@ -77,67 +78,8 @@ struct BwdParams {
   float scale, scale_log2;
   float* delta;       // [Hq, total] (workspace)
   __nv_bfloat16 *dq, *dk, *dv;
-  float* dsink;       // [Hq] or NULL; zero before bwd_prep_kernel
+  float* dsink;       // [Hq] or NULL; zeroed before the dq kernel
 };
-
-constexpr int kBwdPrepTokens = 16;  // tokens per prep CTA
-
-// ---- Delta and dsink ------------------------------------------------------------
-// Rows (token, head) are contiguous in o and dO: D/8 lanes take one row in
-// 16-byte pieces (coalesced), four rows per group in flight; dsink partials
-// gather per head in shared memory, one atomic add per head per CTA.
-template <int D>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
-  constexpr int LPR = D / 8;          // lanes per row
-  constexpr int RPW = 32 / LPR;       // rows per warp per step
-  constexpr int RPS = 8 * RPW;        // rows per CTA per step
-  constexpr int UNR = 4;              // steps in flight
-  extern __shared__ float prep_sink[];  // [Hq]
-  const int tid = threadIdx.x, lane = tid & 31;
-  const int sub = lane / LPR, pl = lane - sub * LPR;
-  const long long row0 = static_cast<long long>(blockIdx.x) * kBwdPrepTokens * p.Hq;
-  const long long row_end =
-      min(row0 + static_cast<long long>(kBwdPrepTokens) * p.Hq,
-          static_cast<long long>(p.total) * p.Hq);
-  for (int h = tid; h < p.Hq; h += blockDim.x) prep_sink[h] = 0.f;
-  __syncthreads();
-  const long long my0 = row0 + (tid >> 5) * RPW + sub;
-  for (long long base = my0; base < row_end; base += static_cast<long long>(RPS) * UNR) {
-    uint4 a[UNR], b[UNR];
-#pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const long long row = base + static_cast<long long>(u) * RPS;
-      a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (row < row_end) {
-        a[u] = __ldg(reinterpret_cast<const uint4*>(p.o + row * D) + pl);
-        b[u] = __ldg(reinterpret_cast<const uint4*>(p.dout + row * D) + pl);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const uint32_t av[4] = {a[u].x, a[u].y, a[u].z, a[u].w};
-      const uint32_t bv[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
-      float acc = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        acc += bf16lo_to_f32(av[e]) * bf16lo_to_f32(bv[e]) +
-               bf16hi_to_f32(av[e]) * bf16hi_to_f32(bv[e]);
-#pragma unroll
-      for (int m = LPR / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-      const long long row = base + static_cast<long long>(u) * RPS;
-      if (pl == 0 && row < row_end) {
-        const int t = static_cast<int>(row / p.Hq), h = static_cast<int>(row - t * p.Hq);
-        const size_t li = static_cast<size_t>(h) * p.total + t;
-        p.delta[li] = acc;
-        if (p.sink != nullptr)
-          atomicAdd(&prep_sink[h], -expf(__ldg(p.sink + h) - __ldg(p.lse + li)) * acc);
-      }
-    }
-  }
-  __syncthreads();
-  if (p.dsink != nullptr && p.sink != nullptr)
-    for (int h = tid; h < p.Hq; h += blockDim.x) atomicAdd(p.dsink + h, prep_sink[h]);
-}
 
 constexpr int kBtThreads = 480;  // 15 warps
 constexpr int kBtQRows = 128;    // dq: query rows per tile
@@ -155,7 +97,10 @@ struct BtParams {
   int n_units;        // dq: token tiles; dk/dv: key tiles
   int n_tiles;        // n_units * Hkv
   const float* lse;   // [Hq, total], natural log
-  const float* delta; // [Hq, total]
+  float* delta;       // [Hq, total]: written by dq, read by dk/dv
+  const __nv_bfloat16 *o, *dout;  // dq: Delta = dout . o
+  const float* sink;  // [Hq] or NULL
+  float* dsink;       // [Hq] or NULL; zero before the dq kernel
   float scale, scale_log2;
   __nv_bfloat16 *dq, *dk, *dv;
   uint32_t q_box_bytes;  // dq: one 64-column box of a Q tile (128 rows)
@@ -248,6 +193,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   extern __shared__ uint8_t bt_smem_q[];
   __shared__ __align__(8) uint64_t q_full[2], q_empty[2], kv_full[NKV], kv_empty[NKV];
   __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], a_full[2], a_empty[2];
+  // Delta of tile k's rows in slot k & 1, from the epilogue warps to the dS warps
+  __shared__ __align__(8) uint64_t dl_full[2], dl_empty[2];
+  __shared__ float delta_s[2][kBtQRows];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -268,12 +216,16 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&q_full[s]), 1);
-      mbar_init(smem_u32(&q_empty[s]), 1);
+      // the S issuer's commit after a tile's last S, and the four epilogue
+      // warps once they have read the tile's dO for Delta
+      mbar_init(smem_u32(&q_empty[s]), 5);
       mbar_init(smem_u32(&s_full[s]), 1);
       mbar_init(smem_u32(&s_empty[s]), 1);
       mbar_init(smem_u32(&p_full[s]), 8);
       mbar_init(smem_u32(&a_full[s]), 1);
       mbar_init(smem_u32(&a_empty[s]), 4);
+      mbar_init(smem_u32(&dl_full[s]), 4);
+      mbar_init(smem_u32(&dl_empty[s]), 8);
     }
     for (int s = 0; s < NKV; ++s) {
       mbar_init(smem_u32(&kv_full[s]), 1);
@@ -315,29 +267,29 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     const int tok = r >> p.lg, hh = r - (tok << p.lg);
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-    // this row's lse (log2 units) and Delta, fetched one tile ahead
-    auto row_stats = [&](int k, float& l2, float& dl) {
-      l2 = 0.f;
-      dl = 0.f;
-      if (k >= ntile) return;
+    // this row's lse (log2 units), fetched one tile ahead
+    auto row_lse = [&](int k) -> float {
+      if (k >= ntile) return 0.f;
       int g, tb;
       tile_of(k, g, tb);
       const int i = tb * p.TM + tok;
-      if (i >= p.total) return;
-      const size_t idx = static_cast<size_t>(g * p.G + hh) * p.total + i;
-      l2 = __ldg(p.lse + idx) * kLog2e;
-      dl = __ldg(p.delta + idx);
+      if (i >= p.total) return 0.f;
+      return __ldg(p.lse + static_cast<size_t>(g * p.G + hh) * p.total + i) * kLog2e;
     };
-    float l2_next, dl_next;
-    row_stats(0, l2_next, dl_next);
+    float l2_next = row_lse(0);
     int n = 0;
     bool ok = true;
     for (int k = 0; k < ntile && ok; ++k) {
       int g, tb, lo, nchunk;
       tile_of(k, g, tb);
       tile_keys(tb, lo, nchunk);
-      const float l2 = l2_next, dl = dl_next;
-      row_stats(k + 1, l2_next, dl_next);
+      const float l2 = l2_next;
+      l2_next = row_lse(k + 1);
+      // this row's Delta from the epilogue warps
+      if (!warp_all(mbar_wait(smem_u32(&dl_full[k & 1]), (k >> 1) & 1, abort))) break;
+      const float dl = delta_s[k & 1][r];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&dl_empty[k & 1]));
       const int t0 = tb * p.TM;
       const int i = t0 + tok;
       int row_lo = 0, row_hi = -1;  // rows past the end see no key
@@ -389,11 +341,67 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       }
     }
   } else if (warp < 12) {
-    // ====================== epilogue: dQ x scale -> bf16 ======================
+    // ========= Delta (a tile ahead) and the epilogue: dQ x scale -> bf16 ======
     const int r = 32 * (warp & 3) + lane;
     const int tok = r >> p.lg, hh = r - (tok << p.lg);
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    for (int k = 0; k < ntile && !*abort; ++k) {
+    // Delta = dO . o of this thread's row of tile k (fp32 over the bf16
+    // values: o from global memory, all its loads in flight at once; dO from
+    // the tile's Q stage, whose release waits for these reads) to slot k & 1
+    // for the dS warps and to the workspace for dk/dv; dsink -= exp(s - lse)
+    // Delta, summed over the warp's rows of each head (lanes with equal hh),
+    // one atomic add per head and warp
+    auto delta_of = [&](int k) -> bool {
+      const int sl = k & 1;
+      int g, tb;
+      tile_of(k, g, tb);
+      const int i = tb * p.TM + tok;
+      const int h = g * p.G + hh;
+      uint4 ov[D / 8];
+      if (i < p.total) {
+        const uint4* orow =
+            reinterpret_cast<const uint4*>(p.o + (static_cast<size_t>(i) * p.Hq + h) * D);
+#pragma unroll
+        for (int u = 0; u < D / 8; ++u) ov[u] = __ldg(orow + u);
+      }
+      if (!warp_all(mbar_wait(smem_u32(&q_full[sl]), (k >> 1) & 1, abort) &&
+                    mbar_wait(smem_u32(&dl_empty[sl]), ((k >> 1) & 1) ^ 1, abort)))
+        return false;
+      float dl = 0.f, ds = 0.f;
+      if (i < p.total) {
+#pragma unroll
+        for (int u = 0; u < D / 8; ++u) {
+          // dO row r, 16-byte unit u of the swizzled 64-column block u / 8
+          uint32_t bv[4];
+          ld_shared_v4(q_addr(sl, 1, u >> 3) + r * 128 + ((((u & 7) ^ (r & 7))) << 4), bv);
+          const uint32_t av[4] = {ov[u].x, ov[u].y, ov[u].z, ov[u].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dl += bf16lo_to_f32(av[e]) * bf16lo_to_f32(bv[e]) +
+                  bf16hi_to_f32(av[e]) * bf16hi_to_f32(bv[e]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&q_empty[sl]));  // dO of this tile is read
+      if (i < p.total) {
+        const size_t idx = static_cast<size_t>(h) * p.total + i;
+        p.delta[idx] = dl;
+        if (p.sink != nullptr) ds = -expf(__ldg(p.sink + h) - __ldg(p.lse + idx)) * dl;
+      }
+      delta_s[sl][r] = dl;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&dl_full[sl]));
+      if (p.dsink != nullptr && p.sink != nullptr) {
+        // a warp's 32 rows: lane % G is the head within the group (G a power
+        // of two); for G = 64 every lane has a head of its own
+        for (int m = 16; m >= p.G; m >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, m);
+        if (lane < p.G) atomicAdd(p.dsink + g * p.G + hh, ds);
+      }
+      return true;
+    };
+    bool ok = ntile == 0 || delta_of(0);
+    for (int k = 0; k < ntile && ok && !*abort; ++k) {
+      if (k + 1 < ntile && !delta_of(k + 1)) break;
       int g, tb;
       tile_of(k, g, tb);
       const int a = k & 1;

@@ -21,14 +21,17 @@
 // columns of O (and its row sums) by exp2(m_old - m_new) in TMEM. The final
 // O / l and LSE = m_used + log2(l) are exact whatever m_used is.
 //
-//   warps 0-7   two softmax warpgroups. Each thread owns one row (TMEM lane)
-//               and reads the chunk's whole S row for the max, so both groups
-//               reach the same m_used without exchanging anything; group hw
-//               then exponentiates columns [64 hw, 64 hw + 64) and writes its
-//               half of P. The groups run unsynchronised, so one group's
-//               exponentials overlap the other's loads and maxima.
-//   warps 8-11  epilogue: after a tile's last PV, O / l -> bf16 -> global (one
-//               row per thread) and the LSE.
+//   warps 0-7   two softmax warpgroups. Each thread owns one row (TMEM lane);
+//               group hw loads only columns [64 hw, 64 hw + 64) of the chunk,
+//               takes the row's chunk max from the max warps, exponentiates
+//               its columns and writes its half of P.
+//   warps 8-11  max and epilogue: per chunk, the masked row max over all 128
+//               columns, handed to the softmax groups through shared memory
+//               (two slots, one chunk ahead where S allows); after a tile's
+//               last PV, O / l -> bf16 -> global (one row per thread) and the
+//               LSE. The exponentials (16 per clock per SM: a chunk's 16384
+//               take as long as its MMAs) then run while the next chunk's
+//               maximum is found, instead of after it.
 //   warp 12     TMA producer: Q tile (2 stages), K and V chunks (2 stages
 //               each; K of chunk n goes out before V of chunk n - 1).
 //   warp 13     TMEM allocation; S = Q K^T into S buffer (chunk & 1).
@@ -116,6 +119,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
   __shared__ __align__(8) uint64_t o_full, o_empty, l_full, l_free;
   __shared__ float red_lr[2][128], red_lx[2][128], m_s[128];
+  // row max of chunk n (raw S units, masked) in slot n & 1, from the max warps
+  __shared__ float m_chunk[2][128];
+  __shared__ __align__(8) uint64_t mx_full[2], mx_empty[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -137,9 +143,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       mbar_init(smem_u32(&v_full[s]), 1);
       mbar_init(smem_u32(&v_empty[s]), 1);
       mbar_init(smem_u32(&s_full[s]), 1);
-      mbar_init(smem_u32(&s_empty[s]), 8);
+      mbar_init(smem_u32(&s_empty[s]), 12);  // 8 softmax warps + 4 max warps
       mbar_init(smem_u32(&p_full[s]), 8);
       mbar_init(smem_u32(&p_empty[s]), 1);
+      mbar_init(smem_u32(&mx_full[s]), 4);
+      mbar_init(smem_u32(&mx_empty[s]), 8);
     }
     mbar_init(smem_u32(&o_full), 1);
     mbar_init(smem_u32(&o_empty), 4);
@@ -210,23 +218,24 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         const int trole = 3 + hw;
         const bool tr = (tid & 127) == 0;
         if (tr) CHUNK_TRACE(trole, n, 0);
-        if (!mbar_wait(smem_u32(&s_full[b]), (n >> 1) & 1, abort)) {
+        // the row's chunk max from the max warps
+        if (!mbar_wait(smem_u32(&mx_full[b]), (n >> 1) & 1, abort) ||
+            !mbar_wait(smem_u32(&s_full[b]), (n >> 1) & 1, abort)) {
           ok = false;
           break;
         }
+        const float cm_raw = m_chunk[b][r];
         __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&mx_empty[b]));
         tc_fence_after();
         if (tr) CHUNK_TRACE(trole, n, 1);
         const uint32_t tS = tmem + lane_off + b * kChunkKeys;
-        // the other group's columns (max only), then this group's (kept)
+        // this group's columns of S
         uint32_t v[HALF];
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        {
+          const int cb = lo + c * kChunkKeys + hw * HALF;  // key of column 0 of this half
 #pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {
-          const int hs = pass == 0 ? (hw ^ 1) : hw;
-          const int cb = lo + c * kChunkKeys + hs * HALF;  // key of column 0 of this half
-#pragma unroll
-          for (int q = 0; q < HALF / 16; ++q) tmem_ld16_at(tS + hs * HALF + q * 16, &v[q * 16]);
+          for (int q = 0; q < HALF / 16; ++q) tmem_ld16_at(tS + hw * HALF + q * 16, &v[q * 16]);
           tmem_ld_wait();
           if (!(cb >= all_lo && cb + HALF - 1 <= all_hi)) {  // a row's edge is in this half
             const int cmin = row_lo - cb;
@@ -235,18 +244,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             for (int e = 0; e < HALF; ++e)
               if (e < cmin || e > cmax) v[e] = 0xff800000u;  // -inf
           }
-#pragma unroll
-          for (int e = 0; e < HALF; e += 4) {
-            mx0 = max3(mx0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-            mx1 = max3(mx1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-          }
         }
         // S of this chunk is in registers: the buffer may take S of chunk n + 2
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&s_empty[b]));
         if (tr) CHUNK_TRACE(trole, n, 2);
-        const float cm = fmaxf(mx0, mx1) * p.scale_log2;
+        const float cm = cm_raw * p.scale_log2;
         // lazy rescale: the reference moves only when the max outgrows it
         const bool grow = cm > m_used + kRescaleLog2;
         if (__any_sync(0xffffffffu, grow)) {
@@ -333,17 +337,19 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       if (lane == 0) mbar_arrive(smem_u32(&l_full));
     }
   } else if (warp < 12) {
-    // ======================= epilogue (warps 8..11) ==========================
+    // =============== chunk maxima and epilogue (warps 8..11) ==================
     const int r = 32 * (warp & 3) + lane;
     const int tok = r / p.G, hh = r - tok * p.G;
-    const uint32_t tO = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + o_col;
-    for (int k = 0; k < ntile && !*abort; ++k) {
+    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const uint32_t tO = tmem + lane_off + o_col;
+    // tile k's epilogue: O / l -> bf16 -> global, and the LSE
+    auto drain = [&](int k) -> bool {
       int g, tb;
       tile_of(k, g, tb);
       if (tid == 256) CHUNK_TRACE(5, k, 0);
-      if (!mbar_wait(smem_u32(&o_full), k & 1, abort)) break;
+      if (!mbar_wait(smem_u32(&o_full), k & 1, abort)) return false;
       if (tid == 256) CHUNK_TRACE(5, k, 1);
-      if (!mbar_wait(smem_u32(&l_full), k & 1, abort)) break;
+      if (!mbar_wait(smem_u32(&l_full), k & 1, abort)) return false;
       if (tid == 256) CHUNK_TRACE(5, k, 2);
       __syncwarp();
       tc_fence_after();
@@ -382,7 +388,76 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       }
       if (valid && p.lse != nullptr) p.lse[static_cast<size_t>(h) * p.total + i] = lse2 * kLn2;
       if (tid == 256) CHUNK_TRACE(5, k, 3);
+      return true;
+    };
+    int n = 0;  // chunk counter over the CTA's tiles, as the softmax counts
+    bool ok = true;
+    for (int k = 0; k < ntile && ok; ++k) {
+      int g, tb, lo, nchunk;
+      tile_of(k, g, tb);
+      tile_keys(tb, lo, nchunk);
+      const int t0 = tb * p.TM;
+      const int i = t0 + tok;
+      int row_lo = 0, row_hi = -1;  // rows past the end see no key
+      if (i < p.total) {
+        row_lo = first_key(p.cu_seqlens, p.num_seqs, p.window, i);
+        row_hi = i;
+      }
+      const int t_last = min(t0 + p.TM, p.total) - 1;
+      // keys visible to every row of the tile
+      const int all_lo = first_key(p.cu_seqlens, p.num_seqs, p.window, t_last);
+      const int all_hi = t0;
+      for (int c = 0; c < nchunk; ++c, ++n) {
+        const int b = n & 1;
+        if (!mbar_wait(smem_u32(&s_full[b]), (n >> 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        tc_fence_after();
+        const uint32_t tS = tmem + lane_off + b * kChunkKeys;
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs) {
+          uint32_t v[HALF];
+          const int cb = lo + c * kChunkKeys + hs * HALF;  // key of column 0 of this half
+#pragma unroll
+          for (int q = 0; q < HALF / 16; ++q) tmem_ld16_at(tS + hs * HALF + q * 16, &v[q * 16]);
+          tmem_ld_wait();
+          if (!(cb >= all_lo && cb + HALF - 1 <= all_hi)) {  // a row's edge is in this half
+            const int cmin = row_lo - cb;
+            const int cmax = row_hi - cb;
+#pragma unroll
+            for (int e = 0; e < HALF; ++e)
+              if (e < cmin || e > cmax) v[e] = 0xff800000u;  // -inf
+          }
+#pragma unroll
+          for (int e = 0; e < HALF; e += 4) {
+            mx0 = max3(mx0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+            mx1 = max3(mx1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&s_empty[b]));
+        // hand the max over once the softmax has read slot b's previous one
+        if (!mbar_wait(smem_u32(&mx_empty[b]), ((n >> 1) & 1) ^ 1, abort)) {
+          ok = false;
+          break;
+        }
+        m_chunk[b][r] = fmaxf(mx0, mx1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&mx_full[b]));
+        // the previous tile's epilogue, once this tile's first max is out
+        // (the softmax needs it before it can finish the tile whose PV the
+        // epilogue waits for)
+        if (c == 0 && k > 0 && !drain(k - 1)) {
+          ok = false;
+          break;
+        }
+      }
     }
+    if (ok && ntile > 0) drain(ntile - 1);
   } else if (warp == 12) {
     // ======================= TMA producer ====================================
     // Order: Q of a tile before its first K; K of chunk n before V of chunk

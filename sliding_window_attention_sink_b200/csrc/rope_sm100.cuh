@@ -126,11 +126,6 @@ __device__ __forceinline__ void ld_global_v4(const void* ptr, uint32_t (&v)[4]) 
                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
                : "l"(ptr));
 }
-__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t (&v)[4]) {
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
-               : "r"(addr));
-}
 
 // Standalone pass (for the prefill kernels that read q and k through TMA
 // without rotating them): one CTA per packed token rotates its Hq query rows

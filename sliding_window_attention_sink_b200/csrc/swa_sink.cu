@@ -622,19 +622,25 @@ int fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seql
 }
 
 // ---- prefill with the rotary embedding ------------------------------------------
-// The ring kernel rotates q and k in shared memory (no workspace); the other
-// prefill kernels read q and k through TMA straight into the MMAs, so for them
-// a standalone pass first writes rotated copies into the caller's workspace
-// (q then k, the k copy 256-byte aligned).
+// Two routes. With a workspace: a standalone pass writes rotated copies of q
+// and k there (q then k, the k copy 256-byte aligned), then the plain prefill
+// runs on them; the prefill kernels read q and k through TMA straight into
+// the MMAs. Without one (ring shapes only): the ring kernel rotates each Q
+// tile and K block in shared memory. The first is the faster for the 32K SWA
+// layer (the rotation inside the ring kernel lengthens its epilogue's
+// critical path more than a separate pass over q and k costs); the second
+// needs no memory beyond the call's inputs and outputs.
 size_t rope_k_offset(int total, int Hq, int D) {
   const size_t qb = static_cast<size_t>(total) * Hq * D * 2;
   return (qb + 255) / 256 * 256;
 }
 
+// The workspace of the two-pass route (rotated q, then k). Every shape can
+// take that route; shapes the ring kernel takes can also rotate in shared
+// memory without a workspace (a call given none).
 size_t rope_workspace_bytes(int total, int Hq, int Hkv, int D, int window) {
+  (void)window;
   if (total <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (D != 64 && D != 128)) return 0;
-  RingShape rs;
-  if (ring_shape(D, Hq / Hkv, window, &rs)) return 0;
   return rope_k_offset(total, Hq, D) + static_cast<size_t>(total) * Hkv * D * 2;
 }
 
@@ -662,8 +668,13 @@ int fwd_rope_impl(const void* q, const void* k, const void* v, const int32_t* cu
   if (!aligned4(cu_seqlens) || (sink && !aligned4(sink)) || (lse && !aligned4(lse)) ||
       (pos0 && !aligned4(pos0)))
     return SWA_ERR_ALIGN;
+  // route: rotate into the workspace and run the plain prefill (when the
+  // caller gives one), else rotate in the ring kernel's shared memory (ring
+  // shapes only)
   const size_t need = rope_workspace_bytes(total_tokens, Hq, Hkv, D, window);
-  if (need > 0) {
+  RingShape rs_probe;
+  const bool fused = workspace == nullptr && ring_shape(D, Hq / Hkv, window, &rs_probe);
+  if (!fused) {
     if (workspace == nullptr) return SWA_ERR_NULL;
     if (workspace_bytes < need) return SWA_ERR_SHAPE;
     if (!aligned16(workspace)) return SWA_ERR_ALIGN;
@@ -686,7 +697,7 @@ int fwd_rope_impl(const void* q, const void* k, const void* v, const int32_t* cu
   ra.v_ring = static_cast<__nv_bfloat16*>(v_ring);
   ra.ring_W = k_ring != nullptr ? ring_W : 0;
 
-  if (need == 0) {  // the ring kernel, fused
+  if (fused) {  // the ring kernel, rotating in shared memory
     return D == 64 ? launch_prefill_ring<64>(q, k, v, cu_seqlens, num_seqs, total_tokens, Hq,
                                              Hkv, window, sink, softmax_scale, o, lse, st, -1,
                                              &ra)
@@ -713,6 +724,15 @@ int fwd_rope_impl(const void* q, const void* k, const void* v, const int32_t* cu
   if (e != cudaSuccess) return cuda_fail("rope pass launch", e);
   const void* qr = pp.q_out;
   const void* kr = pp.k_out;
+  if (window > 0) {
+    const int rc = D == 64 ? launch_prefill_ring<64>(qr, kr, v, cu_seqlens, num_seqs,
+                                                     total_tokens, Hq, Hkv, window, sink,
+                                                     softmax_scale, o, lse, st, -1)
+                           : launch_prefill_ring<128>(qr, kr, v, cu_seqlens, num_seqs,
+                                                      total_tokens, Hq, Hkv, window, sink,
+                                                      softmax_scale, o, lse, st, -1);
+    if (rc != SWA_ERR_UNSUPPORTED) return rc;
+  }
   {
     const int rc = D == 64 ? launch_prefill_chunked<64>(qr, kr, v, cu_seqlens, num_seqs,
                                                         total_tokens, Hq, Hkv, window, sink,
@@ -737,14 +757,11 @@ size_t bwd_workspace_bytes(int total, int Hq) {
 
 size_t g_attr_bt_dq[2][kMaxDevices], g_attr_bt_dkdv[2][kMaxDevices];
 
-// Backward on tcgen05: prep (Delta, dsink), then the dq and dk/dv pipelines
-// (persistent, one CTA per SM).
+// Backward on tcgen05: the dq pipeline (which also writes Delta and adds up
+// dsink), then the dk/dv pipeline (persistent, one CTA per SM).
 template <int D>
 int launch_bwd(const swa::BwdParams& b, cudaStream_t st) {
-  swa::bwd_prep_kernel<D><<<(b.total + swa::kBwdPrepTokens - 1) / swa::kBwdPrepTokens, 256,
-                            sizeof(float) * b.Hq, st>>>(b);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail("backward prep launch", e);
+  cudaError_t e = cudaSuccess;
   const int nsm = sm_count();
   if (nsm <= 0) return SWA_ERR_CUDA;
   swa::BtParams p;
@@ -761,6 +778,10 @@ int launch_bwd(const swa::BwdParams& b, cudaStream_t st) {
   p.TOK = swa::kBtRows / b.G;
   p.lse = b.lse;
   p.delta = b.delta;
+  p.o = b.o;
+  p.dout = b.dout;
+  p.sink = b.sink;
+  p.dsink = b.dsink;
   p.scale = b.scale;
   p.scale_log2 = b.scale_log2;
   p.dq = b.dq;
@@ -819,7 +840,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   if (max_seqlen > total_tokens) return SWA_ERR_SHAPE;
   if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
   if (swa::kBtRows % (Hq / Hkv) != 0) return SWA_ERR_UNSUPPORTED;  // G divides 64
-  if (Hq > 4096) return SWA_ERR_UNSUPPORTED;  // the prep kernel's per-head sums
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (total_tokens == 0) {
     if (dsink != nullptr) {
@@ -842,7 +862,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   if (!aligned16(workspace)) return SWA_ERR_ALIGN;
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
     softmax_scale = 1.0f / std::sqrt(static_cast<float>(D));
-  if (dsink != nullptr) {  // the prep kernel adds into it
+  if (dsink != nullptr) {  // the dq kernel adds into it
     const cudaError_t e = cudaMemsetAsync(dsink, 0, sizeof(float) * Hq, st);
     if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync(dsink)", e);
   }

@@ -185,16 +185,20 @@ def test_fwd_rope_argument_errors():
     assert fwd_rope(window=0) == -1
     assert fwd_rope(window=0, workspace=FAKE, workspace_bytes=16) == -2
     assert fwd_rope(window=0, workspace=FAKE + 4, workspace_bytes=1 << 20) == -4
+    assert fwd_rope(Hq=2, Hkv=2) == -1
+    # a ring shape given a workspace takes the two-pass route: it must be big
+    # enough and aligned
+    assert fwd_rope(workspace=FAKE, workspace_bytes=16) == -2
+    assert fwd_rope(workspace=FAKE + 4, workspace_bytes=1 << 20) == -4
     assert fwd_rope(total_tokens=0, max_seqlen=0) == 0
 
 
 def test_fwd_rope_workspace_sizes():
     ws = B.swa_sink_attn_fwd_rope_workspace
-    # the fused ring kernel needs none
-    assert ws(32768, 64, 8, 128, 128) == 0
-    assert ws(1000, 8, 2, 128, 128) == 0
-    assert ws(1000, 4, 2, 64, 20) == 0
-    # the others: rotated q (padded to 256 bytes) + rotated k
+    # every shape: rotated q (padded to 256 bytes) + rotated k (ring shapes
+    # may also be called without it)
+    assert ws(32768, 64, 8, 128, 128) == 32768 * 64 * 128 * 2 + 32768 * 8 * 128 * 2
+    assert ws(1000, 4, 2, 64, 20) == (1000 * 4 * 64 * 2 + 255) // 256 * 256 + 1000 * 2 * 64 * 2
     q_bytes = 8192 * 64 * 128 * 2
     assert ws(8192, 64, 8, 128, 0) == q_bytes + 8192 * 8 * 128 * 2
     assert ws(300, 2, 2, 64, 128) == (300 * 2 * 64 * 2 + 255) // 256 * 256 + 300 * 2 * 64 * 2
@@ -218,7 +222,6 @@ def test_bwd_argument_errors():
     assert bwd(D=96) == -3
     assert bwd(Hq=96, Hkv=1) == -3          # Hq/Hkv must divide 64
     assert bwd(Hq=128, Hkv=1) == -3         # G = 128 does not divide 64
-    assert bwd(Hq=8192, Hkv=128) == -3      # G = 64 divides 64, but Hq > 4096
     assert bwd(lse=None) == -1
     assert bwd(dout=None) == -1
     assert bwd(dk=None) == -1

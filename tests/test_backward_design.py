@@ -246,8 +246,9 @@ class Sim:
 
 def model_dq(sim, nchunks, NKV):
     for s in range(2):
-        for nm, c in (("q_full", 1), ("q_empty", 1), ("s_full", 1), ("s_empty", 1),
-                      ("p_full", 8), ("a_full", 1), ("a_empty", 4)):
+        for nm, c in (("q_full", 1), ("q_empty", 5), ("s_full", 1), ("s_empty", 1),
+                      ("p_full", 8), ("a_full", 1), ("a_empty", 4), ("dl_full", 4),
+                      ("dl_empty", 8)):
             sim.bar("%s%d" % (nm, s), c)
     for s in range(NKV):
         sim.bar("kv_full%d" % s, 1)
@@ -284,6 +285,10 @@ def model_dq(sim, nchunks, NKV):
     def softmax(w):
         n = 0
         for k, nc in enumerate(nchunks):
+            # the tile's Delta (the rows of warp w % 4), from the epilogue warps
+            yield ("wait", "dl_full%d" % (k & 1), (k >> 1) & 1)
+            yield ("read", [(("DL", k & 1, w % 4), ("D", k))])
+            yield ("arrive", "dl_empty%d" % (k & 1))
             for c in range(nc):
                 b = n & 1
                 yield ("wait", "s_full%d" % b, (n >> 1) & 1)
@@ -312,7 +317,18 @@ def model_dq(sim, nchunks, NKV):
                 n += 1
 
     def epilogue(w):
+        def delta(k):  # Delta of tile k's rows (dO from its Q stage) into slot k & 1
+            yield ("wait", "q_full%d" % (k & 1), (k >> 1) & 1)
+            yield ("wait", "dl_empty%d" % (k & 1), ((k >> 1) & 1) ^ 1)
+            yield ("read", [(("Q", k & 1), k)])
+            yield ("arrive", "q_empty%d" % (k & 1))
+            yield ("write", [(("DL", k & 1, w), ("D", k))])
+            yield ("arrive", "dl_full%d" % (k & 1))
+        if nchunks:
+            yield from delta(0)
         for k, nc in enumerate(nchunks):
+            if k + 1 < len(nchunks):
+                yield from delta(k + 1)
             a = k & 1
             yield ("wait", "a_full%d" % a, (k >> 1) & 1)
             yield ("read", [(("ACC", a), ("A", k, nc - 1))])
@@ -435,14 +451,18 @@ def test_protocol_random_schedules(kernel):
         s.run()
 
 
-@pytest.mark.parametrize("mistake", ["no a_empty wait", "s_empty parity", "qd_full count"])
+@pytest.mark.parametrize("mistake", ["no a_empty wait", "s_empty parity", "qd_full count",
+                                     "dl_full parity", "dl_full count", "q_empty count"])
 def test_protocol_model_catches_mistakes(mistake, monkeypatch):
     """Each mistake, put into the model, fails some schedule."""
-    if mistake == "qd_full count":
+    if mistake in ("qd_full count", "dl_full count", "q_empty count"):
         real_bar = Sim.bar
+        which = mistake.split()[0]
 
         def bar(self, name, count):
-            real_bar(self, name, 2 if name.startswith("qd_full") else count)
+            # fewer arrivals than writers (readers): the next side goes early
+            real_bar(self, name, (1 if which == "q_empty" else 2) if name.startswith(which)
+                     else count)
         monkeypatch.setattr(Sim, "bar", bar)
     real_step = Sim.step_role
 
@@ -454,6 +474,8 @@ def test_protocol_model_catches_mistakes(mistake, monkeypatch):
                 self.roles[name] = (gen, None)  # the wait is skipped
             elif mistake == "s_empty parity" and b.startswith("s_empty"):
                 self.roles[name] = (gen, (b, par ^ 1))
+            elif mistake == "dl_full parity" and b.startswith("dl_full"):
+                self.roles[name] = (gen, (b, par ^ 1))
         return real_step(self, name)
     monkeypatch.setattr(Sim, "step_role", step_role)
     failed = 0
@@ -461,7 +483,10 @@ def test_protocol_model_catches_mistakes(mistake, monkeypatch):
     for i in range(60):
         tiles = [rng.randint(1, 6) for _ in range(rng.randint(2, 7))]
         s = Sim(i)
-        model_dkdv(s, tiles, 3) if mistake != "s_empty parity" else model_dq(s, tiles, 3)
+        if mistake in ("no a_empty wait", "qd_full count"):
+            model_dkdv(s, tiles, 3)
+        else:
+            model_dq(s, tiles, 3)
         try:
             s.run(limit=200000)
         except AssertionError:

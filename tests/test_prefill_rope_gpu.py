@@ -25,7 +25,7 @@ def bits(t):
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def run(c, base, pos0=None, interleaved=False, ring_W=0, window=None):
+def run(c, base, pos0=None, interleaved=False, ring_W=0, window=None, fused=False):
     d = to_cuda(c)
     w = c["window"] if window is None else window
     S = len(c["seqlens"])
@@ -38,7 +38,7 @@ def run(c, base, pos0=None, interleaved=False, ring_W=0, window=None):
     o = torch.full_like(d["q"], float("nan"))
     o, lse = B.attn_fwd_rope(d["q"], d["k"], d["v"], d["cu_seqlens"], w, base, sink=d["sink"],
                              pos0=p0, interleaved=interleaved, k_ring=kr, v_ring=vr, out=o,
-                             max_seqlen=c["max_seqlen"])
+                             max_seqlen=c["max_seqlen"], fused=fused)
     torch.cuda.synchronize()
     assert B.swa_sink_device_error() == 0
     return o, lse, kr, vr
@@ -120,16 +120,18 @@ CASES = [  # (name, seqlens, Hq, Hkv, D, W, pos0, interleaved, ring_W)
 @pytest.mark.parametrize("name,seqlens,Hq,Hkv,D,W,pos0,inter,ring_W", CASES,
                          ids=[c[0] for c in CASES])
 def test_rope_prefill_matches_oracle(name, seqlens, Hq, Hkv, D, W, pos0, inter, ring_W):
+    """Both routes: with the workspace (rotation pass, plain prefill) and, for
+    the ring kernel's shapes, without (rotation in its shared memory)."""
     base = 1e4 if W > 0 else 640000.0
     c = wl.prefill_case(seqlens, Hq, Hkv, D, W, sigma=0.5, sink="normal", seed=13)
-    need = B.swa_sink_attn_fwd_rope_workspace(c["total"], Hq, Hkv, D, W)
-    assert (need == 0) == name.startswith("ring"), need
-    o, lse, kr, vr = run(c, base, pos0=pos0, interleaved=inter, ring_W=ring_W)
+    assert B.swa_sink_attn_fwd_rope_workspace(c["total"], Hq, Hkv, D, W) > 0
     ro, rl, _, k_rot = rope.prefill_rope(c["q"], c["k"], c["v"], c["cu_seqlens"], Hq, Hkv, D,
                                          W, base, pos0=pos0, sink=c["sink"],
                                          interleaved=inter)
-    check(o, lse, ro, rl, name)
-    check_ring(c, kr, vr, k_rot, ring_W, pos0, inter)
+    for fused in ((False, True) if name.startswith("ring") else (False,)):
+        o, lse, kr, vr = run(c, base, pos0=pos0, interleaved=inter, ring_W=ring_W, fused=fused)
+        check(o, lse, ro, rl, "%s fused=%s" % (name, fused))
+        check_ring(c, kr, vr, k_rot, ring_W, pos0, inter)
 
 
 def test_rope_equals_plain_prefill_on_rotated_inputs():
@@ -192,18 +194,20 @@ def rotated_bits(x, pos, base, chunk=2048):
     return out
 
 
-def test_rope_full_swa_layer_every_row():
+@pytest.mark.parametrize("fused", [False, True], ids=["two_pass", "fused"])
+def test_rope_full_swa_layer_every_row(fused):
     """The benchmark's SWA layer (T=32768) with RoPE (base 1e4) and ring
-    emission, in the launch configuration the benchmark times; every row vs
-    the oracle (rotated at bf16, then attended in fp64)."""
+    emission, on both routes (the benchmark's is the two-pass one, with the
+    workspace); every row vs the oracle (rotated at bf16, then attended in
+    fp64)."""
     c = wl.make_prefill(wl.WORKLOADS["swa_prefill_32k_rope"])
     assert c["rope_base"] == 1e4 and c["ring_W"] == 128
-    o, lse, kr, vr = run(c, 1e4, ring_W=128)
+    o, lse, kr, vr = run(c, 1e4, ring_W=128, fused=fused)
     T = c["total"]
     pos = np.arange(T)
     q_rot, k_rot = rotated_bits(c["q"], pos, 1e4), rotated_bits(c["k"], pos, 1e4)
     check_every_row(o, lse, q_rot, k_rot, c["v"], c["cu_seqlens"], c["Hq"], c["Hkv"], c["D"],
-                    c["window"], c["sink"], "swa_prefill_32k rope")
+                    c["window"], c["sink"], "swa_prefill_32k rope fused=%s" % fused)
     # the ring holds the last 128 tokens
     tail = np.arange(T - 128, T)
     kg = bits(kr)[0][tail % 128]
