@@ -29,11 +29,11 @@
  *   4-byte. The library allocates no device memory and keeps no device state
  *   between calls, apart from the error flags of swa_sink_device_error() and
  *   the static slots of swa_sink_attn_fwd_noalloc. (The sliding-window
- *   prefill balances its tiles with the hardware's cluster launch control:
- *   a CTA that finishes early cancels the launch of a CTA of the same grid
- *   that has not started and does its work. Calls on any number of streams
- *   may run at the same time.) Workspaces, where a call needs one, are the
- *   caller's.
+ *   prefill and the bf16-ring decode balance their work with the hardware's
+ *   cluster launch control: a CTA that finishes early cancels the launch of
+ *   a CTA of the same grid that has not started and does its work. Calls on
+ *   any number of streams may run at the same time.) Workspaces, where a
+ *   call needs one, are the caller's.
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   Every call is asynchronous on that stream; the caller synchronises.
  * - Argument errors are returned as a negative status BEFORE anything is

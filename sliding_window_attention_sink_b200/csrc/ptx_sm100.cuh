@@ -326,6 +326,44 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
       : "memory");
 }
 
+// 16 lanes x 256 bits, repeated 4 times along the columns (16 registers):
+// thread T gets, for repetition k (columns 8k .. 8k+7 from taddr), lane T/4
+// columns 8k + 2(T%4) and + 1 in r[4k], r[4k+1], and lane 8 + T/4 at the same
+// columns in r[4k+2], r[4k+3].
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
+      "%10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+        "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+        "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+// The same, repeated twice (8 registers).
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+}
+// 16 lanes x 128 bits, repeated 8 times along the columns: for repetition k
+// (columns 4k .. 4k+3 from taddr) thread T writes r[k] to lane T/4 and to
+// lane 8 + T/4, both at column 4k + T%4.
+__device__ __forceinline__ void tmem_st_16x128b_x8_dup(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1, %1, %2, %2, %3, %3, %4, %4, %5, %5, "
+      "%6, %6, %7, %7, %8, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+// The same, repeated twice.
+__device__ __forceinline__ void tmem_st_16x128b_x2_dup(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.16x128b.x2.b32 [%0], {%1, %1, %2, %2};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1])
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }

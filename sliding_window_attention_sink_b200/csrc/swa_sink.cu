@@ -22,6 +22,7 @@
 #include "backward_sm100.cuh"
 #include "decode_fp8_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "decode_tc_sm100.cuh"
 #include "decode_splitkv_sm100.cuh"
 #include "prefill_chunked_sm100.cuh"
 #include "prefill_sm100.cuh"
@@ -149,6 +150,7 @@ bool g_carve_dec[2][2][2][kMaxDevices];
 
 size_t g_attr_prefill64[kMaxDevices], g_attr_prefill128[kMaxDevices];
 size_t g_attr_dec[2][2][2][2][kMaxDevices];
+size_t g_attr_dec_tc[2][kMaxDevices];
 
 int next_pow2(int x) {
   int p = 32;
@@ -475,8 +477,54 @@ int launch_decode(const swa::DecodeFp8Params& p, cudaStream_t st) {
   return e == cudaSuccess ? SWA_OK : cuda_fail("decode launch", e);
 }
 
+// Key rows of the tcgen05 decode: the ring, the new rows from W8, padded to
+// the MMA's N granule of 16.
+int decode_tc_kp(const swa::DecodeParams& p) { return round_up(p.W8 + p.n_q, 16); }
+
+// The tcgen05 decode takes a bf16 ring whose keys fit its softmax registers
+// and whose slots fit one CTA's shared memory (227 KB with the barriers).
+bool decode_tc_fits(const swa::DecodeParams& p, int D) {
+  const int KP = decode_tc_kp(p);
+  return KP <= swa::kDecTcMaxKP && swa::decode_tc_smem_bytes(D, KP) + 1024 <= 232448;
+}
+
+template <int D>
+int launch_decode_tc(const swa::DecodeParams& p, cudaStream_t st) {
+  // the same boxes as the one-CTA-per-unit kernel
+  CUtensorMap tq, tkr, tkn, tvr, tvn, to;
+  const uint32_t G = static_cast<uint32_t>(p.G), nq = static_cast<uint32_t>(p.n_q);
+  const uint32_t W = static_cast<uint32_t>(p.W);
+  if (encode_4d(&tkr, p.k_ring, D, p.Hkv, p.W, p.B, 64, 1, W, 1) != SWA_OK ||
+      encode_4d(&tvr, p.v_ring, D, p.Hkv, p.W, p.B, 64, 1, W, 1) != SWA_OK ||
+      encode_4d(&tq, p.q, D, p.Hq, p.n_q, p.B, 64, G, nq, 1) != SWA_OK ||
+      encode_4d(&tkn, p.k_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK ||
+      encode_4d(&tvn, p.v_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK ||
+      encode_4d(&to, p.o, D, p.Hq, p.n_q, p.B, 64, G, nq, 1) != SWA_OK)
+    return SWA_ERR_CUDA;
+  swa::DecodeTcParams tp;
+  tp.d = p;
+  tp.d.KP = decode_tc_kp(p);
+  tp.s_stride = static_cast<uint32_t>(round_up(tp.d.KP, 32));
+  tp.o_col = 2 * tp.s_stride;
+  tp.tmem_cols = static_cast<uint32_t>(next_pow2(static_cast<int>(tp.o_col) + D));
+  if (tp.tmem_cols > 512) return SWA_ERR_UNSUPPORTED;
+  const size_t smem = swa::decode_tc_smem_bytes(D, tp.d.KP);
+  auto kern = swa::decode_tc_sm100_kernel<D>;
+  if (ensure_smem_attr(kern, smem, g_attr_dec_tc[D == 128]) != SWA_OK) return SWA_ERR_CUDA;
+  // one CTA per (sequence, kv head); the CTAs that run take over the units of
+  // those that have not started (cluster launch control)
+  const unsigned grid = static_cast<unsigned>(p.B) * static_cast<unsigned>(p.Hkv);
+  kern<<<grid, swa::kDecTcThreads, smem, st>>>(tq, tkr, tkn, tvr, tvn, to, tp);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SWA_OK : cuda_fail("tcgen05 decode launch", e);
+}
+
 template <bool KV8>
 int pick_decode(const swa::DecodeFp8Params& p, int D, cudaStream_t st) {
+  if constexpr (!KV8) {
+    if (decode_tc_fits(p, D))
+      return D == 64 ? launch_decode_tc<64>(p, st) : launch_decode_tc<128>(p, st);
+  }
   const bool two = p.R > 16;
   // 4 warps up to 160 keys, else 8
   if (p.KP <= swa::kDecodeSmallMaxKP) {
