@@ -114,7 +114,7 @@ KERNEL_SOURCES = {
     "chunked_rope": ["prefill_chunked_sm100.cuh", "rope_sm100.cuh", "prefill_sm100.cuh",
                      "ptx_sm100.cuh", "swa_sink.cu"],
     "backward": ["backward_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
-    "decode": ["decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
+    "decode": ["decode_tc_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "decode_fp8": ["decode_fp8_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "splitkv": ["decode_splitkv_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
 }
