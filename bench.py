@@ -630,15 +630,19 @@ def main():
     stream = torch.cuda.Stream()
     sptr = stream.cuda_stream
     if args.steps <= 0:
-        # about one second of timed work (enough clock samples), >= 20 steps
+        # about one second of timed work (enough clock samples), >= 20 steps,
+        # sized from 20 back-to-back calls (one call alone also times its
+        # launch)
         with torch.cuda.stream(stream):
             runner.call(sptr)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            runner.call(sptr)
+            for _ in range(20):
+                runner.call(sptr)
             b.record(stream)
         torch.cuda.synchronize()
-        args.steps = int(max(20, min(50000, 1000.0 / max(a.elapsed_time(b), 1e-3))))
+        per_call = max(a.elapsed_time(b) / 20.0, 1e-3)
+        args.steps = int(max(20, min(100000, 1100.0 / per_call)))
         if world > 1:  # every rank must time the same number of steps
             t = torch.tensor([args.steps], device="cuda", dtype=torch.int64)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -766,7 +770,8 @@ def main():
     roof["algorithmic_flops"] = runner.flops
     roof["kernel_ms"] = kern_avg
     roof["kernel_timed_calls"] = len(kern_ms)  # calls with an event pair around them
-    roof["traffic"] = recorded_traffic(args.workload)
+    # (a record is for the workload's own sizes, not a --seqlen variant)
+    roof["traffic"] = recorded_traffic(args.workload) if args.seqlen <= 0 else None
 
     if rank == 0:
         line = {

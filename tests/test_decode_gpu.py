@@ -121,3 +121,21 @@ def test_kv_commit_flags_bad_n_accept():
     torch.cuda.synchronize()
     assert B.swa_sink_device_error() == 2
     assert B.swa_sink_device_error() == 0
+
+
+def test_decode_flags_negative_position():
+    """A negative position is read as 0 (only the new tokens are visible) and
+    flagged; the other sequences are unaffected."""
+    d = wl.decode_case(4, 2, 16, 2, 128, 128, sigma=0.5, sink="normal", seed=17, pos_lo=0,
+                       pos_hi=300)
+    d["pos"][1] = -3
+    g = to_cuda(d)
+    o = torch.full_like(g["q"], float("nan"))
+    o, lse = B.attn_decode(g["q"], g["k_new"], g["v_new"], g["k_ring"], g["v_ring"], g["pos"],
+                           sink=g["sink"], out=o)
+    torch.cuda.synchronize()
+    assert B.swa_sink_device_error() == 2
+    assert B.swa_sink_device_error() == 0
+    d["pos"][1] = 0
+    ro, rl, _ = oracle_decode(d)
+    check(o, lse, ro, rl, "negative position read as 0")
