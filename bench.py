@@ -116,7 +116,8 @@ KERNEL_SOURCES = {
     "backward": ["backward_sm100.cuh", "prefill_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "decode": ["decode_tc_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
     "decode_fp8": ["decode_fp8_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
-    "splitkv": ["decode_splitkv_sm100.cuh", "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
+    "splitkv": ["decode_splitkv_tc_sm100.cuh", "decode_splitkv_sm100.cuh", "decode_tc_sm100.cuh",
+                "decode_sm100.cuh", "ptx_sm100.cuh", "swa_sink.cu"],
 }
 WORKLOAD_KERNEL = {"tiny_swa_prefill": "ring", "swa_prefill_32k": "ring",
                    "swa_prefill_32k_rope": "ring_rope", "global_prefill_8k_rope": "chunked_rope",

@@ -24,6 +24,7 @@
 #include "decode_sm100.cuh"
 #include "decode_tc_sm100.cuh"
 #include "decode_splitkv_sm100.cuh"
+#include "decode_splitkv_tc_sm100.cuh"
 #include "prefill_chunked_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "prefill_swa_ring_sm100.cuh"
@@ -961,11 +962,13 @@ size_t split_workspace_bytes(int B, int Hkv, int D, int W, int max_ctx) {
   return static_cast<size_t>(B) * Hkv * S * 32 * (D + 4) * sizeof(float);
 }
 
-size_t g_attr_split[2][2][kMaxDevices];
+size_t g_attr_split_tc[2][kMaxDevices];
 
-template <int D, int MT>
-int launch_split(const swa::SplitParams& p, const void* q, const void* k_new, const void* v_new,
-                 const void* k_cache, const void* v_cache, cudaStream_t st) {
+// The split-KV decode on the tcgen05 kernel: one CTA per (sequence, range, kv
+// head), those that run taking over the others' units; then the merge.
+template <int D>
+int launch_split_tc(const swa::SplitParams& p, const void* q, const void* k_new,
+                    const void* v_new, const void* k_cache, const void* v_cache, cudaStream_t st) {
   CUtensorMap tq, tkc, tvc, tkn, tvn;
   const uint32_t G = static_cast<uint32_t>(p.G), nq = static_cast<uint32_t>(p.n_q);
   if (encode_4d(&tq, q, D, p.Hq, p.n_q, p.B, 64, G, nq, 1) != SWA_OK ||
@@ -974,20 +977,22 @@ int launch_split(const swa::SplitParams& p, const void* q, const void* k_new, co
       encode_4d(&tkn, k_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK ||
       encode_4d(&tvn, v_new, D, p.Hkv, p.n_q, p.B, 64, 1, nq, 1) != SWA_OK)
     return SWA_ERR_CUDA;
-  const size_t smem = swa::split_smem_bytes(D);
-  auto kern = swa::decode_split_kernel<D, MT>;
-  if (ensure_smem_attr(kern, smem, g_attr_split[D == 128][MT - 1]) != SWA_OK) return SWA_ERR_CUDA;
+  // at least half an SM's shared memory, so that one CTA (and its 512 TMEM
+  // columns) has the SM
+  const size_t smem = std::max<size_t>(swa::split_tc_smem_bytes(D), 120 * 1024);
+  auto kern = swa::decode_split_tc_kernel<D>;
+  if (ensure_smem_attr(kern, smem, g_attr_split_tc[D == 128]) != SWA_OK) return SWA_ERR_CUDA;
   const long long units = static_cast<long long>(p.B) * p.Hkv;
-  if (units * p.S > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
-  kern<<<static_cast<unsigned>(units * p.S), swa::kSplitWarps * 32, smem, st>>>(tq, tkc, tvc, tkn,
-                                                                                 tvn, p);
+  if (units * p.S > 0x7fffffffLL || units * p.R > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  kern<<<static_cast<unsigned>(units * p.S), swa::kSplTcThreads, smem, st>>>(tq, tkc, tvc, tkn,
+                                                                               tvn, p);
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail("split-KV decode launch", e);
-  if (units * p.R > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return cuda_fail("tcgen05 split-KV decode launch", e);
   swa::decode_split_combine_kernel<D><<<static_cast<unsigned>(units * p.R), 32, 0, st>>>(p);
   e = cudaGetLastError();
   return e == cudaSuccess ? SWA_OK : cuda_fail("split-KV combine launch", e);
 }
+
 
 }  // namespace
 
@@ -1115,12 +1120,8 @@ int swa_sink_attn_decode_splitkv(const void* q, const void* k_new, const void* v
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool two = p.R > 16;
-  if (D == 64)
-    return two ? launch_split<64, 2>(p, q, k_new, v_new, k_cache, v_cache, st)
-               : launch_split<64, 1>(p, q, k_new, v_new, k_cache, v_cache, st);
-  return two ? launch_split<128, 2>(p, q, k_new, v_new, k_cache, v_cache, st)
-             : launch_split<128, 1>(p, q, k_new, v_new, k_cache, v_cache, st);
+  if (D == 64) return launch_split_tc<64>(p, q, k_new, v_new, k_cache, v_cache, st);
+  return launch_split_tc<128>(p, q, k_new, v_new, k_cache, v_cache, st);
 }
 
 int swa_sink_kv_commit(void* k_ring, void* v_ring, const void* k_new, const void* v_new,

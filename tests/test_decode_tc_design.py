@@ -231,3 +231,228 @@ def test_protocol_model_catches_mistakes(mistake, monkeypatch):
         except AssertionError:
             failed += 1
     assert failed > 0
+
+
+def model_split_tc(sim, steps, rescale, zero_v, RING=16, mistake=None):
+    """The split-KV kernel (csrc/decode_splitkv_tc_sm100.cuh): units with
+    steps[i] steps each (0: a range with no position and no new token), K of
+    step n into slot n % 3, V of step n - 2 into slot n % 2, Q per unit into
+    slot q % 2, S double-buffered, one O. Units with no step stay out of the
+    unit ring (the producer marks their state empty). rescale[n]: step n's
+    softmax rescales O (it waits for P V of step n - 1 when the unit has one);
+    zero_v[n]: it zeroes V rows of its step first (waits for V). mistake:
+    "empty in ring" (the first draft: units with no step go through the ring
+    too, and a long run of them fills it while a V load the epilogue waits for
+    is still to be issued), "q by unit" (Q slots and parities counted over
+    every unit) or "l by unit" (the row-state handoff counted likewise); the
+    last two need the first."""
+    for s in range(3):
+        sim.bar("k_full%d" % s, 1)
+        sim.bar("k_empty%d" % s, 1)
+    for s in range(2):
+        for nm, c in (("q_full", 1), ("q_empty", 1), ("v_full", 1), ("v_empty", 1),
+                      ("s_full", 1), ("s_free", 1), ("p_full", 4)):
+            sim.bar("%s%d" % (nm, s), c)
+    for nm, c in (("o_full", 1), ("o_empty", 4), ("l_full", 4), ("l_free", 4)):
+        sim.bar(nm, c)
+    for e in range(RING):
+        sim.bar("ur_full%d" % e, 1)
+        sim.bar("ur_empty%d" % e, 9)
+    in_ring = mistake in ("empty in ring", "q by unit", "l by unit")
+    units = [i for i in range(len(steps)) if in_ring or steps[i] > 0]  # ring order
+    nu = len(units)
+    st = [steps[u] for u in units]
+    first = [sum(st[:i]) for i in range(nu)]  # global index of each unit's first step
+    qidx = []
+    q = 0
+    for i in range(nu):
+        qidx.append(i if mistake == "q by unit" else q)
+        q += st[i] > 0
+
+    def read_unit(i, times=1):
+        e = i % RING
+        yield ("wait", "ur_full%d" % e, (i // RING) & 1)
+        yield ("read", [(("UR", e), ("U", i))])
+        for _ in range(times):
+            yield ("arrive", "ur_empty%d" % e)
+
+    def producer():
+        nk = nv = 0
+        for i in range(nu + 1):
+            e = i % RING
+            yield ("wait", "ur_empty%d" % e, ((i // RING) & 1) ^ 1)
+            yield ("write", [(("UR", e), ("U", i))])
+            yield ("arrive", "ur_full%d" % e)
+            if i == nu:
+                break
+            if st[i] > 0:
+                qs = qidx[i] % 2
+                yield ("wait", "q_empty%d" % qs, ((qidx[i] // 2) & 1) ^ 1)
+                yield ("tma", "q_full%d" % qs, [(("Q", qs), i)], 1)
+            for k in range(st[i]):
+                ks = nk % 3
+                yield ("wait", "k_empty%d" % ks, ((nk // 3) & 1) ^ 1)
+                yield ("tma", "k_full%d" % ks, [(("K", ks), nk)], 1)
+                nk += 1
+                if nk - 2 > nv:
+                    vs = nv & 1
+                    yield ("wait", "v_empty%d" % vs, ((nv >> 1) & 1) ^ 1)
+                    yield ("tma", "v_full%d" % vs, [(("V", vs), nv)], 1)
+                    nv += 1
+        while nv < nk:
+            vs = nv & 1
+            yield ("wait", "v_empty%d" % vs, ((nv >> 1) & 1) ^ 1)
+            yield ("tma", "v_full%d" % vs, [(("V", vs), nv)], 1)
+            nv += 1
+
+    def mma():
+        n = 0
+        units_o = 0
+        prev = None  # (step index, first of its unit, last of its unit, its unit's o index)
+
+        def pv(j, pfirst, plast, po):
+            b = j & 1
+            yield ("wait", "p_full%d" % b, (j >> 1) & 1)
+            yield ("wait", "v_full%d" % b, (j >> 1) & 1)
+            if pfirst:
+                yield ("wait", "o_empty", (po & 1) ^ 1)
+            reads = [(("S", b), ("P", j)), (("V", b), j)]
+            if zero_v[j]:
+                reads.append((("VZ", b), j))
+            if not pfirst:
+                reads.append((("O",), ("O", j - 1), "pipe"))
+            yield ("mma", reads, [(("O",), ("O", j))])
+            yield ("commit", "v_empty%d" % b)
+            yield ("commit", "s_free%d" % b)
+            if plast:
+                yield ("commit", "o_full")
+
+        for i in range(nu + 1):
+            yield from read_unit(i)
+            if i == nu:
+                break
+            qi = i if mistake == "q by unit" else units_o
+            qs = qi % 2
+            if st[i] > 0:
+                yield ("wait", "q_full%d" % qs, (qi // 2) & 1)
+            for k in range(st[i]):
+                b, ks = n & 1, n % 3
+                yield ("wait", "s_free%d" % b, ((n >> 1) & 1) ^ 1)
+                yield ("wait", "k_full%d" % ks, (n // 3) & 1)
+                yield ("mma", [(("Q", qs), i), (("K", ks), n)], [(("S", b), ("S", n))])
+                yield ("commit", "s_full%d" % b)
+                yield ("commit", "k_empty%d" % ks)
+                if k == st[i] - 1:
+                    yield ("commit", "q_empty%d" % qs)
+                if prev is not None:
+                    yield from pv(*prev)
+                po = units_o
+                if k == 0:
+                    units_o += 1
+                prev = (n, k == 0, k == st[i] - 1, po)
+                n += 1
+        if prev is not None:
+            yield from pv(*prev)
+
+    def softmax():
+        n = 0
+        handed = 0
+        for i in range(nu + 1):
+            yield from read_unit(i, 4)
+            if i == nu:
+                break
+            for k in range(st[i]):
+                b = n & 1
+                yield ("wait", "s_full%d" % b, (n >> 1) & 1)
+                yield ("read", [(("S", b), ("S", n))])
+                if rescale[n] and k > 0:
+                    pb = (n - 1) & 1
+                    yield ("wait", "s_free%d" % pb, ((n - 1) >> 1) & 1)
+                    yield ("read", [(("O",), ("O", n - 1))])
+                    yield ("write", [(("O",), ("O", n - 1))])
+                yield ("write", [(("S", b), ("P", n))])
+                if zero_v[n]:
+                    yield ("wait", "v_full%d" % b, (n >> 1) & 1)
+                    yield ("read", [(("V", b), n)])
+                    yield ("write", [(("VZ", b), n)])
+                for _ in range(4):
+                    yield ("arrive", "p_full%d" % b)
+                n += 1
+            if st[i] > 0:
+                yield ("wait", "l_free", ((i if mistake == "l by unit" else handed) & 1) ^ 1)
+                yield ("write", [(("L",), i)])
+                for _ in range(4):
+                    yield ("arrive", "l_full")
+                handed += 1
+
+    def epilogue():
+        done = 0
+        for i in range(nu + 1):
+            yield from read_unit(i, 4)
+            if i == nu:
+                break
+            if st[i] == 0:
+                continue
+            yield ("wait", "l_full", done & 1)
+            yield ("wait", "o_full", done & 1)
+            yield ("read", [(("L",), i), (("O",), ("O", first[i] + st[i] - 1))])
+            for _ in range(4):
+                yield ("arrive", "l_free")
+                yield ("arrive", "o_empty")
+            done += 1
+
+    sim.roles["producer"] = (producer(), None)
+    sim.roles["mma"] = (mma(), None)
+    sim.roles["softmax"] = (softmax(), None)
+    sim.roles["epilogue"] = (epilogue(), None)
+
+
+def _split_case(rng):
+    nu = rng.randint(1, 12)
+    steps = [rng.choice([0, 1, 1, 2, 3, 5, 14]) for _ in range(nu)]
+    if rng.random() < 0.4:  # a long run of empty ranges (short sequences)
+        at = rng.randint(0, nu)
+        steps[at:at] = [0] * rng.randint(16, 40)
+    total = sum(steps)
+    rescale = [rng.random() < 0.3 for _ in range(total)]
+    zero_v = [rng.random() < 0.3 for _ in range(total)]
+    return steps, rescale, zero_v
+
+
+def test_split_protocol_random_schedules():
+    rng = random.Random(31)
+    for i in range(200):
+        steps, rescale, zero_v = _split_case(rng)
+        s = Sim(7000 + i)
+        model_split_tc(s, steps, rescale, zero_v)
+        s.run()
+
+
+@pytest.mark.parametrize("mistake", ["empty in ring", "q by unit", "l by unit", "p_full count"])
+def test_split_protocol_model_catches_mistakes(mistake, monkeypatch):
+    """The first draft's empty units in the unit ring (a run of them fills it
+    and the producer blocks before the V load the epilogue waits for), its
+    counting over every unit (units with no step load no Q and hand over no
+    row state) and too few P arrivals fail some schedule."""
+    if mistake == "p_full count":
+        real_bar = Sim.bar
+
+        def bar(self, name, count):
+            real_bar(self, name, 1 if name.startswith("p_full") else count)
+        monkeypatch.setattr(Sim, "bar", bar)
+    failed = 0
+    rng = random.Random(6)
+    for i in range(80):
+        steps, rescale, zero_v = _split_case(rng)
+        if mistake != "p_full count" and 0 not in steps:
+            steps[rng.randrange(len(steps))] = 0
+        if mistake == "empty in ring" and i % 2 == 0:
+            steps = [3] + [0] * 20 + [2]
+            rescale, zero_v = [False] * 5, [False] * 5
+        s = Sim(300 + i)
+        model_split_tc(s, steps, rescale, zero_v, mistake=None if mistake == "p_full count" else mistake)
+        try:
+            s.run(limit=300000)
+        except AssertionError:
+            failed += 1
+    assert failed > 0
