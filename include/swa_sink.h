@@ -108,9 +108,8 @@ SWA_API int swa_sink_attn_fwd(const void *q, const void *k, const void *v,
  * The pages have no counterpart: this is an interface variant. The arguments
  * and the results (bit for bit) are those of swa_sink_attn_fwd, and like it
  * this call allocates no device memory. It is meant for callers that cannot
- * allocate: code that runs while a CUDA stream is being captured, where
- * cudaMalloc is not allowed, and serving runtimes that hand all device memory
- * to their own pool at start-up. The difference lies in the sliding-window
+ * allocate, such as serving runtimes that hand all device memory to their
+ * own pool at start-up. The difference lies in the sliding-window
  * kernel's load balancing: here the kernel runs on one CTA per SM and draws
  * its tile ranges from two counters in a static device array of the library
  * (8 slots of two 32-bit words, 64 bytes in all, held by every GPU that loads
@@ -130,8 +129,7 @@ SWA_API int swa_sink_attn_fwd(const void *q, const void *k, const void *v,
  *   looks up the array's device address (cudaGetSymbolAddress), raises the
  *   shared-memory limits of every prefill kernel it can launch (all head
  *   dims and windows) and fetches the driver's tensor-map entry point. Later
- *   calls make no set-up call; make that first call before any stream
- *   capture.
+ *   calls make no set-up call.
  * - Only the sliding-window ring kernel has a scheduler; for shapes it does
  *   not take, the call runs the same kernel as swa_sink_attn_fwd and `slot`
  *   is not used.
