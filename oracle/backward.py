@@ -82,13 +82,15 @@ def prefill_backward(q, k, v, dout, cu_seqlens, Hq, Hkv, D, window, sink=None, s
 
 
 def prefill_backward_rows(q, k, v, dout, cu_seqlens, Hq, Hkv, D, window, row_tok, row_head,
-                          key_tok, key_head, sink=None, scale=None, nthreads=None):
+                          key_tok, key_head, sink=None, scale=None, nthreads=None, forward=None):
     """The same gradients at sampled places only, for layers too large to do
     whole: dq at the (token, head) rows row_tok/row_head and dk, dv at the
     (token, kv head) keys key_tok/key_head. A row needs the keys it sees; a
     key needs the rows that see it (W tokens x G heads for a sliding window,
-    the rest of the sequence for a global layer), with their o and lse from
-    the C oracle's prefill on those rows. Returns (dq [n,D], dk [m,D], dv [m,D])."""
+    the rest of the sequence for a global layer), with their o and lse: from
+    `forward` = (o [total,Hq,D], lse [Hq,total]), the C oracle's prefill of
+    the whole layer, when it is given, else from the C oracle's prefill on
+    those rows. Returns (dq [n,D], dk [m,D], dv [m,D])."""
     Q, K, V = _f64(q), _f64(k), _f64(v)
     dO = _f64(dout)
     cu = np.asarray(cu_seqlens, dtype=np.int64)
@@ -114,8 +116,11 @@ def prefill_backward_rows(q, k, v, dout, cu_seqlens, Hq, Hkv, D, window, row_tok
     need = sorted(need)
     rt = np.array([t for t, _ in need], np.int64)
     rh = np.array([h for _, h in need], np.int32)
-    o, lse, _ = _core.prefill_rows(q, k, v, cu_seqlens, Hq, Hkv, D, window, rt, rh, sink=sink,
-                                   scale=scale, nthreads=nthreads)
+    if forward is None:
+        o, lse, _ = _core.prefill_rows(q, k, v, cu_seqlens, Hq, Hkv, D, window, rt, rh,
+                                       sink=sink, scale=scale, nthreads=nthreads)
+    else:
+        o, lse = forward[0][rt, rh], forward[1][rh, rt]
     where = {key: n for n, key in enumerate(need)}
     delta = np.einsum("nd,nd->n", dO[rt, rh], o)
 
@@ -150,3 +155,42 @@ def dsink_from_forward(o, lse, dout, sink):
     s = np.asarray(sink.detach().cpu().numpy() if hasattr(sink, "detach") else sink, np.float64)
     delta = np.einsum("thd,thd->ht", dO, o)
     return -(np.exp(s[:, None] - lse) * delta).sum(axis=1)
+
+
+def key_sums_from_forward(q, o, lse, dout, cu_seqlens, Hq, Hkv, sink=None, scale=None):
+    """The sums of dK and dV over the keys of each sequence and kv head,
+    from a forward's o [total,Hq,D] and lse [Hq,total] (fp64) alone.
+
+    Summed over the keys row i sees, dA_ij gives
+        sum_j p_ij (dO_i . v_j) - Delta_i sum_j p_ij = Delta_i - Delta_i (1 - p_sink,i)
+                                                     = Delta_i p_sink,i,
+    because sum_j p_ij v_j = o_i and the visible weights add up to 1 - p_sink,i.
+    Every key of a sequence is seen only by rows of that sequence, so over the
+    keys of sequence b and kv head g:
+        sum_j dK_j = scale sum_{h in g} sum_{i in b} Delta_ih p_sink,ih q_ih
+        sum_j dV_j = sum_{h in g} sum_{i in b} (1 - p_sink,ih) dO_ih.
+    Without a sink p_sink = 0: the dK sum is zero and the dV sum is that of dO.
+    Returns (sum_dk, sum_dv), each [num_seqs, Hkv, D]."""
+    Q = _f64(q)
+    dO = _f64(dout) if not (hasattr(dout, "dtype") and dout.dtype == np.float64) else dout
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    total, _, D = Q.shape
+    sc = (1.0 / np.sqrt(D)) if (scale is None or scale <= 0) else float(scale)
+    G = Hq // Hkv
+    if sink is None:
+        ps = np.zeros((total, Hq))
+    else:
+        s = np.asarray(sink.detach().cpu().numpy() if hasattr(sink, "detach") else sink,
+                       np.float64)
+        ps = np.exp(s[None, :] - lse.T)                      # p_sink [total, Hq]
+    delta = np.einsum("thd,thd->th", dO, o)
+    wk = (sc * delta * ps)[:, :, None] * Q                   # [total, Hq, D]
+    wv = (1.0 - ps)[:, :, None] * dO
+    n = len(cu) - 1
+    sum_dk = np.zeros((n, Hkv, D))
+    sum_dv = np.zeros((n, Hkv, D))
+    for b in range(n):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        sum_dk[b] = wk[lo:hi].sum(axis=0).reshape(Hkv, G, D).sum(axis=1)
+        sum_dv[b] = wv[lo:hi].sum(axis=0).reshape(Hkv, G, D).sum(axis=1)
+    return sum_dk, sum_dv

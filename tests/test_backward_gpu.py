@@ -2,8 +2,8 @@
 oracle (oracle/backward.py, fp64 gradients of the exact function) on the same
 seeded inputs: whole layers on small shapes (sliding windows, global layers,
 packed sequences with empty and length-1 ones, GQA groups 1..8, head dims 64
-and 128, no sink, extreme sinks), and the full SWA and global layers at
-sampled rows and keys.
+and 128, no sink, extreme sinks), and the bench's full SWA and global layers:
+sampled rows and keys, dsink, and the sums of dk and dv over every key.
 
 Tolerance, from the arithmetic: the kernels take the forward's bf16 o (in
 Delta), round P and dS to bf16 for the tensor cores and round dq, dk, dv to
@@ -21,6 +21,18 @@ Delta_i cancels too: its error scales with S_h = sum_i p_sink,i
 sum_d |dout_id o_id| (each product of Delta off by about 2^-9 of itself
 through the bf16 o, with both signs); measured at most 1.7e-4 S_h, bounded
 by 3.4e-4 S_h.
+
+The key sums. Summed over a sequence's keys, dk and dv are fixed by the
+forward (sum_j dA_ij = Delta_i p_sink,i), so the full layers are checked on
+every key that way. The error of a sum over N keys is rounding noise that
+adds up, measured against g = sqrt(sum_j g_jd^2) of the elements summed: bf16
+rounding of the outputs alone gives about 2^-9 / sqrt(3) of g per sum, and
+Delta from the bf16 o adds errors that are shared by all the keys a row sees,
+so they add up coherently over those keys. Measured on the bench's layers: at
+most 1.04e-2 g (SWA layer, dk; global layer 7.6e-3); the bound is 2e-2 g.
+One 128-key tile of a 32K-key layer lost or doubled moves each column's sum
+by about sqrt(128 / 32768) g = 0.06 g (the square root of its share of the
+summed squares), its largest of 128 columns by nearly three times that.
 """
 import numpy as np
 import pytest
@@ -38,6 +50,7 @@ pytestmark = pytest.mark.gpu
 MAX_REL = 1e-2      # largest error / largest reference magnitude
 MEAN_REL = 6e-3     # mean error / mean reference magnitude
 DSINK_REL = 3.4e-4  # dsink error / S_h
+KEYSUM_REL = 2e-2   # key-sum error / sqrt(sum over the keys of the element squared)
 
 
 def run_bwd(c, dout, sink="case"):
@@ -126,38 +139,63 @@ def test_backward_extreme_sinks(sval):
     check_dsink(ds, rs, dsink_scale(c, dout, c["sink"]), "sink=%g dsink" % sval)
 
 
-@pytest.mark.parametrize("wname", ["swa_prefill_32k", "global_prefill_8k"])
-def test_backward_full_layers_sampled(wname):
-    """The full layers at sampled places: dq at whole query groups of sampled
-    tokens, dk / dv at sampled keys (for the global layer, keys near the end
-    of the sequence, whose rows the oracle can enumerate), dsink for the SWA
-    layer from the C oracle's forward over every row."""
+def check_key_sums(got, ref, sampled, n_first, n_keys, what):
+    """got: the kernel's dk or dv of one sequence [n_keys, Hkv, D]; ref: the
+    oracle's sums over its keys [Hkv, D]; sampled: the oracle's dk or dv at the
+    sampled keys, the first n_first of the sequence and then keys drawn
+    uniformly from the rest. Each sum's error is measured against
+    sqrt(sum_j g_jd^2), the size of the rounding noise that adds up in it,
+    estimated from the samples (the first keys exactly, the rest scaled by
+    their share of the sequence)."""
+    g = got.double().sum(dim=0).cpu().numpy()
+    e2 = (sampled[:n_first] ** 2).sum() + (sampled[n_first:] ** 2).sum() * (
+        (n_keys - n_first) / max(len(sampled) - n_first, 1))
+    noise = np.sqrt(e2 / sampled.shape[1])
+    ratio = float(np.abs(g - ref).max() / noise)
+    print("%s: key-sum error / sqrt(sum_j g_j^2) max %.3g" % (what, ratio))
+    assert ratio <= KEYSUM_REL, (what, ratio)
+
+
+@pytest.mark.parametrize("wname", ["swa_backward_32k", "global_backward_8k"])
+def test_backward_full_layers(wname):
+    """The bench's two backward workloads at full size, in its launch
+    configuration, against the C oracle's forward over every row (o, lse):
+    dq at whole query groups of sampled tokens; dk / dv at the first 16 keys
+    (a global layer's largest: every later row sees them) and at keys drawn
+    across the sequence; dsink; and the sums of dk and dv over every key of
+    each kv head, which the forward fixes (sum_j dA_ij = Delta_i p_sink,i), so
+    that a tile computed twice, dropped or written to the wrong keys anywhere
+    in the launch moves a sum."""
     c = wl.make_prefill(wl.WORKLOADS[wname])
-    dout = wl.make_dout(c["q"].shape, seed=25)
+    dout = c["dout"]
     dq, dk, dv, ds = run_bwd(c, dout)
     T, Hq, Hkv, D, W = c["total"], c["Hq"], c["Hkv"], c["D"], c["window"]
+    assert len(c["seqlens"]) == 1
     G = Hq // Hkv
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t.float()).all().item()
+    o, lse, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], Hq, Hkv, D, W,
+                               sink=c["sink"])
     rng = np.random.default_rng(5)
     toks = np.unique(np.concatenate([rng.integers(0, T, 24), [0, 1, 127, T - 1]]))
     gq = rng.integers(0, Hkv, len(toks))
     rt = np.repeat(toks, G)
     rh = (np.repeat(gq * G, G) + np.tile(np.arange(G), len(toks))).astype(np.int32)
-    if W > 0:
-        kt = np.unique(np.concatenate([rng.integers(0, T, 24), [0, 63, 64, T - 1]]))
-    else:
-        kt = np.unique(np.concatenate([rng.integers(T - 300, T, 8), [T - 1]]))
+    n_first = 16
+    kt = np.concatenate([np.arange(n_first), rng.choice(np.arange(n_first, T), 24,
+                                                        replace=False)])
     kh = rng.integers(0, Hkv, len(kt))
     sq, sk, sv = ob.prefill_backward_rows(c["q"], c["k"], c["v"], dout, c["cu_seqlens"], Hq, Hkv,
-                                          D, W, rt, rh, kt, kh, sink=c["sink"])
+                                          D, W, rt, rh, kt, kh, sink=c["sink"],
+                                          forward=(o, lse))
     ti, hi = torch.from_numpy(rt).cuda(), torch.from_numpy(rh.astype(np.int64)).cuda()
     check_grad(dq[ti, hi], sq, wname + " dq")
     ki, khi = torch.from_numpy(kt).cuda(), torch.from_numpy(kh.astype(np.int64)).cuda()
     check_grad(dk[ki, khi], sk, wname + " dk")
     check_grad(dv[ki, khi], sv, wname + " dv")
-    for t in (dq, dk, dv):
-        assert torch.isfinite(t.float()).all().item()
-    if W > 0:
-        o, lse, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], Hq, Hkv, D, W,
-                                   sink=c["sink"])
-        check_dsink(ds, ob.dsink_from_forward(o, lse, dout, c["sink"]),
-                    dsink_scale_from(o, lse, dout, c["sink"]), wname + " dsink")
+    check_dsink(ds, ob.dsink_from_forward(o, lse, dout, c["sink"]),
+                dsink_scale_from(o, lse, dout, c["sink"]), wname + " dsink")
+    rk, rv = ob.key_sums_from_forward(c["q"], o, lse, dout, c["cu_seqlens"], Hq, Hkv,
+                                      sink=c["sink"])
+    check_key_sums(dk, rk[0], sk, n_first, T, wname + " dk")
+    check_key_sums(dv, rv[0], sv, n_first, T, wname + " dv")

@@ -2,8 +2,8 @@
 swa_sink_kv_commit_fp8 (through the C ABI), against the fp64 oracle over the
 dequantized ring: shapes as for the bf16 ring (n_q 1..8, rings empty / partly
 filled / full, odd W, D 64 and 128, no sink), every finite code in the ring,
-NaN codes in never-written slots, the full FP8 decode workload (a sample of
-sequences), agreement with the bf16 kernel on exactly representable rings,
+NaN codes in never-written slots, the full FP8 decode workload (every row),
+agreement with the bf16 kernel on exactly representable rings,
 and bit-exact commits (saturation, ties, subnormals)."""
 import numpy as np
 import pytest
@@ -104,14 +104,13 @@ def test_fp8_decode_nan_in_unwritten_slots():
     check(o, lse, ro, rl, "NaN in unwritten slots")
 
 
-def test_fp8_full_workload_sampled():
+def test_fp8_full_workload_all_rows():
+    """The bench's FP8-ring decode (256 sequences, 4 new tokens, ring 128,
+    Hq = 64, Hkv = 8) in its launch configuration, every row."""
     d = wl.make_decode(wl.WORKLOADS["swa_decode_mtp_fp8"])
     o, lse = run_fp8(d)
-    rows = np.random.default_rng(1).choice(d["B"], 24, replace=False)
-    rows.sort()
-    ro, rl = oracle_fp8(d, rows=rows)
-    check(o[torch.from_numpy(rows).cuda()], lse[torch.from_numpy(rows).cuda()], ro, rl,
-          "swa_decode_mtp_fp8 sample")
+    ro, rl = oracle_fp8(d)
+    check(o, lse, ro, rl, "swa_decode_mtp_fp8")
 
 
 def test_fp8_equals_bf16_kernel_on_exact_rings():

@@ -2,8 +2,9 @@
 cache: the global-attention layers) against the fp64 oracle: caches of a
 global layer (W >= the context), a ring that has wrapped (pos > W), D = 64,
 n_q = 8, caches whose unwritten slots hold NaN, agreement with
-swa_sink_attn_decode on rings both support, and the device flag when max_ctx
-understates a position. Also the NaN-slot case for swa_sink_attn_decode."""
+swa_sink_attn_decode on rings both support, the device flag when max_ctx
+understates a position, and the bench's global-layer decode at full size on
+every row. Also the NaN-slot case for swa_sink_attn_decode."""
 import numpy as np
 import pytest
 import torch
@@ -92,6 +93,23 @@ def test_ring_decode_ignores_unwritten_slots():
     assert B.swa_sink_device_error() == 0
     ro, rl, _ = oracle_decode(d)
     check(o, lse, ro, rl, "ring decode, NaN in unwritten slots")
+
+
+def test_splitkv_full_workload_all_rows():
+    """The bench's global-layer decode (16 sequences, contexts 8K to 16K over a
+    16384-slot cache, 4 new tokens, Hq = 64, Hkv = 8) in its launch
+    configuration (max_ctx = the largest context it draws), every row; then
+    the same call with the never-written slots holding NaN, which no range may
+    read."""
+    case = wl.WORKLOADS["ga_decode_16k"]
+    d = wl.make_decode(case)
+    ro, rl, _ = oracle_decode(d)
+    o, lse = run_split(d, max_ctx=case.pos_hi)
+    assert B.swa_sink_device_error() == 0
+    check(o, lse, ro, rl, "ga_decode_16k")
+    o, lse = run_split(poison_unwritten(d), max_ctx=case.pos_hi)
+    assert B.swa_sink_device_error() == 0
+    check(o, lse, ro, rl, "ga_decode_16k, NaN in unwritten slots")
 
 
 def test_splitkv_flags_pos_beyond_max_ctx():

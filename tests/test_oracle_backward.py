@@ -9,8 +9,11 @@
   dL/dscale = sum_i q_i.dq_i / scale = sum_j k_j.dk_j / scale;
 * a closed form: with q = 0 every visible weight is 1 / (n_i + e^s), so
   dv_j = sum over the rows i that see j of dO_i / (n_i + e^s);
-* the sampled-place entry and dsink from a forward's o / lse equal the full
-  backward.
+* the sampled-place entry (o and lse computed for the rows it needs, or
+  taken from a whole forward) and dsink from a forward's o / lse equal the
+  full backward;
+* the sums of dk and dv over each sequence's keys, from the forward's o and
+  lse alone (sum_j dA_ij = Delta_i p_sink,i), equal the full backward's.
 """
 import math
 
@@ -132,5 +135,35 @@ def test_sampled_entry_and_dsink_from_forward(W):
     np.testing.assert_allclose(sv, dv[kt, kh], rtol=0, atol=1e-12)
     o, lse, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], 8, 2, 16, W,
                                sink=c["sink"])
+    # the same places with o and lse taken from the whole layer's forward
+    fq, fk, fv = ob.prefill_backward_rows(c["q"], c["k"], c["v"], dout, c["cu_seqlens"], 8, 2,
+                                          16, W, rt, rh, kt, kh, sink=c["sink"],
+                                          forward=(o, lse))
+    np.testing.assert_allclose(fq, dq[rt, rh], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(fk, dk[kt, kh], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(fv, dv[kt, kh], rtol=0, atol=1e-12)
     np.testing.assert_allclose(ob.dsink_from_forward(o, lse, dout, c["sink"]), ds, rtol=0,
                                atol=1e-12)
+
+
+@pytest.mark.parametrize("W,sink", [(7, "normal"), (0, "uniform2"), (3, None)])
+def test_key_sums_from_forward_equal_the_full_backward(W, sink):
+    """The sums of dk and dv over each sequence's keys, from the forward's o
+    and lse alone, equal the full backward's; a sequence of length 1 and an
+    empty one included."""
+    seqlens = [40, 1, 0, 23]
+    c = wl.prefill_case(seqlens, 8, 2, 16, W, sigma=0.7, sink=sink, seed=10)
+    dout = torch.randn(c["q"].shape, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    s = c["sink"] if sink else None
+    _, dk, dv, _ = ob.prefill_backward(c["q"], c["k"], c["v"], dout, c["cu_seqlens"], 8, 2, 16,
+                                       W, sink=s)
+    o, lse, _ = oracle.prefill(c["q"], c["k"], c["v"], c["cu_seqlens"], 8, 2, 16, W, sink=s)
+    sk, sv = ob.key_sums_from_forward(c["q"], o, lse, dout, c["cu_seqlens"], 8, 2, sink=s)
+    cu = c["cu_seqlens"].tolist()
+    for b in range(len(seqlens)):
+        np.testing.assert_allclose(sk[b], dk[cu[b]:cu[b + 1]].sum(axis=0), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(sv[b], dv[cu[b]:cu[b + 1]].sum(axis=0), rtol=0, atol=1e-11)
+    if sink is None:
+        assert np.abs(sk).max() == 0.0
+    else:  # the identity is not trivially zero: the sink term carries it
+        assert np.abs(sk).max() > 1e-3
