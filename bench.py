@@ -255,6 +255,17 @@ def workload_config(case, wl, world, c=None):
                  "dp%d" % world, "l2": note}, **desc)
 
 
+def percentiles(values):
+    """p10, median and p90 of per-call durations (p10 and p90 by nearest rank
+    on the sorted values)."""
+    v = sorted(values)
+    n = len(v)
+
+    def rank(p):
+        return v[min(n - 1, max(0, int(math.ceil(p * n)) - 1))]
+    return {"p10": rank(0.10), "median": statistics.median(v), "p90": rank(0.90)}
+
+
 def cpu_model():
     try:
         with open("/proc/cpuinfo") as f:
@@ -658,6 +669,10 @@ def main():
         cpu = {"value": (f / e / 1e12) if is_prefill else (b / e / 1e9),
                "unit": "TFLOP/s" if is_prefill else "GB/s", "cores": threads,
                "cpu_model": cpu_model(), "kind": "oracle", "sample": desc + ", %.1f s" % e}
+        # the same oracle on one core, a smaller bounded sample
+        f, b, e, desc, _ = oracle_sample(args.workload, wl, args.cpu_seconds / 5, 1, seed=7)
+        cpu["one_core"] = {"value": (f / e / 1e12) if is_prefill else (b / e / 1e9),
+                           "unit": cpu["unit"], "cores": 1, "sample": desc + ", %.1f s" % e}
 
     def barrier():
         if world > 1:
@@ -771,6 +786,7 @@ def main():
     roof["algorithmic_flops"] = runner.flops
     roof["kernel_ms"] = kern_avg
     roof["kernel_timed_calls"] = len(kern_ms)  # calls with an event pair around them
+    roof["kernel_ms_percentiles"] = percentiles(kern_ms)
     # (a record is for the workload's own sizes, not a --seqlen variant)
     roof["traffic"] = recorded_traffic(args.workload) if args.seqlen <= 0 else None
 

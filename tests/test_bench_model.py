@@ -60,3 +60,13 @@ def test_decode_work(pos, n_q, W):
     B = len(pos)
     assert nbytes == (cached * Hkv * D * 2 * 2 + B * n_q * Hkv * D * 2 * 2
                       + B * n_q * Hq * D * 2 * 2 + B * n_q * Hq * 4 + B * 4 + Hq * 4)
+
+
+def test_percentiles():
+    # nearest rank on the sorted values: p10 of 1..20 is the 2nd, p90 the 18th
+    got = bench.percentiles(list(range(20, 0, -1)))
+    assert got == {"p10": 2, "median": 10.5, "p90": 18}
+    one = bench.percentiles([3.0])
+    assert one == {"p10": 3.0, "median": 3.0, "p90": 3.0}
+    got = bench.percentiles([5.0, 1.0, 4.0, 2.0, 3.0])
+    assert got == {"p10": 1.0, "median": 3.0, "p90": 5.0}
