@@ -24,8 +24,8 @@
 //   about a third of a CTA's cycles just to issue.) The new rows go to row
 //   roundup8(W) so that every box starts on a 1024-byte swizzle atom.
 // * The contraction has ~25 flop per HBM byte, above what CUDA-core FMAs hide,
-//   so S = Q K^T and O = P V use the tensor cores through mma.sync m16n8k16
-//   (bf16, f32 accumulate); the tiles (32 rows) are too small for tcgen05.
+//   so S = Q K^T and O = P V use the tensor cores, here through mma.sync m16n8k16
+//   (bf16, f32 accumulate); rings of <= 144 padded keys take decode_tc_sm100.cuh.
 //   ldmatrix addresses follow the swizzle.
 // * Softmax: the warps split the keys for S; row maxima and sums are
 //   reduced inside the quad that shares a row (warp shuffles), then across
