@@ -51,6 +51,11 @@ CASES = [  # (B, n_q, Hq, Hkv, D, W, sink)
     (8, 3, 16, 2, 64, 13, "uniform2"),
     (8, 1, 8, 1, 128, 1, "normal"),
     (8, 8, 16, 4, 128, 100, "normal"),
+    # either side of the tcgen05 kernel's limit of 144 padded keys: a ring of
+    # 136 slots and 8 new tokens fills it exactly (no padding rows); 137 slots
+    # take the mma.sync kernel (160 padded keys)
+    (6, 8, 16, 4, 128, 136, "normal"),
+    (6, 8, 16, 4, 128, 137, "uniform2"),
     # more units than SMs with few rows per unit
     (400, 1, 8, 8, 64, 128, "normal"),
 ]
