@@ -133,7 +133,33 @@ def test_splitkv_workspace_and_argument_errors():
     assert f(**dict(a, workspace=FAKE + 4)) == -4
     assert f(**dict(a, n_q=9)) == -3
     assert f(**dict(a, Hq=64, Hkv=6)) == -2
+    assert f(**dict(a, B=-1)) == -2
+    assert f(**dict(a, max_ctx=-1)) == -2
+    assert f(**dict(a, D=96)) == -3
+    assert f(**dict(a, Hq=64, Hkv=4)) == -3   # 4 tokens x 16 heads: 64 query rows per kv head
+    assert f(**dict(a, pos=None)) == -1
+    assert f(**dict(a, q=FAKE + 8)) == -4
+    assert f(**dict(a, pos=FAKE + 2)) == -4
+    assert f(**dict(a, lse=FAKE + 2)) == -4
+    assert f(**dict(a, sink=FAKE + 1)) == -4
     assert f(**dict(a, B=0)) == 0
+    wsf = B.swa_sink_decode_splitkv_workspace
+    for bad in (dict(B=-1), dict(n_q=0), dict(Hq=0), dict(Hkv=0), dict(W=0), dict(max_ctx=-1)):
+        args = dict(B=4, n_q=4, Hq=64, Hkv=8, D=128, W=4096, max_ctx=4000)
+        args.update(bad)
+        assert wsf(**args) == 0, bad
+
+
+def test_splitkv_workspace_of_the_global_layer_decode():
+    # 16 sequences x 8 kv heads = 128 units; about 1184 CTAs wanted, so 10
+    # ranges each; 16380 cached positions / 10 = 1638, rounded up to a whole
+    # 64-position tile: ranges of 1664, 10 of them cover 16380. Each range
+    # keeps 32 query rows of D + 4 floats (O, m, and the two sums).
+    assert B.swa_sink_decode_splitkv_workspace(16, 4, 64, 8, 128, 16384, 16380) == (
+        16 * 8 * 10 * 32 * (128 + 4) * 4)
+    # one (sequence, kv head) and a short context: one range per 64 positions
+    assert B.swa_sink_decode_splitkv_workspace(1, 1, 8, 1, 64, 4096, 200) == (
+        1 * 1 * 4 * 32 * (64 + 4) * 4)
 
 
 def test_fp8_decode_and_commit_argument_errors():
