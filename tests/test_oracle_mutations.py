@@ -9,8 +9,12 @@ fail at least one pin, so the pins would catch it in the oracle itself.
 * Backward oracle (oracle/backward.py, imported as a mutant module): Delta
   dropped from dS, dsink's sign flipped, dq without the scale, dk of a kv head
   overwritten instead of summed over its query heads, the sink left out of
-  the denominator, the window off by one. Pins: torch autograd, finite
-  differences of the C oracle, the zero-query closed form.
+  the denominator, the window off by one; in the key sums from a forward,
+  p_sink dropped from dk, dv weighted by 1 instead of 1 - p_sink, query heads
+  grouped by stride; in the sampled entry given a whole forward, o taken from
+  the wrong head. Pins: torch autograd, finite differences of the C oracle,
+  the zero-query closed form, the sampled entry and the key sums against the
+  full backward.
 * RoPE oracle (oracle/rope.py): the frequency exponent halved, the rotation's
   sign flipped, the rotate-half pairing replaced by the interleaved one. Pins:
   the complex-multiplication form, the closed forms, the invariants.
@@ -119,6 +123,10 @@ BWD_PINS = [
     ("autograd window 1", lambda: TB.test_backward_equals_autograd(*TB.CASES[3])),
     ("finite differences", lambda: TB.test_backward_finite_differences_of_the_c_oracle(6)),
     ("zero query", TB.test_backward_zero_query_closed_form),
+    ("sampled entry", lambda: TB.test_sampled_entry_and_dsink_from_forward(7)),
+    ("key sums", lambda: TB.test_key_sums_from_forward_equal_the_full_backward(7, "normal")),
+    ("key sums global", lambda: TB.test_key_sums_from_forward_equal_the_full_backward(
+        0, "uniform2")),
 ]
 
 BWD_MUTATIONS = {
@@ -130,6 +138,15 @@ BWD_MUTATIONS = {
                                                    "dk[lo:hi, g] = sc * (da.T @ q_)")],
     "sink left out of the denominator": [("den = e.sum(axis=1) + es", "den = e.sum(axis=1)")],
     "window off by one": [("vis &= j >= i - window + 1", "vis &= j >= i - window")],
+    "key sums: p_sink dropped from dk": [("wk = (sc * delta * ps)[:, :, None] * Q",
+                                          "wk = (sc * delta)[:, :, None] * Q")],
+    "key sums: dv weighted by 1, not 1 - p_sink": [("wv = (1.0 - ps)[:, :, None] * dO",
+                                                    "wv = dO")],
+    "key sums: query heads grouped by stride": [(".reshape(Hkv, G, D).sum(axis=1)",
+                                                 ".reshape(G, Hkv, D).sum(axis=0)")],
+    "sampled entry: o of the group's first head": [
+        ("o, lse = forward[0][rt, rh], forward[1][rh, rt]",
+         "o, lse = forward[0][rt, rh // G * G], forward[1][rh, rt]")],
 }
 
 
